@@ -1,0 +1,199 @@
+/*
+ * libqlora: QLoRA projection through a frozen NF4 base weight plus a rank-r
+ * LoRA adapter, forward and hand-derived backward, and the gated MLP built
+ * from three such projections.  Hand-written CUDA for sm_100a (B200).
+ *
+ * Sources (web pages on Unsloth's QLoRA kernels, cited by title + section):
+ *  - Mistral blog "用 Unsloth 微调 Mistral，速度提升 14 倍": benchmark
+ *    configuration (QLoRA nf4 on q/k/v/o/gate/up/down, rank 16, alpha 16,
+ *    dropout 0); per-optimisation table items "2. Bitsandbytes bfloat16"
+ *    (dequantise straight to bf16) and "10、11. 手动 Autograd" (hand-derived
+ *    backward, rank-r factor bracketed first).
+ *  - Gemma blog "使用 Unsloth 微调 Gemma：速度提升 2.4 倍，显存占用降低 58%",
+ *    section "GeGLU 与 Swiglu 激活函数" (gated MLP activations and their
+ *    derivatives).
+ *  - Show HN "80% faster, 50% less memory, 0% loss of accuracy Llama
+ *    finetuning": highlight 1 (manual autograd), highlight 4 (exact), and the
+ *    link to the QLoRA paper for the NF4 format.
+ *
+ * Conventions for every call
+ *  - All tensors are row-major and contiguous, in device memory owned by the
+ *    caller; every pointer must be 16-byte aligned.  bf16 values are passed as
+ *    `qlora_bf16` (their 16-bit pattern).
+ *  - Shapes follow nn.Linear: base weight W [n_out, k_in], LoRA A [k_in, r],
+ *    LoRA B [r, n_out], activations X [M, k_in], output Y [M, n_out].
+ *    The LoRA scale is s = alpha / r (passed as `scale`).
+ *  - Every call enqueues work on the caller's stream and returns without
+ *    synchronising.  The library never allocates device memory: the caller
+ *    passes a workspace of at least the size the matching *_workspace_bytes
+ *    query returns; its first 256 bytes hold the device status word and must
+ *    be zeroed by the caller once before first use.
+ *  - Invalid arguments are rejected on the host before anything is enqueued
+ *    (QLORA_ERR_INVALID_ARG, _UNSUPPORTED_SHAPE, _MISALIGNED,
+ *    _WORKSPACE_TOO_SMALL).  A failed launch returns QLORA_ERR_CUDA.  Errors
+ *    found on the device (a pipeline wait that exceeded its time limit) are
+ *    recorded in the status word and reported by qlora_last_device_status.
+ *  - M = 0 is valid and enqueues nothing.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qlora_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+typedef uint16_t qlora_bf16;                /* bf16 bit pattern */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* k_in % 256 != 0 for the GEMM paths, n_out % 8 != 0, r != 16 ... */
+  QLORA_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+  QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
+  QLORA_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  QLORA_ERR_TIMEOUT = 6,            /* a device pipeline wait exceeded its limit */
+  QLORA_ERR_DEVICE = 7              /* other device-side error flag */
+} qlora_status;
+
+typedef enum { QLORA_ACT_SWIGLU = 0, QLORA_ACT_GEGLU_TANH = 1 } qlora_act;
+
+/* NF4 weight: codes uint8 [n_out * k_in / 2] (two 4-bit level indices per
+ * byte, even element in the high nibble), absmax fp32 [n_out * k_in / 64]
+ * (one per block of 64 consecutive elements along k_in). */
+typedef struct {
+  const uint8_t* codes;
+  const float* absmax;
+  int64_t n_out;
+  int64_t k_in;
+} qlora_nf4;
+
+/* One QLoRA projection: frozen NF4 base W plus LoRA A [k_in, r], B [r, n_out]. */
+typedef struct {
+  qlora_nf4 w;
+  const qlora_bf16* A;
+  const qlora_bf16* B;
+  int32_t r;   /* must be 16 */
+  float scale; /* s = alpha / r */
+} qlora_lora_linear;
+
+/* Tensors the MLP forward saves for its backward (caller-allocated):
+ * E, G, H [M, h] (e = gate projection, g = up projection, h = act(e) * g),
+ * XA_g, XA_u [M, r] (X A_g, X A_u) and HA_d [M, r] (H A_d). */
+typedef struct {
+  qlora_bf16* E;
+  qlora_bf16* G;
+  qlora_bf16* H;
+  qlora_bf16* XA_g;
+  qlora_bf16* XA_u;
+  qlora_bf16* HA_d;
+} qlora_mlp_saved;
+
+/* The 16 NF4 levels this library uses, as binary32, ascending.  Host only;
+ * needs no GPU.  Levels: QLoRA NormalFloat construction (Show HN thread's
+ * QLoRA link), normalised to [-1, 1] with an exact 0 at index 7. */
+QLORA_API qlora_status qlora_nf4_codebook(float out[16]);
+
+/* NF4 block quantisation of a bf16 weight [n_out, k_in] (k_in % 64 == 0).
+ * absmax = max |w| per 64-block; v = w / absmax rounded to binary32; level =
+ * number of level midpoints strictly below v (ties to the lower level);
+ * all-zero blocks store level 7.  Writes codes [n_out*k_in/2] and
+ * absmax [n_out*k_in/64].  (Mistral blog benchmark configuration, QLoRA nf4.) */
+QLORA_API qlora_status nf4_quantize(const qlora_bf16* w, int64_t n_out, int64_t k_in, uint8_t* codes, float* absmax,
+                          qlora_stream_t stream);
+
+/* NF4 dequantisation straight to bf16 (Mistral blog item "2. Bitsandbytes
+ * bfloat16"): out[n, k] = RNE_bf16(level[q] * absmax) with the product in
+ * binary32.  Bit-exact.  out is [n_out, k_in]. */
+QLORA_API qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n_out, int64_t k_in, qlora_bf16* out,
+                            qlora_stream_t stream);
+
+/* Workspace bytes needed by qlora_linear_fwd and qlora_linear_bwd. */
+QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t k_in, int64_t n_out, int32_t r);
+
+/* Forward of one QLoRA projection (Mistral blog "10、11. 手动 Autograd"):
+ *   XA = X A                      -> XA_saved [M, r]  (kept for the backward)
+ *   Y  = X dequant(W)^T + s XA B  -> Y [M, n_out]
+ * X [M, k_in].  Requires k_in % 256 == 0, n_out % 8 == 0, r == 16. */
+QLORA_API qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                              qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Hand-derived backward (Mistral blog "10、11. 手动 Autograd"; Show HN
+ * highlight 1), rank-r factor bracketed first, no gradient for the frozen W:
+ *   G  = dY B^T                    [M, r]
+ *   dX = dY dequant(W) + s G A^T   -> dX [M, k_in]
+ *   dA = s X^T G                   -> dA [k_in, r]
+ *   dB = s (XA)^T dY               -> dB [r, n_out]
+ * dY [M, n_out]; XA_saved from qlora_linear_fwd. */
+QLORA_API qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                              const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Workspace bytes needed by qlora_mlp_fwd and qlora_mlp_bwd (d = model
+ * width, h = MLP width). */
+QLORA_API size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r);
+
+/* Gated MLP forward (Gemma blog "GeGLU 与 Swiglu 激活函数"):
+ *   e = X Wg^T + s_g (X A_g) B_g,  g = X Wu^T + s_u (X A_u) B_u,
+ *   h = act(e) * g,  Y = h Wd^T + s_d (h A_d) B_d,
+ * act = SiLU (QLORA_ACT_SWIGLU) or tanh-approximate GELU
+ * (QLORA_ACT_GEGLU_TANH).  gate/up: n_out = h, k_in = d; down: n_out = d,
+ * k_in = h.  X [M, d], Y [M, d]; `saved` receives E, G, H, XA_g, XA_u, HA_d.
+ * Requires d % 256 == 0, h % 256 == 0, r == 16. */
+QLORA_API qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                           const qlora_mlp_saved* saved, void* workspace, size_t workspace_bytes,
+                           qlora_stream_t stream);
+
+/* Gated MLP backward by the chain rule with closed-form act':
+ *   dH = dY Wd + s_d (dY B_d^T) A_d^T,  dE = dH * g * act'(e),  dG = dH * act(e),
+ *   dX = dE Wg + dG Wu + s_g (dE B_g^T) A_g^T + s_u (dG B_u^T) A_u^T,
+ * and the six adapter gradients dA_* [k_in, r], dB_* [r, n_out] of the three
+ * projections as in qlora_linear_bwd.  dY [M, d] -> dX [M, d]. */
+QLORA_API qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* saved,
+                           const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                           qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* workspace,
+                           size_t workspace_bytes, qlora_stream_t stream);
+
+/* Reads the device status word in `workspace` (synchronising `stream`),
+ * clears it, and maps it to a status: QLORA_OK, QLORA_ERR_TIMEOUT or
+ * QLORA_ERR_DEVICE. */
+QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+QLORA_API const char* qlora_status_string(qlora_status status);
+
+/* Selects the tensor-core tile shape of the NF4 GEMMs: 1 = one CTA per
+ * 128-row tile, 2 = a CTA pair (cta_group::2) per 256-row tile (default).
+ * Returns the previous value.  Not thread-safe. */
+QLORA_API int32_t qlora_set_cta_group(int32_t cta_group);
+
+/* Kernel tracing (host side, not thread-safe).  While enabled, every kernel
+ * launch of the library is bracketed by CUDA events on its stream. */
+typedef struct {
+  const char* name; /* static kernel name */
+  int64_t launches;
+  double total_ms;  /* summed device time between the bracketing events */
+} qlora_trace_entry;
+QLORA_API qlora_status qlora_trace_begin(void);
+/* Stops tracing, waits for the recorded events and fills up to `max_entries`
+ * per-kernel totals; returns the number of distinct kernels (or -1). */
+QLORA_API int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries);
+/* Number of kernels this library has launched since it was loaded. */
+QLORA_API uint64_t qlora_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

@@ -1,0 +1,717 @@
+// C ABI of libqlora: argument validation, TMA tensor maps, workspace layout,
+// split planning and the launch sequence of every entry point in qlora.h.
+// All device work is enqueued on the caller's stream; nothing here allocates
+// device memory or synchronises (except qlora_last_device_status and
+// qlora_trace_end, which say so).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <vector>
+
+#include "../../include/qlora.h"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace ql {
+// kernels implemented in the other translation units
+cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st);
+cudaError_t launch_nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t numel, bf16* out,
+                                  cudaStream_t st, int num_sms);
+cudaError_t launch_gemm_nf4(int mode, int epi, int cg, const GemmMaps& maps, const GemmArgs& args,
+                            cudaStream_t stream);
+cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1, float* part,
+                           int M, int K, int splits, int kb_per_split, int* status, cudaStream_t st);
+cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, float* part, int M, int N, int splits,
+                           int mb_per_split, int* status, cudaStream_t st);
+cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, float* gpart,
+                          float* qpart, int M, int N, int rc_per_cta, int* status, cudaStream_t st);
+cudaError_t launch_reduce(const float* part, int S, int rows, int R, const ReduceOuts& outs, cudaStream_t st);
+extern const uint32_t h_nf4_bits[16];
+}  // namespace ql
+
+using namespace ql;
+
+namespace {
+
+// ------------------------------------------------------------- tracing ---
+enum KernelId : int {
+  K_QUANT = 0, K_DEQUANT, K_GEMM_FWD, K_GEMM_GLU_FWD, K_GEMM_BWD, K_GEMM_GLU_BWD, K_ROWPROJ, K_COLPROJ, K_DYPASS,
+  K_REDUCE, K_COUNT
+};
+const char* const kKernelNames[K_COUNT] = {
+    "nf4_quantize", "nf4_dequantize", "gemm_nf4_fwd", "gemm_nf4_gateup_glu_fwd", "gemm_nf4_bwd_dx",
+    "gemm_nf4_down_bwd_glu", "skinny_rowproj", "skinny_colproj", "skinny_dypass", "skinny_reduce"};
+
+std::atomic<uint64_t> g_launches{0};
+bool g_trace = false;
+struct TraceRec {
+  int id;
+  cudaEvent_t a, b;
+};
+std::vector<TraceRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+size_t g_pool_used = 0;
+int32_t g_cta_group = 2;
+
+cudaEvent_t pool_event() {
+  if (g_pool_used == g_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_pool.push_back(e);
+  }
+  return g_pool[g_pool_used++];
+}
+
+struct KScope {
+  int id;
+  cudaStream_t st;
+  cudaEvent_t b = nullptr;
+  KScope(int id_, cudaStream_t st_) : id(id_), st(st_) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (g_trace) {
+      cudaEvent_t a = pool_event();
+      b = pool_event();
+      if (a && b) {
+        cudaEventRecord(a, st);
+        g_recs.push_back({id, a, b});
+      } else {
+        b = nullptr;
+      }
+    }
+  }
+  ~KScope() {
+    if (b) cudaEventRecord(b, st);
+  }
+};
+
+// ------------------------------------------------------------ helpers ---
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+// 2-D tensor map over a row-major [rows, cols] matrix with `ld` elements per row.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, int64_t cols, int64_t rows,
+              int64_t ld, int box_cols, int box_rows, CUtensorMapSwizzle swz) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool map_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t ld, int bc, int br,
+              CUtensorMapSwizzle s) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, cols, rows, ld, bc, br, s);
+}
+
+// ---------------------------------------------------------- planning ----
+constexpr int kTargetCtas = 2 * 148;
+
+struct RowPlan { int splits, kb_per; };
+RowPlan plan_rowproj(int64_t M, int64_t K) {
+  const int64_t mblocks = cdiv(M, 64), kbs = K / 64;
+  int64_t splits = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, mblocks), 1), kbs);
+  const int64_t per = cdiv(kbs, splits);
+  return {static_cast<int>(cdiv(kbs, per)), static_cast<int>(per)};
+}
+struct ColPlan { int splits, mb_per; };
+ColPlan plan_colproj(int64_t M, int64_t ncols) {
+  const int64_t nblocks = cdiv(ncols, 64), mbs = cdiv(M, 64);
+  int64_t splits = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, nblocks), 1), mbs);
+  const int64_t per = cdiv(mbs, splits);
+  return {static_cast<int>(cdiv(mbs, per)), static_cast<int>(per)};
+}
+struct DyPlan { int gsplits, qsplits, rc; };
+DyPlan plan_dypass(int64_t M, int64_t N) {
+  const int64_t gx = cdiv(N, 256), mch = cdiv(M, 64);
+  int64_t gy = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, gx), 1), mch);
+  const int64_t rc = cdiv(mch, gy);
+  return {static_cast<int>(gx), static_cast<int>(cdiv(mch, rc)), static_cast<int>(rc)};
+}
+size_t rowproj_part_bytes(int64_t M, int64_t K, int R) {
+  return static_cast<size_t>(plan_rowproj(M, K).splits) * M * R * 4;
+}
+size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
+  return static_cast<size_t>(plan_colproj(M, ncols).splits) * ncols * R * 4;
+}
+size_t dypass_part_bytes(int64_t M, int64_t N) {
+  const DyPlan p = plan_dypass(M, N);
+  return align256(static_cast<size_t>(p.gsplits) * M * 16 * 4) + static_cast<size_t>(p.qsplits) * N * 16 * 4;
+}
+
+// ------------------------------------------------------------ passes ----
+qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+// P = T V (V = one or two [K, 16] LoRA A factors) -> out[j] (bf16, optional scaled copy)
+qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, float* part,
+                          ReduceOuts outs, int* status, cudaStream_t st) {
+  CUtensorMap mt, mv0, mv1;
+  const int nv = V1 ? 2 : 1;
+  if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mv0, V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mv1, V1 ? V1 : V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
+  const RowPlan p = plan_rowproj(M, K);
+  {
+    KScope k(K_ROWPROJ, st);
+    qlora_status s = cuda_status(launch_rowproj(nv, mt, mv0, mv1, part, (int)M, (int)K, p.splits, p.kb_per, status, st));
+    if (s != QLORA_OK) return s;
+  }
+  KScope k(K_REDUCE, st);
+  return cuda_status(launch_reduce(part, p.splits, (int)M, 16 * nv, outs, st));
+}
+
+// Q = T^T U (U [M, R]) -> outs
+qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U, int R, float* part,
+                          ReduceOuts outs, int* status, cudaStream_t st) {
+  CUtensorMap mt, mu;
+  if (!map_bf16(&mt, T, ncols, M, ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mu, U, R, M, R, R, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
+  const ColPlan p = plan_colproj(M, ncols);
+  {
+    KScope k(K_COLPROJ, st);
+    qlora_status s = cuda_status(launch_colproj(R, mt, mu, part, (int)M, (int)ncols, p.splits, p.mb_per, status, st));
+    if (s != QLORA_OK) return s;
+  }
+  KScope k(K_REDUCE, st);
+  return cuda_status(launch_reduce(part, p.splits, (int)ncols, R, outs, st));
+}
+
+// G = T Bl^T ([M,16]) and Q = T^T U ([N,16]) from one read of T [M, N].
+qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, const bf16* Bl, float* part,
+                         ReduceOuts gouts, ReduceOuts qouts, int* status, cudaStream_t st) {
+  CUtensorMap mt, mu, mb;
+  if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mu, U, 16, M, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mb, Bl, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  const DyPlan p = plan_dypass(M, N);
+  float* gpart = part;
+  float* qpart = reinterpret_cast<float*>(reinterpret_cast<char*>(part) +
+                                          align256(static_cast<size_t>(p.gsplits) * M * 16 * 4));
+  {
+    KScope k(K_DYPASS, st);
+    qlora_status s = cuda_status(launch_dypass(mt, mu, mb, gpart, qpart, (int)M, (int)N, p.rc, status, st));
+    if (s != QLORA_OK) return s;
+  }
+  {
+    KScope k(K_REDUCE, st);
+    qlora_status s = cuda_status(launch_reduce(gpart, p.gsplits, (int)M, 16, gouts, st));
+    if (s != QLORA_OK) return s;
+  }
+  KScope k(K_REDUCE, st);
+  return cuda_status(launch_reduce(qpart, p.qsplits, (int)N, 16, qouts, st));
+}
+
+ReduceOut rout(bf16* p, int col0, int ld, int transpose, float scale) { return {p, col0, ld, transpose, scale}; }
+ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0.f}, ReduceOut c = {nullptr, 0, 0, 0, 0.f},
+                 ReduceOut d = {nullptr, 0, 0, 0, 0.f}) {
+  ReduceOuts o;
+  o.o[0] = a;
+  o.o[1] = b;
+  o.o[2] = c;
+  o.o[3] = d;
+  return o;
+}
+
+// NF4 weight maps for the GEMM B operand (K-major for forward, MN-major for dX).
+bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const qlora_nf4& w, bool bwd, int cg) {
+  const int64_t N = w.n_out, K = w.k_in;
+  if (!bwd) {
+    return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, 32, 128,
+                    CU_TENSOR_MAP_SWIZZLE_32B) &&
+           make_map(absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.absmax, K / 64, N, K / 64, 4, 128,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  const int rb = 128 / cg;  // bytes of codes per W row per CTA tile
+  return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, rb, 64,
+                  cg == 1 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map(absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.absmax, K / 64, N, K / 64, 4, 64,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+qlora_status check_linear(const qlora_lora_linear* lin) {
+  if (!lin || !lin->w.codes || !lin->w.absmax || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
+  if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
+  if (lin->r != 16) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (lin->w.k_in % 256 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (lin->w.k_in > (1 << 30) || lin->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->A) || misaligned(lin->B))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// Y-side GEMM launch helpers -------------------------------------------------
+qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, const bf16* XAs, bf16* Y, int* status,
+                      cudaStream_t st) {
+  const int cg = g_cta_group;
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int64_t K = lin.w.k_in, N = lin.w.n_out;
+  if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin.w, false, cg)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&maps.la[0], XAs, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&maps.lb[0], lin.B, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  maps.a[1] = maps.a[0];
+  maps.codes[1] = maps.codes[0];
+  maps.absmax[1] = maps.absmax[0];
+  maps.la[1] = maps.la[0];
+  maps.lb[1] = maps.lb[0];
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)N;
+  a.nkb0 = (int)(K / 64);
+  a.nkb1 = 0;
+  a.lora = 1;
+  a.ldo = (int)N;
+  a.D = Y;
+  a.status = status;
+  KScope k(K_GEMM_FWD, st);
+  return cuda_status(launch_gemm_nf4(MODE_FWD, EPI_STORE, cg, maps, a, st));
+}
+
+}  // namespace
+
+// =========================================================== C entry points
+extern "C" {
+
+const char* qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "QLORA_ERR_UNSUPPORTED_SHAPE";
+    case QLORA_ERR_MISALIGNED: return "QLORA_ERR_MISALIGNED";
+    case QLORA_ERR_WORKSPACE_TOO_SMALL: return "QLORA_ERR_WORKSPACE_TOO_SMALL";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+    case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT";
+    case QLORA_ERR_DEVICE: return "QLORA_ERR_DEVICE";
+  }
+  return "QLORA_UNKNOWN_STATUS";
+}
+
+qlora_status qlora_nf4_codebook(float out[16]) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < 16; ++i) std::memcpy(&out[i], &h_nf4_bits[i], 4);
+  return QLORA_OK;
+}
+
+int32_t qlora_set_cta_group(int32_t cg) {
+  const int32_t prev = g_cta_group;
+  if (cg == 1 || cg == 2) g_cta_group = cg;
+  return prev;
+}
+
+qlora_status nf4_quantize(const qlora_bf16* w, int64_t n_out, int64_t k_in, uint8_t* codes, float* absmax,
+                          qlora_stream_t stream) {
+  if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (k_in % 64) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (n_out == 0 || k_in == 0) return QLORA_OK;
+  if (!w || !codes || !absmax) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(w) || misaligned(codes) || misaligned(absmax)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  KScope k(K_QUANT, st);
+  return cuda_status(launch_nf4_quantize(reinterpret_cast<const bf16*>(w), n_out * k_in, codes, absmax, st));
+}
+
+qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n_out, int64_t k_in, qlora_bf16* out,
+                            qlora_stream_t stream) {
+  if (n_out < 0 || k_in < 0) return QLORA_ERR_INVALID_ARG;
+  if (k_in % 64) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (n_out == 0 || k_in == 0) return QLORA_OK;
+  if (!codes || !absmax || !out) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(codes) || misaligned(absmax) || misaligned(out)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  KScope k(K_DEQUANT, st);
+  return cuda_status(launch_nf4_dequantize(codes, absmax, n_out * k_in, reinterpret_cast<bf16*>(out), st, num_sms()));
+}
+
+size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
+  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
+  size_t part = rowproj_part_bytes(M, K, 16);
+  part = std::max(part, dypass_part_bytes(M, N));
+  part = std::max(part, colproj_part_bytes(M, K, 16));
+  return 256 + vec + align256(part);
+}
+
+qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                              qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_linear(lin);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !Y || !XA_saved || !ws) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t K = lin->w.k_in, N = lin->w.n_out;
+  if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  bf16* XAs = reinterpret_cast<bf16*>(w + 256);
+  float* part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
+  bf16* xa = reinterpret_cast<bf16*>(XA_saved);
+  const bool scaled = lin->scale != 1.0f;
+  if (!scaled) XAs = xa;
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
+                   routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
+  if (s != QLORA_OK) return s;
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, st);
+}
+
+qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                              const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_linear(lin);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;  // NOTE: dA, dB are left untouched when there are no rows
+  if (!X || !XA_saved || !dY || !dX || !dA || !dB || !ws) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(XA_saved) || misaligned(dY) || misaligned(dX) || misaligned(dA) ||
+      misaligned(dB) || misaligned(ws))
+    return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t K = lin->w.k_in, N = lin->w.n_out;
+  if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int cg = g_cta_group;
+  char* w = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  bf16* sG = reinterpret_cast<bf16*>(w + 256);
+  float* part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
+  const float sc = lin->scale;
+  // G = dY B^T (stored scaled: sG), dB = s (XA)^T dY
+  s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, N, reinterpret_cast<const bf16*>(XA_saved),
+                  reinterpret_cast<const bf16*>(lin->B), part, routs(rout(sG, 0, 16, 0, sc)),
+                  routs(rout(reinterpret_cast<bf16*>(dB), 0, (int)N, 1, sc)), status, st);
+  if (s != QLORA_OK) return s;
+  // dX = dY W + (s G) A^T
+  {
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!map_bf16(&maps.a[0], dY, N, M, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[0], sG, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    maps.a[1] = maps.a[0];
+    maps.codes[1] = maps.codes[0];
+    maps.absmax[1] = maps.absmax[0];
+    maps.la[1] = maps.la[0];
+    maps.lb[1] = maps.lb[0];
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = (int)M;
+    a.N = (int)K;
+    a.nkb0 = (int)cdiv(N, 64);
+    a.lora = 1;
+    a.ldo = (int)K;
+    a.D = reinterpret_cast<bf16*>(dX);
+    a.status = status;
+    KScope k(K_GEMM_BWD, st);
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, cg, maps, a, st));
+    if (s != QLORA_OK) return s;
+  }
+  // dA = X^T (s G)
+  return pass_colproj(reinterpret_cast<const bf16*>(X), M, K, sG, 16, part,
+                      routs(rout(reinterpret_cast<bf16*>(dA), 0, 16, 0, 1.f)), status, st);
+}
+
+size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
+  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
+  const size_t big = align256(static_cast<size_t>(M) * h * 2);
+  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
+  size_t part = rowproj_part_bytes(M, d, 32);
+  part = std::max(part, rowproj_part_bytes(M, h, 16));
+  part = std::max(part, dypass_part_bytes(M, d));
+  part = std::max(part, dypass_part_bytes(M, h));
+  part = std::max(part, colproj_part_bytes(M, h, 16));
+  part = std::max(part, colproj_part_bytes(M, d, 32));
+  return 256 + 2 * big + 5 * vec + align256(part);
+}
+
+namespace {
+struct MlpWs {
+  int* status;
+  bf16 *dE, *dG, *v0, *v1, *v2, *gu;  // v*: [M,16] vectors; gu: [M,32]
+  float* part;
+};
+MlpWs carve_mlp(void* ws, int64_t M, int64_t h) {
+  char* w = static_cast<char*>(ws);
+  const size_t big = align256(static_cast<size_t>(M) * h * 2);
+  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
+  MlpWs m;
+  m.status = reinterpret_cast<int*>(w);
+  size_t off = 256;
+  m.dE = reinterpret_cast<bf16*>(w + off); off += big;
+  m.dG = reinterpret_cast<bf16*>(w + off); off += big;
+  m.v0 = reinterpret_cast<bf16*>(w + off); off += vec;
+  m.v1 = reinterpret_cast<bf16*>(w + off); off += vec;
+  m.v2 = reinterpret_cast<bf16*>(w + off); off += vec;
+  m.gu = reinterpret_cast<bf16*>(w + off); off += 2 * vec;
+  m.part = reinterpret_cast<float*>(w + off);
+  return m;
+}
+qlora_status check_mlp(const qlora_lora_linear* g, const qlora_lora_linear* u, const qlora_lora_linear* d) {
+  qlora_status s;
+  if ((s = check_linear(g)) != QLORA_OK || (s = check_linear(u)) != QLORA_OK || (s = check_linear(d)) != QLORA_OK)
+    return s;
+  if (g->w.n_out != u->w.n_out || g->w.k_in != u->w.k_in || d->w.k_in != g->w.n_out || d->w.n_out != g->w.k_in)
+    return QLORA_ERR_INVALID_ARG;
+  if (g->w.n_out % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+}  // namespace
+
+qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                           const qlora_mlp_saved* sv, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
+  qlora_status s = check_mlp(gate, up, down);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !Y || !sv || !sv->E || !sv->G || !sv->H || !sv->XA_g || !sv->XA_u || !sv->HA_d || !ws)
+    return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(Y) || misaligned(sv->E) || misaligned(sv->G) || misaligned(sv->H) ||
+      misaligned(sv->XA_g) || misaligned(sv->XA_u) || misaligned(sv->HA_d) || misaligned(ws))
+    return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t d = gate->w.k_in, h = gate->w.n_out;
+  if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int cg = g_cta_group;
+  MlpWs w = carve_mlp(ws, M, h);
+  const bf16* x = reinterpret_cast<const bf16*>(X);
+  bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
+  bf16* xau = reinterpret_cast<bf16*>(sv->XA_u);
+  bf16* had = reinterpret_cast<bf16*>(sv->HA_d);
+  bf16* xags = gate->scale != 1.f ? w.v0 : xag;
+  bf16* xaus = up->scale != 1.f ? w.v1 : xau;
+  bf16* hads = down->scale != 1.f ? w.v2 : had;
+  // XA_g, XA_u = X [A_g | A_u] (one pass over X)
+  s = pass_rowproj(x, M, d, reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A), w.part,
+                   routs(rout(xag, 0, 16, 0, 1.f), rout(xau, 16, 16, 0, 1.f),
+                         rout(xags != xag ? xags : nullptr, 0, 16, 0, gate->scale),
+                         rout(xaus != xau ? xaus : nullptr, 16, 16, 0, up->scale)),
+                   w.status, st);
+  if (s != QLORA_OK) return s;
+  // gate/up GEMM with the gated activation in the epilogue -> E, G, H
+  {
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    maps.a[1] = maps.a[0];
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, false, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, false, cg)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[0], xags, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[1], xaus, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], gate->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[1], up->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = (int)M;
+    a.N = (int)h;
+    a.nkb0 = (int)(d / 64);
+    a.lora = 2;
+    a.act = act == QLORA_ACT_SWIGLU ? ACT_SILU : ACT_GELU_TANH;
+    a.ldo = (int)h;
+    a.E = reinterpret_cast<bf16*>(sv->E);
+    a.G = reinterpret_cast<bf16*>(sv->G);
+    a.H = reinterpret_cast<bf16*>(sv->H);
+    a.status = w.status;
+    KScope k(K_GEMM_GLU_FWD, st);
+    s = cuda_status(launch_gemm_nf4(MODE_FWD_GLU, EPI_GLU_FWD, cg, maps, a, st));
+    if (s != QLORA_OK) return s;
+  }
+  // HA_d = H A_d
+  s = pass_rowproj(reinterpret_cast<const bf16*>(sv->H), M, h, reinterpret_cast<const bf16*>(down->A), nullptr,
+                   w.part, routs(rout(had, 0, 16, 0, 1.f), rout(hads != had ? hads : nullptr, 0, 16, 0, down->scale)),
+                   w.status, st);
+  if (s != QLORA_OK) return s;
+  // Y = H W_d^T + (s H A_d) B_d
+  return gemm_fwd(*down, reinterpret_cast<const bf16*>(sv->H), M, hads, reinterpret_cast<bf16*>(Y), w.status, st);
+}
+
+qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
+                           const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                           qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
+                           size_t ws_bytes, qlora_stream_t stream) {
+  if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
+  qlora_status s = check_mlp(gate, up, down);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !sv || !sv->E || !sv->G || !sv->H || !sv->XA_g || !sv->XA_u || !sv->HA_d || !dY || !dX || !dA_g ||
+      !dB_g || !dA_u || !dB_u || !dA_d || !dB_d || !ws)
+    return QLORA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, sv->E, sv->G, sv->H, sv->XA_g, sv->XA_u, sv->HA_d, dY, dX, dA_g, dB_g, dA_u, dB_u, dA_d,
+                        dB_d, ws};
+  for (const void* p : ptrs)
+    if (misaligned(p)) return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t d = gate->w.k_in, h = gate->w.n_out;
+  if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int cg = g_cta_group;
+  MlpWs w = carve_mlp(ws, M, h);
+  bf16* sGd = w.v0;
+  // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
+  s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, d, reinterpret_cast<const bf16*>(sv->HA_d),
+                  reinterpret_cast<const bf16*>(down->B), w.part, routs(rout(sGd, 0, 16, 0, down->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_d), 0, (int)d, 1, down->scale)), w.status, st);
+  if (s != QLORA_OK) return s;
+  // 2. dH = dY W_d + sG_d A_d^T, with dE, dG formed in the epilogue
+  {
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!map_bf16(&maps.a[0], dY, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], down->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[0], sGd, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    maps.a[1] = maps.a[0];
+    maps.codes[1] = maps.codes[0];
+    maps.absmax[1] = maps.absmax[0];
+    maps.la[1] = maps.la[0];
+    maps.lb[1] = maps.lb[0];
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = (int)M;
+    a.N = (int)h;
+    a.nkb0 = (int)cdiv(d, 64);
+    a.lora = 1;
+    a.act = act == QLORA_ACT_SWIGLU ? ACT_SILU : ACT_GELU_TANH;
+    a.ldo = (int)h;
+    a.Ein = reinterpret_cast<const bf16*>(sv->E);
+    a.Gin = reinterpret_cast<const bf16*>(sv->G);
+    a.dE = w.dE;
+    a.dG = w.dG;
+    a.status = w.status;
+    KScope k(K_GEMM_GLU_BWD, st);
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_GLU_BWD, cg, maps, a, st));
+    if (s != QLORA_OK) return s;
+  }
+  // 3. dA_d = H^T (s_d G_d)
+  s = pass_colproj(reinterpret_cast<const bf16*>(sv->H), M, h, sGd, 16, w.part,
+                   routs(rout(reinterpret_cast<bf16*>(dA_d), 0, 16, 0, 1.f)), w.status, st);
+  if (s != QLORA_OK) return s;
+  // 4. G_g = dE B_g^T, dB_g = s_g XA_g^T dE ; G_u = dG B_u^T, dB_u = s_u XA_u^T dG
+  s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), w.part,
+                  routs(rout(w.gu, 0, 32, 0, gate->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_g), 0, (int)h, 1, gate->scale)), w.status, st);
+  if (s != QLORA_OK) return s;
+  s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), w.part,
+                  routs(rout(w.gu + 16, 0, 32, 0, up->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_u), 0, (int)h, 1, up->scale)), w.status, st);
+  if (s != QLORA_OK) return s;
+  // 5. dX = [dE | dG] [W_g ; W_u] + [sG_g | sG_u] [A_g^T ; A_u^T]
+  {
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[0], w.gu, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.la[1], w.gu + 16, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[1], up->A, 16, d, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = (int)M;
+    a.N = (int)d;
+    a.nkb0 = (int)cdiv(h, 64);
+    a.nkb1 = (int)cdiv(h, 64);
+    a.lora = 2;
+    a.ldo = (int)d;
+    a.D = reinterpret_cast<bf16*>(dX);
+    a.status = w.status;
+    KScope k(K_GEMM_BWD, st);
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, cg, maps, a, st));
+    if (s != QLORA_OK) return s;
+  }
+  // 6. [dA_g | dA_u] = X^T [sG_g | sG_u]
+  return pass_colproj(reinterpret_cast<const bf16*>(X), M, d, w.gu, 32, w.part,
+                      routs(rout(reinterpret_cast<bf16*>(dA_g), 0, 16, 0, 1.f),
+                            rout(reinterpret_cast<bf16*>(dA_u), 16, 16, 0, 1.f)),
+                      w.status, st);
+}
+
+qlora_status qlora_last_device_status(void* ws, qlora_stream_t stream) {
+  if (!ws) return QLORA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyAsync(ws, &zero, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+  if (v & QL_DEV_TIMEOUT) return QLORA_ERR_TIMEOUT;
+  return v ? QLORA_ERR_DEVICE : QLORA_OK;
+}
+
+qlora_status qlora_trace_begin(void) {
+  g_recs.clear();
+  g_pool_used = 0;
+  g_trace = true;
+  return QLORA_OK;
+}
+
+int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries) {
+  g_trace = false;
+  double tot[K_COUNT] = {0};
+  int64_t cnt[K_COUNT] = {0};
+  for (const TraceRec& r : g_recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return -1;
+    tot[r.id] += ms;
+    cnt[r.id] += 1;
+  }
+  g_recs.clear();
+  int32_t n = 0;
+  for (int i = 0; i < K_COUNT; ++i) {
+    if (!cnt[i]) continue;
+    if (out && n < max_entries) out[n] = {kKernelNames[i], cnt[i], tot[i]};
+    ++n;
+  }
+  return n;
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

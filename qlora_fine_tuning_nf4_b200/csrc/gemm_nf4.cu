@@ -1,0 +1,489 @@
+// NF4 x bf16 tensor-core GEMM for sm_100a with the frozen weight dequantised
+// into shared memory inside the mainloop, the LoRA term as extra K=16 MMAs
+// into the same TMEM accumulator, and fused gated-activation epilogues.
+//
+// What it computes (Mistral blog "用 Unsloth 微调 Mistral，速度提升 14 倍",
+// items "2. Bitsandbytes bfloat16" and "10、11. 手动 Autograd"; Gemma blog
+// section "GeGLU 与 Swiglu 激活函数"):
+//   forward   Y  = X  dequant(W)^T + (s X A) B            (MODE_FWD)
+//   gate/up   e, g as above; h = act(e) g                  (MODE_FWD_GLU)
+//   backward  dX = dY dequant(W)   + (s dY B^T) A^T        (MODE_BWD)
+//   down bwd  dH as above; dE = dH g act'(e), dG = dH act(e) (EPI_GLU_BWD)
+// The dequantised weight never exists in HBM: each CTA expands the NF4 codes
+// of its B tile straight to bf16 in shared memory.
+//
+// Structure (one output tile per CTA, or per CTA pair with cta_group::2):
+//   warp 0      TMA producer: A tiles, raw NF4 codes + absmax, LoRA operands
+//   warp 1      TMEM allocation; lane 0 of the leader CTA issues tcgen05.mma
+//   warps 2-5   epilogue: TMEM -> registers -> activation -> global
+//   warps 6-13  dequantisers: raw codes -> bf16 B tile (128B-swizzled)
+// Pipelines: raw ring (TMA -> dequantisers), operand ring (A by TMA, B by the
+// dequantisers -> MMA), one accumulator barrier (MMA -> epilogue).
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace ql {
+
+// NF4 levels (QLoRA NormalFloat construction, binary32), as bit patterns.
+__device__ __forceinline__ float nf4_level(int i) {
+  constexpr uint32_t kBits[16] = {0xbf800000u, 0xbf3239b1u, 0xbf066b2eu, 0xbeca329eu, 0xbe91a24bu, 0xbe3d353du,
+                                  0xbdba7869u, 0x00000000u, 0x3da2fb01u, 0x3e24cadfu, 0x3e7c04dau, 0x3ead0336u,
+                                  0x3ee1a4b5u, 0x3f1007a9u, 0x3f3913b0u, 0x3f800000u};
+  return __uint_as_float(kBits[i]);
+}
+
+// Per-block product table T[q] = bf16(level[q] * absmax), split into the low
+// bytes (tl) and high bytes (th) of the 16 bf16 values, 4 per register.
+QL_DEV void nf4_block_table(float absmax, uint32_t (&tl)[4], uint32_t (&th)[4]) {
+  uint32_t p[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) p[k] = pack_bf16x2(nf4_level(2 * k) * absmax, nf4_level(2 * k + 1) * absmax);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    tl[k] = prmt(p[2 * k], p[2 * k + 1], 0x6420u);
+    th[k] = prmt(p[2 * k], p[2 * k + 1], 0x7531u);
+  }
+}
+
+// Eight 4-bit codes (one 32-bit word; byte b holds element 2b in its high
+// nibble and 2b+1 in its low nibble) -> eight bf16 in element order.
+// Byte-permute lookups: the low three bits of each nibble index an 8-entry
+// half of the table; bit 3 chooses the half through a sign-replicated mask.
+QL_DEV uint4 nf4_decode8(uint32_t w, const uint32_t (&tl)[4], const uint32_t (&th)[4]) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t sel_hi = sel >> 16;
+  const uint32_t w4 = w << 4;
+  const uint32_t m_lo = prmt(w, w4, 0x9D8Cu);
+  const uint32_t m_hi = prmt(w, w4, 0xBFAEu);
+  uint4 out;
+  uint32_t L = (prmt(tl[0], tl[1], sel) & ~m_lo) | (prmt(tl[2], tl[3], sel) & m_lo);
+  uint32_t H = (prmt(th[0], th[1], sel) & ~m_lo) | (prmt(th[2], th[3], sel) & m_lo);
+  out.x = prmt(L, H, 0x4051u);
+  out.y = prmt(L, H, 0x6273u);
+  L = (prmt(tl[0], tl[1], sel_hi) & ~m_hi) | (prmt(tl[2], tl[3], sel_hi) & m_hi);
+  H = (prmt(th[0], th[1], sel_hi) & ~m_hi) | (prmt(th[2], th[3], sel_hi) & m_hi);
+  out.z = prmt(L, H, 0x4051u);
+  out.w = prmt(L, H, 0x6273u);
+  return out;
+}
+
+QL_DEV float act_f(int act, float e) {
+  if (act == ACT_SILU) return e / (1.0f + expf(-e));
+  const float t = tanhf(0.7978845608028654f * (e + 0.044715f * e * e * e));
+  return 0.5f * e * (1.0f + t);
+}
+// (act(e), act'(e))
+QL_DEV void act_fg(int act, float e, float& f, float& g) {
+  if (act == ACT_SILU) {
+    const float s = 1.0f / (1.0f + expf(-e));
+    f = e * s;
+    g = s * (1.0f + e * (1.0f - s));
+  } else {
+    const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+    const float t = tanhf(k0 * (e + k1 * e * e * e));
+    f = 0.5f * e * (1.0f + t);
+    g = 0.5f * (1.0f + t) + 0.5f * e * (1.0f - t * t) * k0 * (1.0f + 3.0f * k1 * e * e);
+  }
+}
+
+template <int MODE, int CG>
+struct GemmCfg {
+  static constexpr int BM = 128;                 // rows per CTA (TMEM lanes)
+  static constexpr int BNT = 256;                // MMA N (whole pair)
+  static constexpr int BNC = BNT / CG;           // B columns produced per CTA
+  static constexpr int BK = 64;                  // reduction block (one NF4 block, one 128B row)
+  static constexpr int NB = BNC;                 // NF4 blocks dequantised per CTA per k-block
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BNC * BK * 2;
+  static constexpr int RC_BYTES = NB * 32;
+  static constexpr int RA_BYTES = (MODE == MODE_BWD) ? 64 * 16 : BNC * 16;
+  static constexpr int S = (CG == 1) ? 3 : 5;    // operand stages
+  static constexpr int RS = (CG == 1) ? 4 : 6;   // raw stages
+  static constexpr int LA_BYTES = BM * 16 * 2;
+  static constexpr int LB_BYTES = 8192;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + S * A_BYTES;
+  static constexpr int OFF_RC = OFF_B + S * B_BYTES;
+  static constexpr int OFF_RA = OFF_RC + RS * RC_BYTES;
+  static constexpr int OFF_LA = OFF_RA + RS * RA_BYTES;
+  static constexpr int OFF_LB = OFF_LA + 2 * LA_BYTES;
+  static constexpr int OFF_BAR = OFF_LB + 2 * LB_BYTES;
+  static constexpr int NBAR = 2 * S + 2 * RS + 3;
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 14 * 32;
+  static constexpr int TMEM_COLS = 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0, "1024B alignment of swizzled regions");
+};
+
+template <int MODE, int EPI, int CG>
+__global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
+  using C = GemmCfg<MODE, CG>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+
+  // Tile coordinates: N tiles vary fastest so CTAs in flight share an A row block.
+  const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
+  const int n_tiles = (args.N + bn_out - 1) / bn_out;
+  const int pair = blockIdx.x / CG;
+  const int nt = pair % n_tiles;
+  const int mt = pair / n_tiles;
+  const int m0 = mt * (C::BM * CG) + static_cast<int>(rank) * C::BM;
+  const int n0 = nt * bn_out;
+  const int nk = args.nkb0 + args.nkb1;
+
+  // barriers
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::S + s); };
+  auto rfull_bar = [&](int s) { return bar0 + 8u * (2 * C::S + s); };
+  auto rempty_bar = [&](int s) { return bar0 + 8u * (2 * C::S + C::RS + s); };
+  const uint32_t lora_bar = bar0 + 8u * (2 * C::S + 2 * C::RS);
+  const uint32_t acc_bar = lora_bar + 8u;
+  const uint32_t drain_bar = lora_bar + 16u;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + C::NBAR * 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::S; ++s) {
+      mbar_init(full_bar(s), 1 + CG * (C::NB / 32));
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int s = 0; s < C::RS; ++s) {
+      mbar_init(rfull_bar(s), 1);
+      mbar_init(rempty_bar(s), C::NB / 32);
+    }
+    mbar_init(lora_bar, 1);
+    mbar_init(acc_bar, 1);
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc<CG>(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish<CG>();
+  }
+  tc_fence_before();
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+
+  // shared::cluster address of a barrier in the pair's leader CTA
+  auto leader = [&](uint32_t bar) { return (CG == 2) ? mapa_shared(bar, 0) : bar; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < 2; ++i) {
+        tma_prefetch_desc(&maps.a[i]);
+        tma_prefetch_desc(&maps.codes[i]);
+        tma_prefetch_desc(&maps.absmax[i]);
+      }
+      auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar_local, int x, int y) {
+        if constexpr (CG == 2) tma_load_2d_pair(dst, m, leader(bar_local), x, y);
+        else tma_load_2d(dst, m, bar_local, x, y);
+      };
+      if (args.lora > 0) {
+        int bytes = args.lora * C::LA_BYTES;
+        if (MODE == MODE_FWD) bytes += C::BNC * 32;
+        if (MODE == MODE_FWD_GLU) bytes += 2 * (128 / CG) * 32;
+        if (MODE == MODE_BWD) bytes += args.lora * C::BNC * 32;
+        if (rank == 0) mbar_arrive_expect_tx(lora_bar, bytes * CG);
+        for (int i = 0; i < args.lora; ++i) {
+          load(sbase + C::OFF_LA + i * C::LA_BYTES, &maps.la[i], lora_bar, 0, m0);
+          if (MODE == MODE_FWD) {
+            for (int c = 0; c < C::BNC / 64; ++c)
+              load(sbase + C::OFF_LB + c * 2048, &maps.lb[0], lora_bar, n0 + (int)rank * C::BNC + c * 64, 0);
+          } else if (MODE == MODE_FWD_GLU) {
+            for (int c = 0; c < (128 / CG) / 64; ++c)
+              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 2048, &maps.lb[i], lora_bar,
+                   n0 + (int)rank * (128 / CG) + c * 64, 0);
+          } else {
+            for (int c = 0; c < C::BNC / 128; ++c)
+              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 4096, &maps.lb[i], lora_bar, 0,
+                   n0 + (int)rank * C::BNC + c * 128);
+          }
+        }
+      }
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        const int seg = kb >= args.nkb0 ? 1 : 0;
+        const int kl = kb - seg * args.nkb0;
+        // raw NF4 codes + absmax for the dequantisers (local barrier)
+        const int rs = kb % C::RS;
+        ok = mbar_wait(rempty_bar(rs), ((kb / C::RS) & 1) ^ 1, args.status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(rfull_bar(rs), C::RC_BYTES + C::RA_BYTES);
+        const uint32_t rc = sbase + C::OFF_RC + rs * C::RC_BYTES;
+        const uint32_t ra = sbase + C::OFF_RA + rs * C::RA_BYTES;
+        if (MODE == MODE_BWD) {
+          const int kw0 = n0 + (int)rank * C::BNC;
+          tma_load_2d(rc, &maps.codes[seg], rfull_bar(rs), kw0 / 2, kl * 64);
+          tma_load_2d(ra, &maps.absmax[seg], rfull_bar(rs), (kw0 / 64) & ~3, kl * 64);
+        } else {
+          for (int h = 0; h < C::BNC / 128; ++h) {
+            int src = 0, row = n0 + (int)rank * C::BNC + h * 128;
+            if (MODE == MODE_FWD_GLU) {
+              src = (CG == 1) ? h : (int)rank;
+              row = n0;
+            }
+            tma_load_2d(rc + h * 4096, &maps.codes[src], rfull_bar(rs), kl * 32, row);
+            tma_load_2d(ra + h * 2048, &maps.absmax[src], rfull_bar(rs), kl & ~3, row);
+          }
+        }
+        // A operand tile (completes on the leader's full barrier)
+        const int s = kb % C::S;
+        ok = mbar_wait(empty_bar(s), ((kb / C::S) & 1) ^ 1, args.status);
+        if (!ok) break;
+        if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
+        load(sbase + C::OFF_A + s * C::A_BYTES, &maps.a[seg], full_bar(s), kl * 64, m0);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA -----
+    if (rank == 0 && lane == 0) {
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16(C::BM * CG, C::BNT, false, MODE == MODE_BWD);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::S;
+        ok = mbar_wait<CG == 2>(full_bar(s), (kb / C::S) & 1, args.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a = sbase + C::OFF_A + s * C::A_BYTES;
+        const uint32_t b = sbase + C::OFF_B + s * C::B_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, QL_SWZ_128B);
+          const uint64_t bd = (MODE == MODE_BWD) ? smem_desc(b + kk * 2048, 8192, 1024, QL_SWZ_128B)
+                                                 : smem_desc(b + kk * 32, 16, 1024, QL_SWZ_128B);
+          umma_bf16<CG>(tmem, ad, bd, idesc, (kb | kk) != 0);
+        }
+        umma_commit<CG>(empty_bar(s));
+      }
+      if (ok && args.lora > 0) {
+        ok = mbar_wait<CG == 2>(lora_bar, 0, args.status);
+        if (ok) {
+          tc_fence_after();
+          for (int i = 0; i < args.lora; ++i) {
+            const uint64_t ad = smem_desc(sbase + C::OFF_LA + i * C::LA_BYTES, 16, 256, QL_SWZ_32B);
+            if (MODE == MODE_FWD) {
+              const uint64_t bd = smem_desc(sbase + C::OFF_LB, 2048, 1024, QL_SWZ_128B);
+              umma_bf16<CG>(tmem, ad, bd, idesc_bf16(C::BM * CG, 256, false, true), 1);
+            } else if (MODE == MODE_FWD_GLU) {
+              const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 2048, 1024, QL_SWZ_128B);
+              umma_bf16<CG>(tmem + i * 128, ad, bd, idesc_bf16(C::BM * CG, 128, false, true), 1);
+            } else {
+              const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 16, 256, QL_SWZ_32B);
+              umma_bf16<CG>(tmem, ad, bd, idesc_bf16(C::BM * CG, 256, false, false), 1);
+            }
+          }
+        }
+      }
+      if (ok) {
+        umma_commit<CG>(acc_bar);
+      } else {
+        umma_commit<CG>(drain_bar);  // let issued MMAs finish before TMEM is released
+        mbar_wait(drain_bar, 0, args.status);
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------ epilogue -----
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;
+    const int grow = m0 + row;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, args.status));
+    tc_fence_after();
+    if (ok) {
+      const uint32_t trow = tmem + (static_cast<uint32_t>(lg * 32) << 16);
+      const bool row_ok = grow < args.M;
+      const size_t rbase = static_cast<size_t>(grow) * args.ldo;
+      if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          float v[32];
+          tmem_ld_32x32b_x32(trow + c * 32, v);
+          if (!row_ok) continue;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = n0 + c * 32 + q * 8;
+            if (col >= args.N) break;
+            uint4 o0, o1;
+            if (EPI == EPI_STORE) {
+              o0.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              o0.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              o0.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              o0.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              *reinterpret_cast<uint4*>(args.D + rbase + col) = o0;
+            } else {
+              const uint4 ev = *reinterpret_cast<const uint4*>(args.Ein + rbase + col);
+              const uint4 gv = *reinterpret_cast<const uint4*>(args.Gin + rbase + col);
+              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              uint32_t de[4], dg[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float f0, d0, f1, d1;
+                const float e0 = bf16_lo(ew[j]), e1 = bf16_hi(ew[j]);
+                const float g0 = bf16_lo(gw[j]), g1 = bf16_hi(gw[j]);
+                act_fg(args.act, e0, f0, d0);
+                act_fg(args.act, e1, f1, d1);
+                const float h0 = v[q * 8 + 2 * j], h1 = v[q * 8 + 2 * j + 1];
+                de[j] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
+                dg[j] = pack_bf16x2(h0 * f0, h1 * f1);
+              }
+              o0 = make_uint4(de[0], de[1], de[2], de[3]);
+              o1 = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              *reinterpret_cast<uint4*>(args.dE + rbase + col) = o0;
+              *reinterpret_cast<uint4*>(args.dG + rbase + col) = o1;
+            }
+          }
+        }
+      } else {  // EPI_GLU_FWD: columns [0,128) hold e, [128,256) hold g
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float e[32], g[32];
+          tmem_ld_32x32b_x32(trow + c * 32, e);
+          tmem_ld_32x32b_x32(trow + 128 + c * 32, g);
+          if (!row_ok) continue;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = n0 + c * 32 + q * 8;
+            if (col >= args.N) break;
+            uint32_t ew[4], gw[4], hw[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float e0 = e[q * 8 + 2 * j], e1 = e[q * 8 + 2 * j + 1];
+              const float g0 = g[q * 8 + 2 * j], g1 = g[q * 8 + 2 * j + 1];
+              ew[j] = pack_bf16x2(e0, e1);
+              gw[j] = pack_bf16x2(g0, g1);
+              hw[j] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
+            }
+            *reinterpret_cast<uint4*>(args.E + rbase + col) = make_uint4(ew[0], ew[1], ew[2], ew[3]);
+            *reinterpret_cast<uint4*>(args.G + rbase + col) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+            *reinterpret_cast<uint4*>(args.H + rbase + col) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          }
+        }
+      }
+    }
+  } else {
+    // --------------------------------------------------- dequantisers ----
+    const int dq = (warp - 6) * 32 + lane;  // 0..255
+    constexpr int groups = 256 / C::NB;
+    const int grp = dq / C::NB;
+    const int t = dq % C::NB;
+    for (int kb = grp; kb < nk; kb += groups) {
+      const int seg = kb >= args.nkb0 ? 1 : 0;
+      const int kl = kb - seg * args.nkb0;
+      const int rs = kb % C::RS;
+      if (!__all_sync(0xffffffffu, mbar_wait(rfull_bar(rs), (kb / C::RS) & 1, args.status))) break;
+      const uint8_t* rc = sgen + C::OFF_RC + rs * C::RC_BYTES;
+      const float* ra = reinterpret_cast<const float*>(sgen + C::OFF_RA + rs * C::RA_BYTES);
+      uint4 w0, w1;
+      float amax;
+      int r = 0, cchunk = 0;
+      if (MODE == MODE_BWD) {
+        // raw tile: 64 rows x (BNC/2) bytes, swizzled 128B (CG=1) or 64B (CG=2)
+        r = t & 63;
+        cchunk = t >> 6;
+        constexpr int RB = C::BNC / 2;
+        constexpr int SHIFT = (RB == 128) ? 0 : 1;
+        constexpr int MASK = (RB == 128) ? 7 : 3;
+        const int x = (r >> SHIFT) & MASK;
+        w0 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk) ^ x) << 4));
+        w1 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk + 1) ^ x) << 4));
+        amax = ra[r * 4 + cchunk + (CG == 2 ? 2 * (int)rank : 0)];
+      } else {
+        // raw tile: NB rows x 32 bytes, 32B swizzle
+        r = t;
+        const int x = (r >> 2) & 1;
+        w0 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((0 ^ x) << 4));
+        w1 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((1 ^ x) << 4));
+        amax = ra[r * 4 + (kl & 3)];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rempty_bar(rs));
+
+      const int s = kb % C::S;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((kb / C::S) & 1) ^ 1, args.status))) break;
+      uint32_t tl[4], th[4];
+      nf4_block_table(amax, tl, th);
+      uint8_t* bt = sgen + C::OFF_B + s * C::B_BYTES;
+      uint8_t* dst = (MODE == MODE_BWD) ? bt + cchunk * 8192 + (r >> 3) * 1024 + (r & 7) * 128
+                                        : bt + (r >> 3) * 1024 + (r & 7) * 128;
+      const int x7 = r & 7;
+      const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(dst + ((j ^ x7) << 4)) = nf4_decode8(wv[j], tl, th);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(leader(full_bar(s)));
+        else mbar_arrive(full_bar(s));
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown --
+  tc_fence_before();
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<CG>(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- launch --
+template <int MODE, int EPI, int CG>
+static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaStream_t stream) {
+  using C = GemmCfg<MODE, CG>;
+  auto kern = gemm_nf4_kernel<MODE, EPI, CG>;
+  static bool configured = false;  // per instantiation; attribute set once per process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
+  const int n_tiles = (args.N + bn_out - 1) / bn_out;
+  const int m_tiles = (args.M + C::BM * CG - 1) / (C::BM * CG);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * n_tiles * CG), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, maps, args);
+}
+
+cudaError_t launch_gemm_nf4(int mode, int epi, int cg, const GemmMaps& maps, const GemmArgs& args,
+                            cudaStream_t stream) {
+#define QL_CASE(M_, E_, C_) \
+  if (mode == M_ && epi == E_ && cg == C_) return launch_one<M_, E_, C_>(maps, args, stream);
+  QL_CASE(MODE_FWD, EPI_STORE, 1)
+  QL_CASE(MODE_FWD, EPI_STORE, 2)
+  QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD, 1)
+  QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD, 2)
+  QL_CASE(MODE_BWD, EPI_STORE, 1)
+  QL_CASE(MODE_BWD, EPI_STORE, 2)
+  QL_CASE(MODE_BWD, EPI_GLU_BWD, 1)
+  QL_CASE(MODE_BWD, EPI_GLU_BWD, 2)
+#undef QL_CASE
+  return cudaErrorInvalidValue;
+}
+
+int gemm_nf4_smem_bytes(int mode, int cg) {
+  if (mode == MODE_BWD) return cg == 1 ? GemmCfg<MODE_BWD, 1>::SMEM_BYTES : GemmCfg<MODE_BWD, 2>::SMEM_BYTES;
+  return cg == 1 ? GemmCfg<MODE_FWD, 1>::SMEM_BYTES : GemmCfg<MODE_FWD, 2>::SMEM_BYTES;
+}
+
+}  // namespace ql

@@ -1,0 +1,74 @@
+// Kernel-side argument structs and launch helpers shared by the .cu files of
+// libqlora.  Host code fills these; kernels only read them.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ql {
+
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ GEMM ---
+// D = A * op(dequant(W)) + LoRA, on tcgen05 tensor cores.
+//   MODE_FWD:     reduction over k_in, W [N, K] is the K-major B operand.
+//   MODE_FWD_GLU: as MODE_FWD with two weights (gate | up) side by side in
+//                 one 256-wide N tile; epilogue forms the gated activation.
+//   MODE_BWD:     reduction over n_out, W [N, K] is the MN-major B operand
+//                 (dX = dY W); up to two reduction segments (concatenated K).
+enum GemmMode : int { MODE_FWD = 0, MODE_FWD_GLU = 1, MODE_BWD = 2 };
+enum GemmEpi : int { EPI_STORE = 0, EPI_GLU_FWD = 1, EPI_GLU_BWD = 2 };
+enum Act : int { ACT_SILU = 0, ACT_GELU_TANH = 1 };
+
+struct GemmMaps {
+  CUtensorMap a[2];       // A operand per segment: bf16 [M, Kseg], box {64,128}, 128B swizzle
+  CUtensorMap codes[2];   // NF4 codes (per segment, or gate/up half for MODE_FWD_GLU)
+  CUtensorMap absmax[2];  // fp32 absmax, matching codes[]
+  CUtensorMap la[2];      // LoRA left operand(s): bf16 [M, 16], box {16,128}, 32B swizzle
+  CUtensorMap lb[2];      // LoRA right operand(s)
+};
+
+struct GemmArgs {
+  int M;        // rows of A and of the output
+  int N;        // output columns (MODE_FWD_GLU: h, the width of E/G/H)
+  int nkb0;     // 64-wide reduction blocks in segment 0
+  int nkb1;     // ... in segment 1 (0 if one segment)
+  int lora;     // number of LoRA MMAs (0, 1 or 2)
+  int act;      // Act
+  int ldo;      // leading dimension (elements) of all outputs / epilogue inputs
+  bf16* D;      // EPI_STORE output [M, N]
+  bf16* E;      // EPI_GLU_FWD outputs [M, N]: e, g and h = act(e) * g
+  bf16* G;
+  bf16* H;
+  const bf16* Ein;  // EPI_GLU_BWD inputs: saved e and g
+  const bf16* Gin;
+  bf16* dE;     // EPI_GLU_BWD outputs
+  bf16* dG;
+  int* status;  // device status word (timeouts)
+};
+
+// --------------------------------------------------------------- skinny ---
+// Rank-r products on warp-level mma.sync, split into fp32 partials that a
+// reduction kernel sums in a fixed order (deterministic).
+struct SkinnyMaps {
+  CUtensorMap t;   // main operand T: bf16 [rows, cols], box {64, 64}, 128B swizzle
+  CUtensorMap u;   // row-side factor U: bf16 [rows, R], box {R, 64}
+  CUtensorMap v;   // column-side factor: A-like [cols, R] box {R,64} or B-like [R, cols] box {64,R}
+};
+
+// Output of the partial-sum reduction: 16 of the R partial columns, scaled,
+// rounded to bf16 and written row-major or transposed.
+struct ReduceOut {
+  bf16* ptr;      // destination (nullptr = unused)
+  int col0;       // first of the 16 partial columns this output takes
+  int ld;         // row stride of the destination (elements)
+  int transpose;  // 0: dst[row * ld + c], 1: dst[c * ld + row]
+  float scale;
+};
+struct ReduceOuts {
+  ReduceOut o[4];
+};
+
+}  // namespace ql

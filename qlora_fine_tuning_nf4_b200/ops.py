@@ -1,0 +1,290 @@
+"""ctypes binding of libqlora (include/qlora.h), with the same entry-point names.
+
+Argument marshalling only: tensors are PyTorch CUDA tensors (device memory and
+streams), their data pointers and the current stream are passed to the C ABI,
+and every step of the computation runs in the library's CUDA kernels.  There
+is no CPU fallback: if ``lib/libqlora.so`` is missing, every call raises.
+"""
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libqlora.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
+
+QLORA_OK = 0
+QLORA_ACT = {"swiglu": 0, "geglu_tanh": 1}
+STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE",
+                3: "QLORA_ERR_MISALIGNED", 4: "QLORA_ERR_WORKSPACE_TOO_SMALL", 5: "QLORA_ERR_CUDA",
+                6: "QLORA_ERR_TIMEOUT", 7: "QLORA_ERR_DEVICE"}
+
+
+class QloraNF4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64)]
+
+
+class QloraLoraLinear(ctypes.Structure):
+    _fields_ = [("w", QloraNF4), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("r", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class QloraMlpSaved(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("E", "G", "H", "XA_g", "XA_u", "HA_d")]
+
+
+class QloraTraceEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
+
+
+class QloraError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+_SIGS = {
+    "qlora_nf4_codebook": (ctypes.c_int, [ctypes.c_void_p]),
+    "nf4_quantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p]),
+    "nf4_dequantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_linear_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                       ctypes.c_int32]),
+    "qlora_linear_fwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
+    "qlora_linear_bwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_mlp_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                    ctypes.c_int32]),
+    "qlora_mlp_fwd": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear),
+                                     ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
+                                     ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                     ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.c_void_p]),
+    "qlora_mlp_bwd": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear),
+                                     ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
+                                     ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
+                                     ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_last_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_set_cta_group": (ctypes.c_int32, [ctypes.c_int32]),
+    "qlora_trace_begin": (ctypes.c_int, []),
+    "qlora_trace_end": (ctypes.c_int32, [ctypes.POINTER(QloraTraceEntry), ctypes.c_int32]),
+    "qlora_launch_count": (ctypes.c_uint64, []),
+}
+
+
+def lib():
+    """Load libqlora.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m qlora_fine_tuning_nf4_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn, status):
+    if status != QLORA_OK:
+        raise QloraError(fn, status)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _p(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dev(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return t
+
+
+# ------------------------------------------------------------------ NF4 ----
+
+@dataclass
+class NF4Weight:
+    codes: torch.Tensor   # uint8 [n_out * k_in / 2]
+    absmax: torch.Tensor  # float32 [n_out * k_in / 64]
+    n_out: int
+    k_in: int
+
+    def c(self):
+        return QloraNF4(self.codes.data_ptr(), self.absmax.data_ptr(), self.n_out, self.k_in)
+
+
+def qlora_nf4_codebook():
+    out = (ctypes.c_float * 16)()
+    _check("qlora_nf4_codebook", lib().qlora_nf4_codebook(out))
+    return [float(v) for v in out]
+
+
+def nf4_quantize(w):
+    """bf16 weight [n_out, k_in] on the GPU -> NF4Weight."""
+    _dev(w, "w")
+    n_out, k_in = w.shape
+    codes = torch.empty(n_out * k_in // 2, dtype=torch.uint8, device=w.device)
+    absmax = torch.empty(n_out * k_in // 64, dtype=torch.float32, device=w.device)
+    _check("nf4_quantize", lib().nf4_quantize(_p(w), n_out, k_in, _p(codes), _p(absmax), _stream()))
+    return NF4Weight(codes, absmax, n_out, k_in)
+
+
+def nf4_dequantize(w: NF4Weight, out=None):
+    """NF4Weight -> bf16 [n_out, k_in] (bit-exact)."""
+    if out is None:
+        out = torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    _check("nf4_dequantize", lib().nf4_dequantize(_p(w.codes), _p(w.absmax), w.n_out, w.k_in, _p(out), _stream()))
+    return out
+
+
+# ---------------------------------------------------------- projections ----
+
+@dataclass
+class LoraLinear:
+    w: NF4Weight
+    A: torch.Tensor  # bf16 [k_in, r]
+    B: torch.Tensor  # bf16 [r, n_out]
+    scale: float
+
+    def c(self):
+        return QloraLoraLinear(self.w.c(), self.A.data_ptr(), self.B.data_ptr(), self.A.shape[1], self.scale)
+
+
+class Workspace:
+    """Caller-owned device workspace (zeroed once; grows on demand)."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    def get(self, nbytes):
+        if self.buf.numel() < nbytes:
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def qlora_linear_workspace_bytes(M, K, N, r=16):
+    return int(lib().qlora_linear_workspace_bytes(M, K, N, r))
+
+
+def qlora_mlp_workspace_bytes(M, d, h, r=16):
+    return int(lib().qlora_mlp_workspace_bytes(M, d, h, r))
+
+
+def qlora_linear_fwd(lin: LoraLinear, X, ws: Workspace, Y=None, XA=None):
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, lin.w.n_out, dtype=torch.bfloat16, device=X.device)
+    if XA is None:
+        XA = torch.empty(M, lin.A.shape[1], dtype=torch.bfloat16, device=X.device)
+    nb = qlora_linear_workspace_bytes(M, lin.w.k_in, lin.w.n_out, lin.A.shape[1])
+    buf = ws.get(nb)
+    c = lin.c()
+    _check("qlora_linear_fwd", lib().qlora_linear_fwd(ctypes.byref(c), _p(X), M, _p(Y), _p(XA), _p(buf),
+                                                      buf.numel(), _stream()))
+    return Y, XA
+
+
+def qlora_linear_bwd(lin: LoraLinear, X, XA, dY, ws: Workspace, dX=None, dA=None, dB=None):
+    M = X.shape[0]
+    dev = X.device
+    if dX is None:
+        dX = torch.empty(M, lin.w.k_in, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty_like(lin.A)
+    if dB is None:
+        dB = torch.empty_like(lin.B)
+    nb = qlora_linear_workspace_bytes(M, lin.w.k_in, lin.w.n_out, lin.A.shape[1])
+    buf = ws.get(nb)
+    c = lin.c()
+    _check("qlora_linear_bwd", lib().qlora_linear_bwd(ctypes.byref(c), _p(X), _p(XA), _p(dY), M, _p(dX), _p(dA),
+                                                      _p(dB), _p(buf), buf.numel(), _stream()))
+    return dX, dA, dB
+
+
+def make_mlp_saved(M, h, r, device):
+    e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device=device)
+    return {"E": e(M, h), "G": e(M, h), "H": e(M, h), "XA_g": e(M, r), "XA_u": e(M, r), "HA_d": e(M, r)}
+
+
+def _saved_c(sv):
+    return QloraMlpSaved(*[sv[k].data_ptr() for k in ("E", "G", "H", "XA_g", "XA_u", "HA_d")])
+
+
+def qlora_mlp_fwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, ws: Workspace, Y=None, saved=None):
+    M, d = X.shape
+    h = gate.w.n_out
+    r = gate.A.shape[1]
+    if Y is None:
+        Y = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
+    if saved is None:
+        saved = make_mlp_saved(M, h, r, X.device)
+    buf = ws.get(qlora_mlp_workspace_bytes(M, d, h, r))
+    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
+    _check("qlora_mlp_fwd", lib().qlora_mlp_fwd(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn),
+                                                _p(X), M, _p(Y), ctypes.byref(sv), _p(buf), buf.numel(), _stream()))
+    return Y, saved
+
+
+def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, dY, ws: Workspace, grads=None):
+    M, d = X.shape
+    h = gate.w.n_out
+    if grads is None:
+        grads = {"dX": torch.empty(M, d, dtype=torch.bfloat16, device=X.device),
+                 "dA_g": torch.empty_like(gate.A), "dB_g": torch.empty_like(gate.B),
+                 "dA_u": torch.empty_like(up.A), "dB_u": torch.empty_like(up.B),
+                 "dA_d": torch.empty_like(down.A), "dB_d": torch.empty_like(down.B)}
+    buf = ws.get(qlora_mlp_workspace_bytes(M, d, h, gate.A.shape[1]))
+    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
+    outs = [_p(grads[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
+    _check("qlora_mlp_bwd", lib().qlora_mlp_bwd(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn),
+                                                _p(X), ctypes.byref(sv), _p(dY), M, *outs, _p(buf), buf.numel(),
+                                                _stream()))
+    return grads
+
+
+# ------------------------------------------------------------ utilities ----
+
+def qlora_last_device_status(ws: Workspace):
+    return int(lib().qlora_last_device_status(_p(ws.buf), _stream()))
+
+
+def qlora_status_string(status):
+    return lib().qlora_status_string(status).decode()
+
+
+def qlora_set_cta_group(cg):
+    return int(lib().qlora_set_cta_group(cg))
+
+
+def qlora_launch_count():
+    return int(lib().qlora_launch_count())
+
+
+def qlora_trace_begin():
+    _check("qlora_trace_begin", lib().qlora_trace_begin())
+
+
+def qlora_trace_end(max_entries=64):
+    arr = (QloraTraceEntry * max_entries)()
+    n = int(lib().qlora_trace_end(arr, max_entries))
+    if n < 0:
+        raise QloraError("qlora_trace_end", 5)
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(min(n, max_entries))}

@@ -1,0 +1,116 @@
+"""Shared helpers for the GPU parity tests: run a problem through the CUDA path
+(via the C ABI binding) and through the fp64 oracle, and compare.
+
+Inputs come from the seeded generators in ``qlora_fine_tuning_nf4_b200.synth``;
+each side quantises the base weights with its own NF4 implementation, and the
+tests assert that the two quantisations are bit-identical.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+from oracle.nf4 import nf4_dequantize_f64
+from qlora_fine_tuning_nf4_b200 import ops
+from qlora_fine_tuning_nf4_b200.synth import bits_to_torch
+
+TOL = 2e-2  # max |gpu - oracle| <= TOL * RMS(oracle), per tensor
+
+
+def f64(bits):
+    return oracle.bf16_bits_to_f64(bits)
+
+
+def gpu_f64(t):
+    return t.float().cpu().double().numpy()
+
+
+def rel_err(gpu, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    err = float(np.max(np.abs(np.asarray(gpu, dtype=np.float64) - ref))) if ref.size else 0.0
+    return err, rms
+
+
+def assert_close(name, gpu, ref, tol=TOL):
+    err, rms = rel_err(gpu, ref)
+    assert err <= tol * rms, f"{name}: max|err| {err:.3e} > {tol} * RMS {rms:.3e} (ratio {err / max(rms, 1e-300):.3e})"
+    return err / max(rms, 1e-300)
+
+
+def dev(bits):
+    return bits_to_torch(bits, "cuda")
+
+
+def gpu_weight(w_bits):
+    """Quantise on the GPU; returns (NF4Weight, codes np, absmax np)."""
+    n, k = w_bits.shape
+    w = ops.nf4_quantize(dev(w_bits))
+    return w, w.codes.cpu().numpy(), w.absmax.cpu().numpy()
+
+
+def oracle_weight(w_bits):
+    n, k = w_bits.shape
+    codes, absmax = oracle.nf4_quantize(w_bits, n, k)
+    return codes, absmax, nf4_dequantize_f64(codes, absmax, n, k)
+
+
+def run_linear_gpu(p, cg=2, ws=None):
+    ops.qlora_set_cta_group(cg)
+    w, codes, absmax = gpu_weight(p["W"])
+    lin = ops.LoraLinear(w, dev(p["A"]), dev(p["B"]), p["s"])
+    ws = ws or ops.Workspace()
+    X, dY = dev(p["X"]), dev(p["dY"])
+    Y, XA = ops.qlora_linear_fwd(lin, X, ws)
+    dX, dA, dB = ops.qlora_linear_bwd(lin, X, XA, dY, ws)
+    torch.cuda.synchronize()
+    st = ops.qlora_last_device_status(ws)
+    return {"Y": gpu_f64(Y), "XA": gpu_f64(XA), "dX": gpu_f64(dX), "dA": gpu_f64(dA), "dB": gpu_f64(dB),
+            "codes": codes, "absmax": absmax, "status": st}
+
+
+def run_linear_oracle(p):
+    codes, absmax, W = oracle_weight(p["W"])
+    X, A, B, dY = f64(p["X"]), f64(p["A"]), f64(p["B"]), f64(p["dY"])
+    Y, XA = oracle.linear_fwd(X, W, A, B, p["s"])
+    dX, dA, dB = oracle.linear_bwd(X, W, A, B, p["s"], dY)
+    return {"Y": Y, "XA": XA, "dX": dX, "dA": dA, "dB": dB, "codes": codes, "absmax": absmax}
+
+
+def run_mlp_gpu(p, act, cg=2, ws=None):
+    ops.qlora_set_cta_group(cg)
+    lins = {}
+    qs = {}
+    for k in ("g", "u", "d"):
+        w, c, a = gpu_weight(p["W_" + k])
+        lins[k] = ops.LoraLinear(w, dev(p["A_" + k]), dev(p["B_" + k]), p["s"])
+        qs[k] = (c, a)
+    ws = ws or ops.Workspace()
+    X, dY = dev(p["X"]), dev(p["dY"])
+    Y, saved = ops.qlora_mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws)
+    grads = ops.qlora_mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws)
+    torch.cuda.synchronize()
+    out = {"Y": gpu_f64(Y), "status": ops.qlora_last_device_status(ws), "q": qs}
+    for k in ("E", "G", "H", "XA_g", "XA_u", "HA_d"):
+        out[k] = gpu_f64(saved[k])
+    for k, v in grads.items():
+        out[k] = gpu_f64(v)
+    return out
+
+
+def run_mlp_oracle(p, act):
+    lin, qs = {}, {}
+    for k in ("g", "u", "d"):
+        c, a, W = oracle_weight(p["W_" + k])
+        lin[k] = (W, f64(p["A_" + k]), f64(p["B_" + k]), p["s"])
+        qs[k] = (c, a)
+    X, dY = f64(p["X"]), f64(p["dY"])
+    fwd = oracle.mlp_fwd(act, X, lin["g"], lin["u"], lin["d"])
+    bwd = oracle.mlp_bwd(act, X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+    out = dict(fwd)
+    out.update(bwd)
+    out["XA_g"] = X @ lin["g"][1]
+    out["XA_u"] = X @ lin["u"][1]
+    out["HA_d"] = fwd["H"] @ lin["d"][1]
+    out["q"] = qs
+    return out

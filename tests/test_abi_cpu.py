@@ -1,0 +1,89 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every entry
+point declared in include/qlora.h, returns the oracle's NF4 levels, and rejects
+bad arguments on the host (no GPU is touched by any call here)."""
+
+import ctypes
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from qlora_fine_tuning_nf4_b200 import build, ops
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.lib()
+
+
+def _declared():
+    src = open(ops.HEADER_PATH).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(ops._SIGS), "binding and header disagree"
+
+
+def test_codebook_matches_oracle_construction_bit_for_bit(lib):
+    ours = np.array(ops.qlora_nf4_codebook(), dtype=np.float32)
+    ref = oracle.nf4_codebook().astype(np.float32)
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+def test_status_strings(lib):
+    for code, name in ops.STATUS_NAMES.items():
+        assert ops.qlora_status_string(code) == name
+
+
+def test_workspace_queries(lib):
+    small = ops.qlora_linear_workspace_bytes(256, 512, 1024)
+    big = ops.qlora_linear_workspace_bytes(8192, 4096, 4096)
+    assert 256 < small < big
+    m = ops.qlora_mlp_workspace_bytes(8192, 4096, 11008)
+    assert m >= 2 * 8192 * 11008 * 2  # dE and dG live in the workspace
+    assert ops.qlora_linear_workspace_bytes(0, 512, 1024) == 256
+    assert ops.qlora_linear_workspace_bytes(16, 512, 1024, 8) == 256  # r != 16 unsupported
+
+
+def _lin(codes=16, absmax=16, A=16, B=16, n=512, k=512, r=16, scale=1.0):
+    # fake device addresses: every call below is rejected before any CUDA call
+    return ops.QloraLoraLinear(ops.QloraNF4(codes, absmax, n, k), A, B, r, scale)
+
+
+def test_host_side_rejections(lib):
+    c = _lin()
+    f = lib.qlora_linear_fwd
+    assert f(ctypes.byref(c), 16, 0, 16, 16, 16, 1 << 30, None) == 0          # M = 0: nothing to do
+    assert f(ctypes.byref(c), 16, -1, 16, 16, 16, 1 << 30, None) == 1         # negative M
+    assert f(None, 16, 8, 16, 16, 16, 1 << 30, None) == 1                     # null struct
+    assert f(ctypes.byref(c), None, 8, 16, 16, 16, 1 << 30, None) == 1        # null X
+    assert f(ctypes.byref(c), 24, 8, 16, 16, 16, 1 << 30, None) == 3          # misaligned X
+    assert f(ctypes.byref(c), 16, 8, 16, 16, 16, 64, None) == 4               # workspace too small
+    assert f(ctypes.byref(_lin(r=8)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # r != 16
+    assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in % 256
+    assert f(ctypes.byref(_lin(n=500)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # n_out % 8
+    assert f(ctypes.byref(_lin(codes=8)), 16, 8, 16, 16, 16, 1 << 30, None) == 3
+    assert lib.nf4_dequantize(16, 16, 4, 100, 16, None) == 2                    # k_in % 64
+    assert lib.nf4_dequantize(16, 16, 4, 64, 8, None) == 3
+    assert lib.nf4_quantize(16, 0, 64, 16, 16, None) == 0                       # empty
+    g, u, d = _lin(n=512, k=256), _lin(n=512, k=256), _lin(n=256, k=512)
+    sv = ops.QloraMlpSaved(16, 16, 16, 16, 16, 16)
+    mf = lib.qlora_mlp_fwd
+    assert mf(5, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, 8, 16, ctypes.byref(sv), 16, 1 << 40, None) == 1
+    bad_d = _lin(n=256, k=768)
+    assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(bad_d), 16, 8, 16, ctypes.byref(sv), 16, 1 << 40,
+              None) == 1                                                        # shapes do not chain
+    assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, 8, 16, ctypes.byref(sv), 16, 10, None) == 4
+
+
+def test_cta_group_setting(lib):
+    prev = ops.qlora_set_cta_group(1)
+    assert ops.qlora_set_cta_group(prev) == 1
+    assert ops.qlora_set_cta_group(3) == prev  # invalid values are ignored
