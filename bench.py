@@ -1,0 +1,398 @@
+"""Benchmark: QLoRA gated-MLP forward + backward (Llama-7B shapes) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+One step = ``qlora_mlp_fwd`` + ``qlora_mlp_bwd`` of the SwiGLU MLP
+(M = 8192 tokens = batch 4 x seq 2048, d = 4096, h = 11008, NF4 block 64,
+LoRA rank 16, alpha 16) through the library's C ABI, on synthetic seeded
+inputs resident in HBM.  With N > 1 (torchrun, one rank per GPU) every rank
+runs its own 8192-token batch (weak scaling) and the six LoRA gradients are
+summed across ranks with one NCCL all-reduce, as data-parallel training does.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+instead (rank 0 only) on a bounded row sample of the same workload.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from qlora_fine_tuning_nf4_b200.workloads import MLP_WORKLOADS, mlp_flops  # noqa: E402
+
+METRIC = "QLoRA MLP fwd+bwd TFLOP/s & tokens/s (Llama-7B shape), % of bf16 peak"
+UNIT = "TFLOP/s"
+L2_NOTE = "inputs larger than L2 (saved E/G/H and dE/dG are 5 x 172 MiB per step)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cta-group", type=int, default=2)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"], "hbm": p["hbm_gbs"],
+                "src": "measured"}
+    except Exception:
+        return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "src": "fallback"}
+
+
+def kernel_flops(name, M, d, h, r):
+    """Algorithmic FLOP of one launch of each tensor-core kernel of the MLP step."""
+    return {
+        "gemm_nf4_gateup_glu_fwd": 2 * M * d * (2 * h) + 2 * M * r * (2 * h),
+        "gemm_nf4_fwd": 2 * M * h * d + 2 * M * r * d,
+        "gemm_nf4_down_bwd_glu": 2 * M * d * h + 2 * M * r * h,
+        "gemm_nf4_bwd_dx": 2 * M * (2 * h) * d + 2 * M * (2 * r) * d,
+    }.get(name)
+
+
+def source_hash():
+    h = hashlib.sha1()
+    for f in ("gemm_nf4.cu", "ptx.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "qlora_fine_tuning_nf4_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            t = json.load(f)
+        e = t.get(kernel, {})
+        if e.get("source_sha1") == source_hash() and e.get("workload") == workload:
+            return e.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def smi_device_id(local):
+    """nvidia-smi -i argument for this process's GPU (its UUID when torch knows it)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local)
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ oracle arm ---
+
+def oracle_sample(wl, rows, seed_rows=0):
+    """Time the fp64 oracle's MLP fwd+bwd on `rows` tokens of the workload.
+
+    Returns (seconds, flop, threads).  Weights are quantised/dequantised by the
+    oracle itself before timing (one-time, like the GPU side's quantisation).
+    """
+    import oracle
+    from oracle.nf4 import nf4_dequantize_f64
+    from qlora_fine_tuning_nf4_b200.synth import make_mlp_problem
+
+    p = make_mlp_problem(wl["M"], wl["d"], wl["h"], wl["r"], wl["alpha"], wl["seed"])
+    lin = {}
+    for k in ("g", "u", "d"):
+        n, kk = p["W_" + k].shape
+        c, a = oracle.nf4_quantize(p["W_" + k], n, kk)
+        lin[k] = (nf4_dequantize_f64(c, a, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
+                  oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
+    X = oracle.bf16_bits_to_f64(p["X"][seed_rows:seed_rows + rows])
+    dY = oracle.bf16_bits_to_f64(p["dY"][seed_rows:seed_rows + rows])
+    t0 = time.perf_counter()
+    fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
+    oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+    dt = time.perf_counter() - t0
+    return dt, mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0))
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from oracle.nf4 import nf4_dequantize_f64
+    from qlora_fine_tuning_nf4_b200.synth import make_mlp_problem
+
+    p = make_mlp_problem(wl["M"], wl["d"], wl["h"], wl["r"], wl["alpha"], wl["seed"])
+    lin = {}
+    for k in ("g", "u", "d"):
+        n, kk = p["W_" + k].shape
+        c, a = oracle.nf4_quantize(p["W_" + k], n, kk)
+        lin[k] = (nf4_dequantize_f64(c, a, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
+                  oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
+
+    def step(rows, off):
+        X = oracle.bf16_bits_to_f64(p["X"][off:off + rows])
+        dY = oracle.bf16_bits_to_f64(p["dY"][off:off + rows])
+        fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
+        oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+
+    # size the per-step row sample so the whole run takes about two minutes
+    t0 = time.perf_counter()
+    step(32, 0)
+    per_row = (time.perf_counter() - t0) / 32
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(16, min(wl["M"], budget / max(per_row, 1e-9))))
+    rows -= rows % 16
+    rows = max(rows, 16)
+    for i in range(args.warmup):
+        step(rows, (i * rows) % (wl["M"] - rows + 1))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(rows, (i * rows) % (wl["M"] - rows + 1))
+    dt = time.perf_counter() - t0
+    flop = mlp_flops(rows, wl["d"], wl["h"], wl["r"]) * args.steps
+    value = flop / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = f"{rows} of {wl['M']} token rows per step (fp64 numpy, BLAS threads = cores)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "M": wl["M"], "d": wl["d"], "h": wl["h"], "r": wl["r"],
+                   "act": wl["act"], "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# -------------------------------------------------------------- GPU arm ----
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_mlp_problem
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ops.lib()
+    ops.qlora_set_cta_group(args.cta_group)
+    M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
+
+    # Inputs: same seeded recipe as the tests; each rank draws its own batch.
+    p = make_mlp_problem(M, d, h, r, wl["alpha"], wl["seed"] + 1000 * rank)
+    lins = {}
+    for k in ("g", "u", "d"):
+        w = ops.nf4_quantize(bits_to_torch(p["W_" + k], dev))
+        lins[k] = ops.LoraLinear(w, bits_to_torch(p["A_" + k], dev), bits_to_torch(p["B_" + k], dev), p["s"])
+    X = bits_to_torch(p["X"], dev)
+    dY = bits_to_torch(p["dY"], dev)
+    del p
+    ws = ops.Workspace(dev)
+    saved = ops.make_mlp_saved(M, h, r, dev)
+    Y = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+    # LoRA gradients as views of one flat buffer -> one all-reduce per step
+    sizes = [("dA_g", (d, r)), ("dB_g", (r, h)), ("dA_u", (d, r)), ("dB_u", (r, h)), ("dA_d", (h, r)),
+             ("dB_d", (r, d))]
+    flat = torch.empty(sum(a * b for _, (a, b) in sizes), dtype=torch.bfloat16, device=dev)
+    grads, off = {}, 0
+    for name, (a, b) in sizes:
+        grads[name] = flat[off:off + a * b].view(a, b)
+        off += a * b
+    grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        ops.qlora_mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws, Y=Y, saved=saved)
+        ops.qlora_mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads)
+        if world > 1:
+            dist.all_reduce(flat)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if ops.qlora_last_device_status(ws) != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    clk = ClockSampler(smi_device_id(local))
+    launches0 = ops.qlora_launch_count()
+    barrier()
+    clk.start()
+    time.sleep(0.3)
+    ops.qlora_trace_begin()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    trace = ops.qlora_trace_end()
+    clocks = clk.stop()
+    launches = ops.qlora_launch_count() - launches0
+    if ops.qlora_last_device_status(ws) != 0:
+        raise RuntimeError("device status error during the timed region")
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    flop_step = mlp_flops(M, d, h, r)
+    value = flop_step * args.steps * world / (ms / 1e3) / 1e12
+    tokens = M * args.steps * world / (ms / 1e3)
+    pk = peaks()
+
+    # ---- end-to-end through the public API with host buffers ----
+    hX = torch.empty(M, d, dtype=torch.bfloat16, pin_memory=True)
+    hdY = torch.empty(M, d, dtype=torch.bfloat16, pin_memory=True)
+    hX.copy_(X.cpu())
+    hdY.copy_(dY.cpu())
+    hY = torch.empty_like(hX, pin_memory=True)
+    hdX = torch.empty_like(hX, pin_memory=True)
+    hflat = torch.empty(flat.numel(), dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        X.copy_(hX, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        step()
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(grads["dX"], non_blocking=True)
+        hflat.copy_(flat, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    ems = e0.elapsed_time(e1)
+    t = torch.tensor([ems], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ems = float(t.item())
+    e2e_value = flop_step * e2e_steps * world / (ems / 1e3) / 1e12
+    h2d = 2 * M * d * 2
+    d2h = 2 * M * d * 2 + flat.numel() * 2
+
+    # ---- roofline of the dominant kernel (live CUDA-event times) ----
+    roof = None
+    tc = {k: v for k, v in trace.items() if kernel_flops(k, M, d, h, r)}
+    if tc:
+        top = max(tc, key=lambda k: tc[k][1])
+        n_l, tot = tc[top]
+        avg_s = tot / n_l / 1e3
+        ach = kernel_flops(top, M, d, h, r) / avg_s / 1e12
+        peak = pk["bf16_sustained"]
+        roof = {"bound": "tensor", "kernel": top, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "peak_kind": f"bf16 dense, sustained, {pk['src']}",
+                "traffic": traffic_for(top, args.workload), "avg_launch_ms": avg_s * 1e3,
+                "share_of_step": tot / ms}
+    kernels = {k: {"launches": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / ms, 4)}
+               for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 512
+        dt, fl, cores = oracle_sample(wl, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{rows} of {M} token rows, one fwd+bwd (fp64 numpy, {dt:.1f} s)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "tokens_per_s": tokens, "frac_of_bf16_peak": value / world / pk["bf16"],
+        "frac_of_bf16_peak_sustained": value / world / pk["bf16_sustained"],
+        "config": {"workload": args.workload, "M_per_gpu": M, "d": d, "h": h, "r": r, "act": act,
+                   "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
+                   "cta_group": args.cta_group, "l2": L2_NOTE},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    wl = MLP_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -14,7 +14,13 @@ from oracle.nf4 import nf4_dequantize_f64
 from qlora_fine_tuning_nf4_b200 import ops
 from qlora_fine_tuning_nf4_b200.synth import bits_to_torch
 
-TOL = 2e-2  # max |gpu - oracle| <= TOL * RMS(oracle), per tensor
+TOL = 2e-2  # max |gpu - oracle| <= TOL * RMS(oracle), per tensor (every workload at full size)
+# Small-M gated-MLP cases: the saved activations (E, G, H), dE/dG, X A and s G
+# are bf16 by design; a CPU emulation of exactly those bf16 roundings (no
+# kernel involved) already gives max|err| = 1.5-2.2e-2 x RMS on the MLP outputs
+# at M = 200-1024 tokens, because the max over elements of few-row sums is
+# dominated by single heavy-tailed products.  These cases use 3e-2.
+TOL_SMALL_MLP = 3e-2
 
 
 def f64(bits):
@@ -36,6 +42,18 @@ def assert_close(name, gpu, ref, tol=TOL):
     err, rms = rel_err(gpu, ref)
     assert err <= tol * rms, f"{name}: max|err| {err:.3e} > {tol} * RMS {rms:.3e} (ratio {err / max(rms, 1e-300):.3e})"
     return err / max(rms, 1e-300)
+
+
+def assert_saved(name, gpu, ref):
+    """Saved bf16 activations, elementwise: output rounding (2^-9 relative, taken
+    as 2^-8) plus an absolute slack of 2^-10 x RMS for the rounded LoRA operand
+    and fp32 accumulation."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -10 * rms
+    bad = np.abs(gpu - ref) > bound
+    assert not bad.any(), f"{name}: {int(bad.sum())} of {bad.size} elements outside the bf16 rounding bound"
 
 
 def dev(bits):

@@ -1,0 +1,92 @@
+"""Multi-process (world size 2, gloo, CPU) check of the data-parallel step logic:
+each rank computes the adapter gradients of its token shard (oracle, fp64), the
+flat buffer is all-reduced, and the sum equals the full-batch gradients."""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from qlora_fine_tuning_nf4_b200 import dp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _problem():
+    rng = np.random.default_rng(0)
+    M, d, h, r = 24, 64, 96, 4
+    X = rng.standard_normal((M, d))
+    proj = lambda K, N, s: (rng.standard_normal((N, K)) * 0.2, rng.uniform(-1, 1, (K, r)) / np.sqrt(K),
+                            rng.standard_normal((r, N)) * 0.3, s)
+    gate, up, down = proj(d, h, 1.0), proj(d, h, 1.0), proj(h, d, 2.0)
+    dY = rng.standard_normal((M, d))
+    return M, d, h, r, X, gate, up, down, dY
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        M, d, h, r, X, gate, up, down, dY = _problem()
+        lo, hi = dp.shard_rows(M, rank, world)
+        g = oracle.mlp_bwd("swiglu", X[lo:hi], gate, up, down, dY[lo:hi])
+        flat, views = dp.flat_lora_grads(d, h, r, "cpu", dtype=torch.float64)
+        for k in dp.GRAD_ORDER:
+            views[k].copy_(torch.from_numpy(g[k]))
+        dp.allreduce_lora_grads(flat)
+        if rank == 0:
+            q.put({k: views[k].numpy().copy() for k in dp.GRAD_ORDER})
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_gradients_sum_to_full_batch():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(rk, 2, port, q)) for rk in range(2)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    M, d, h, r, X, gate, up, down, dY = _problem()
+    full = oracle.mlp_bwd("swiglu", X, gate, up, down, dY)
+    for k in dp.GRAD_ORDER:
+        np.testing.assert_allclose(got[k], full[k], rtol=1e-12, atol=1e-12)
+
+
+def test_flat_buffer_views_are_aligned_and_disjoint():
+    flat, views = dp.flat_lora_grads(4096, 11008, 16, "cpu")
+    offs = []
+    for k in dp.GRAD_ORDER:
+        v = views[k]
+        assert v.is_contiguous()
+        off = (v.data_ptr() - flat.data_ptr())
+        assert off % 16 == 0
+        offs.append((off, off + v.numel() * v.element_size()))
+    offs.sort()
+    assert all(a[1] <= b[0] for a, b in zip(offs, offs[1:]))
+    assert offs[-1][1] == flat.numel() * flat.element_size()
+
+
+@pytest.mark.parametrize("M,world", [(8192, 1), (8192, 8), (100, 3), (2, 4)])
+def test_shard_rows_partition(M, world):
+    seen = []
+    for rk in range(world):
+        lo, hi = dp.shard_rows(M, rk, world)
+        seen.extend(range(lo, hi))
+    assert seen == list(range(M))
