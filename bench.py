@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-group", type=int, default=2)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override M (tokens per GPU) for small profiling cases; 0 = the workload's M")
     return ap.parse_args()
 
 
@@ -387,7 +389,9 @@ def run_ours(args, wl):
 
 def main():
     args = parse()
-    wl = MLP_WORKLOADS[args.workload]
+    wl = dict(MLP_WORKLOADS[args.workload])
+    if args.tokens:
+        wl["M"] = args.tokens
     if args.impl == "reference":
         run_reference(args, wl)
     else:

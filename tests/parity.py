@@ -44,14 +44,33 @@ def assert_close(name, gpu, ref, tol=TOL):
     return err / max(rms, 1e-300)
 
 
-def assert_saved(name, gpu, ref):
-    """Saved bf16 activations, elementwise: output rounding (2^-9 relative, taken
-    as 2^-8) plus an absolute slack of 2^-10 x RMS for the rounded LoRA operand
-    and fp32 accumulation."""
+def saved_bounds(o, p):
+    """Elementwise error bounds of the saved bf16 activations E, G, H.
+
+    bf16 keeps 8 significant bits, so one round-to-nearest-even costs at most
+    u = 2^-8 relative.  e and g are fp32 accumulations whose LoRA operand s*XA
+    is rounded to bf16: |de| <= u s |XA||B| plus an fp32 accumulation slack
+    2^-16 |X||W|^T; both carry a safety factor 4, and the stored value's own
+    rounding (u |e|) a factor 2.  h = act(e) g is formed from the fp32 e, g:
+    |dh| <= 2u |h| + |act'(e) g| |de| + |act(e)| |dg|.
+    """
+    u = 2.0 ** -8
+    act = o["act"]
+    out = {}
+    de = {}
+    for k, key in (("g", "E"), ("u", "G")):
+        W, A, B, s = o["lin"][k]
+        de[key] = 4 * u * s * (np.abs(o["X"] @ A) @ np.abs(B)) + 2.0 ** -14 * (np.abs(o["X"]) @ np.abs(W).T)
+        out[key] = 2 * u * np.abs(o[key]) + de[key]
+    out["H"] = (2 * u * np.abs(o["H"]) + np.abs(oracle.act_grad(act, o["E"]) * o["G"]) * de["E"]
+                + np.abs(oracle.act_fwd(act, o["E"])) * de["G"])
+    return out
+
+
+def assert_saved(name, gpu, ref, bound):
+    """Saved bf16 activations, elementwise against `saved_bounds`."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    rms = float(np.sqrt(np.mean(ref * ref)))
-    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -10 * rms
     bad = np.abs(gpu - ref) > bound
     assert not bad.any(), f"{name}: {int(bad.sum())} of {bad.size} elements outside the bf16 rounding bound"
 
@@ -131,4 +150,5 @@ def run_mlp_oracle(p, act):
     out["XA_u"] = X @ lin["u"][1]
     out["HA_d"] = fwd["H"] @ lin["d"][1]
     out["q"] = qs
+    out["lin"], out["X"], out["act"] = lin, X, act
     return out

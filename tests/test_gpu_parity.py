@@ -15,7 +15,7 @@ from qlora_fine_tuning_nf4_b200 import ops
 from qlora_fine_tuning_nf4_b200.synth import bf16_bits, make_linear_problem, make_mlp_problem
 
 from parity import (TOL_SMALL_MLP, assert_close, assert_saved, dev, gpu_weight, oracle_weight, run_linear_gpu,
-                    run_linear_oracle, run_mlp_gpu, run_mlp_oracle)
+                    run_linear_oracle, run_mlp_gpu, run_mlp_oracle, saved_bounds)
 
 pytestmark = pytest.mark.gpu
 
@@ -149,8 +149,9 @@ def test_mlp_fwd_bwd_parity(cg, act, M, d, h):
     assert g["status"] == 0
     for k in ("g", "u", "d"):
         assert np.array_equal(g["q"][k][0], o["q"][k][0]) and np.array_equal(g["q"][k][1], o["q"][k][1])
+    bounds = saved_bounds(o, p)
     for k in ("E", "G", "H"):
-        assert_saved(k, g[k], o[k])
+        assert_saved(k, g[k], o[k], bounds[k])
     for k in ("XA_g", "XA_u", "HA_d"):
         assert_close(k, g[k], o[k])
     for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
