@@ -192,6 +192,24 @@ QLORA_API int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries);
 /* Number of kernels this library has launched since it was loaded. */
 QLORA_API uint64_t qlora_launch_count(void);
 
+/* Same computation and outputs as qlora_linear_fwd, for callers that cannot
+ * allocate device memory and so cannot pass a workspace: for example a plugin
+ * that only receives the device pointers of its tensors from a host framework
+ * that owns all device memory, or a path where allocating is not permitted.
+ * (The pages describe no such call; it has no counterpart there.)
+ * Its scratch is a fixed 4 MiB array inside the library that every GPU which
+ * loads the library keeps until the process exits; problems that need more
+ * (M above about 43,000 rows) return QLORA_ERR_WORKSPACE_TOO_SMALL before
+ * anything is enqueued.  It allocates nothing and frees nothing.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array: calls whose GPU work overlaps (on
+ * different streams, or from different threads) race and must not be issued.
+ * Each call zeroes the status word it uses; device-side timeouts are recorded
+ * there and are not reported back through this call. */
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M,
+                                                qlora_bf16* Y, qlora_bf16* XA_saved, qlora_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -715,3 +715,65 @@ int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries) {
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward projection without a caller-supplied workspace.
+//
+// Some callers cannot hand us device memory: a kernel plugin that only receives
+// the device pointers of its tensors from a host framework which owns all
+// device memory (a raw cudaMalloc there would bypass the framework's allocator
+// and memory budget), or a code path where allocating is not allowed at all.
+// For them the scratch of qlora_linear_fwd (the status word, the s-scaled copy
+// of X A and the split-K partial sums) lives in this fixed array instead.  Every
+// GPU that loads the library holds it until the process exits.
+static constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static void* g_noalloc_scratch_ptr[64] = {};
+
+// Device address of g_noalloc_scratch for the current device.  The host-side
+// name of the array is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static qlora_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_CUDA;
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return QLORA_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev] = p;
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return QLORA_OK;
+}
+
+extern "C" {
+
+qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                                      qlora_bf16* XA_saved, qlora_stream_t stream) {
+  qlora_status s = check_linear(lin);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !Y || !XA_saved) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(Y) || misaligned(XA_saved)) return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t K = lin->w.k_in;
+  const size_t vec = align256(static_cast<size_t>(M) * 32);
+  const size_t need = 256 + vec + align256(rowproj_part_bytes(M, K, 16));
+  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  void* base = nullptr;
+  if ((s = noalloc_scratch(&base)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps whatever the previous call left; only the status word must start at zero.
+  if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  char* w = static_cast<char*>(base);
+  int* status = reinterpret_cast<int*>(w);
+  bf16* xa = reinterpret_cast<bf16*>(XA_saved);
+  bf16* XAs = lin->scale != 1.0f ? reinterpret_cast<bf16*>(w + 256) : xa;
+  float* part = reinterpret_cast<float*>(w + 256 + vec);
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
+                   routs(rout(xa, 0, 16, 0, 1.f), rout(XAs != xa ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
+  if (s != QLORA_OK) return s;
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, st);
+}
+
+}  // extern "C"

@@ -80,6 +80,8 @@ _SIGS = {
     "qlora_trace_begin": (ctypes.c_int, []),
     "qlora_trace_end": (ctypes.c_int32, [ctypes.POINTER(QloraTraceEntry), ctypes.c_int32]),
     "qlora_launch_count": (ctypes.c_uint64, []),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -199,6 +201,21 @@ def qlora_linear_fwd(lin: LoraLinear, X, ws: Workspace, Y=None, XA=None):
     c = lin.c()
     _check("qlora_linear_fwd", lib().qlora_linear_fwd(ctypes.byref(c), _p(X), M, _p(Y), _p(XA), _p(buf),
                                                       buf.numel(), _stream()))
+    return Y, XA
+
+
+def qlora_linear_fwd_noalloc(lin: LoraLinear, X, Y=None, XA=None):
+    """qlora_linear_fwd without a workspace, for callers that cannot allocate
+    device memory; its scratch is a fixed array inside the library (shared by
+    all calls, so calls must not overlap on the GPU)."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, lin.w.n_out, dtype=torch.bfloat16, device=X.device)
+    if XA is None:
+        XA = torch.empty(M, lin.A.shape[1], dtype=torch.bfloat16, device=X.device)
+    c = lin.c()
+    _check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(ctypes.byref(c), _p(X), M, _p(Y), _p(XA),
+                                                                      _stream()))
     return Y, XA
 
 
