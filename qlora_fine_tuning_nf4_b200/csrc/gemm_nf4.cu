@@ -67,20 +67,28 @@ QL_DEV uint4 nf4_decode8(uint32_t w, const uint32_t (&tl)[4], const uint32_t (&t
   return out;
 }
 
+// Activations in fp32 on the hardware's approximate exp2 / reciprocal / tanh
+// units (relative error well below the bf16 rounding of the stored results).
+QL_DEV float fast_sigmoid(float e) { return __frcp_rn(1.0f + __expf(-e)); }
+QL_DEV float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 QL_DEV float act_f(int act, float e) {
-  if (act == ACT_SILU) return e / (1.0f + expf(-e));
-  const float t = tanhf(0.7978845608028654f * (e + 0.044715f * e * e * e));
+  if (act == ACT_SILU) return e * fast_sigmoid(e);
+  const float t = tanh_approx(0.7978845608028654f * (e + 0.044715f * e * e * e));
   return 0.5f * e * (1.0f + t);
 }
 // (act(e), act'(e))
 QL_DEV void act_fg(int act, float e, float& f, float& g) {
   if (act == ACT_SILU) {
-    const float s = 1.0f / (1.0f + expf(-e));
+    const float s = fast_sigmoid(e);
     f = e * s;
     g = s * (1.0f + e * (1.0f - s));
   } else {
     const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-    const float t = tanhf(k0 * (e + k1 * e * e * e));
+    const float t = tanh_approx(k0 * (e + k1 * e * e * e));
     f = 0.5f * e * (1.0f + t);
     g = 0.5f * (1.0f + t) + 0.5f * e * (1.0f - t * t) * k0 * (1.0f + 3.0f * k1 * e * e);
   }
@@ -108,16 +116,23 @@ struct GemmCfg {
   static constexpr int OFF_LA = OFF_RA + RS * RA_BYTES;
   static constexpr int OFF_LB = OFF_LA + 2 * LA_BYTES;
   static constexpr int OFF_BAR = OFF_LB + 2 * LB_BYTES;
-  static constexpr int NBAR = 2 * S + 2 * RS + 3;
+  static constexpr int NBAR = 2 * S + 2 * RS + 7;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
-  static constexpr int THREADS = 14 * 32;
-  static constexpr int TMEM_COLS = 256;
+  static constexpr int EPI_WARPS = 8;            // two per TMEM lane quadrant
+  static constexpr int DQ_WARPS = 8;
+  static constexpr int THREADS = (2 + EPI_WARPS + DQ_WARPS) * 32;
+  static constexpr int TMEM_COLS = 512;          // two 256-column accumulators
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0, "1024B alignment of swizzled regions");
 };
 
+// Persistent kernel: each CTA (or CTA pair) walks the output tiles
+// t = cluster, cluster + clusters, ... (N tiles fastest).  Every role iterates
+// the same tile sequence; j counts 64-wide reduction blocks across tiles and
+// indexes the rings, so barrier phases follow from j and the tile counter.
 template <int MODE, int EPI, int CG>
-__global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
+__global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
+    gemm_nf4_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
   using C = GemmCfg<MODE, CG>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -127,14 +142,12 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
   const int lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
 
-  // Tile coordinates: N tiles vary fastest so CTAs in flight share an A row block.
   const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
   const int n_tiles = (args.N + bn_out - 1) / bn_out;
-  const int pair = blockIdx.x / CG;
-  const int nt = pair % n_tiles;
-  const int mt = pair / n_tiles;
-  const int m0 = mt * (C::BM * CG) + static_cast<int>(rank) * C::BM;
-  const int n0 = nt * bn_out;
+  const int m_tiles = (args.M + C::BM * CG - 1) / (C::BM * CG);
+  const int total_tiles = n_tiles * m_tiles;
+  const int cluster = blockIdx.x / CG;
+  const int clusters = gridDim.x / CG;
   const int nk = args.nkb0 + args.nkb1;
 
   // barriers
@@ -143,9 +156,11 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::S + s); };
   auto rfull_bar = [&](int s) { return bar0 + 8u * (2 * C::S + s); };
   auto rempty_bar = [&](int s) { return bar0 + 8u * (2 * C::S + C::RS + s); };
-  const uint32_t lora_bar = bar0 + 8u * (2 * C::S + 2 * C::RS);
-  const uint32_t acc_bar = lora_bar + 8u;
-  const uint32_t drain_bar = lora_bar + 16u;
+  const uint32_t lora_full = bar0 + 8u * (2 * C::S + 2 * C::RS);
+  const uint32_t lora_empty = lora_full + 8u;
+  const uint32_t acc_full0 = lora_full + 16u;   // [2]
+  const uint32_t acc_empty0 = lora_full + 32u;  // [2]
+  const uint32_t drain_bar = lora_full + 48u;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + C::NBAR * 8);
 
   if (threadIdx.x == 0) {
@@ -157,8 +172,12 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
       mbar_init(rfull_bar(s), 1);
       mbar_init(rempty_bar(s), C::NB / 32);
     }
-    mbar_init(lora_bar, 1);
-    mbar_init(acc_bar, 1);
+    mbar_init(lora_full, 1);
+    mbar_init(lora_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full0 + 8u * b, 1);
+      mbar_init(acc_empty0 + 8u * b, CG * C::EPI_WARPS);
+    }
     mbar_init(drain_bar, 1);
     fence_mbar_init();
   }
@@ -173,6 +192,10 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
 
   // shared::cluster address of a barrier in the pair's leader CTA
   auto leader = [&](uint32_t bar) { return (CG == 2) ? mapa_shared(bar, 0) : bar; };
+  auto tile_coords = [&](int t, int& m0, int& n0) {
+    m0 = (t / n_tiles) * (C::BM * CG) + static_cast<int>(rank) * C::BM;
+    n0 = (t % n_tiles) * bn_out;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -187,59 +210,66 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
         if constexpr (CG == 2) tma_load_2d_pair(dst, m, leader(bar_local), x, y);
         else tma_load_2d(dst, m, bar_local, x, y);
       };
-      if (args.lora > 0) {
-        int bytes = args.lora * C::LA_BYTES;
-        if (MODE == MODE_FWD) bytes += C::BNC * 32;
-        if (MODE == MODE_FWD_GLU) bytes += 2 * (128 / CG) * 32;
-        if (MODE == MODE_BWD) bytes += args.lora * C::BNC * 32;
-        if (rank == 0) mbar_arrive_expect_tx(lora_bar, bytes * CG);
+      int lora_bytes = args.lora * C::LA_BYTES;
+      if (MODE == MODE_FWD) lora_bytes += C::BNC * 32;
+      if (MODE == MODE_FWD_GLU) lora_bytes += 2 * (128 / CG) * 32;
+      if (MODE == MODE_BWD) lora_bytes += args.lora * C::BNC * 32;
+      int j = 0, tl = 0;
+      for (int t = cluster; t < total_tiles && ok; t += clusters, ++tl) {
+        int m0, n0;
+        tile_coords(t, m0, n0);
+        for (int kb = 0; kb < nk; ++kb, ++j) {
+          const int seg = kb >= args.nkb0 ? 1 : 0;
+          const int kl = kb - seg * args.nkb0;
+          // raw NF4 codes + absmax for the dequantisers (local barrier)
+          const int rs = j % C::RS;
+          ok = mbar_wait(rempty_bar(rs), ((j / C::RS) & 1) ^ 1, args.status);
+          if (!ok) break;
+          mbar_arrive_expect_tx(rfull_bar(rs), C::RC_BYTES + C::RA_BYTES);
+          const uint32_t rc = sbase + C::OFF_RC + rs * C::RC_BYTES;
+          const uint32_t ra = sbase + C::OFF_RA + rs * C::RA_BYTES;
+          if (MODE == MODE_BWD) {
+            const int kw0 = n0 + (int)rank * C::BNC;
+            tma_load_2d(rc, &maps.codes[seg], rfull_bar(rs), kw0 / 2, kl * 64);
+            tma_load_2d(ra, &maps.absmax[seg], rfull_bar(rs), (kw0 / 64) & ~3, kl * 64);
+          } else {
+            for (int h = 0; h < C::BNC / 128; ++h) {
+              int src = 0, row = n0 + (int)rank * C::BNC + h * 128;
+              if (MODE == MODE_FWD_GLU) {
+                src = (CG == 1) ? h : (int)rank;
+                row = n0;
+              }
+              tma_load_2d(rc + h * 4096, &maps.codes[src], rfull_bar(rs), kl * 32, row);
+              tma_load_2d(ra + h * 2048, &maps.absmax[src], rfull_bar(rs), kl & ~3, row);
+            }
+          }
+          // A operand tile (completes on the leader's full barrier)
+          const int s = j % C::S;
+          ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
+          if (!ok) break;
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
+          load(sbase + C::OFF_A + s * C::A_BYTES, &maps.a[seg], full_bar(s), kl * 64, m0);
+        }
+        if (!ok || args.lora == 0) continue;
+        // LoRA operands of this tile (single buffer, released by the MMA's commit)
+        ok = mbar_wait(lora_empty, (tl & 1) ^ 1, args.status);
+        if (!ok) break;
+        if (rank == 0) mbar_arrive_expect_tx(lora_full, lora_bytes * CG);
         for (int i = 0; i < args.lora; ++i) {
-          load(sbase + C::OFF_LA + i * C::LA_BYTES, &maps.la[i], lora_bar, 0, m0);
+          load(sbase + C::OFF_LA + i * C::LA_BYTES, &maps.la[i], lora_full, 0, m0);
           if (MODE == MODE_FWD) {
             for (int c = 0; c < C::BNC / 64; ++c)
-              load(sbase + C::OFF_LB + c * 2048, &maps.lb[0], lora_bar, n0 + (int)rank * C::BNC + c * 64, 0);
+              load(sbase + C::OFF_LB + c * 2048, &maps.lb[0], lora_full, n0 + (int)rank * C::BNC + c * 64, 0);
           } else if (MODE == MODE_FWD_GLU) {
             for (int c = 0; c < (128 / CG) / 64; ++c)
-              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 2048, &maps.lb[i], lora_bar,
+              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 2048, &maps.lb[i], lora_full,
                    n0 + (int)rank * (128 / CG) + c * 64, 0);
           } else {
             for (int c = 0; c < C::BNC / 128; ++c)
-              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 4096, &maps.lb[i], lora_bar, 0,
+              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 4096, &maps.lb[i], lora_full, 0,
                    n0 + (int)rank * C::BNC + c * 128);
           }
         }
-      }
-      for (int kb = 0; kb < nk && ok; ++kb) {
-        const int seg = kb >= args.nkb0 ? 1 : 0;
-        const int kl = kb - seg * args.nkb0;
-        // raw NF4 codes + absmax for the dequantisers (local barrier)
-        const int rs = kb % C::RS;
-        ok = mbar_wait(rempty_bar(rs), ((kb / C::RS) & 1) ^ 1, args.status);
-        if (!ok) break;
-        mbar_arrive_expect_tx(rfull_bar(rs), C::RC_BYTES + C::RA_BYTES);
-        const uint32_t rc = sbase + C::OFF_RC + rs * C::RC_BYTES;
-        const uint32_t ra = sbase + C::OFF_RA + rs * C::RA_BYTES;
-        if (MODE == MODE_BWD) {
-          const int kw0 = n0 + (int)rank * C::BNC;
-          tma_load_2d(rc, &maps.codes[seg], rfull_bar(rs), kw0 / 2, kl * 64);
-          tma_load_2d(ra, &maps.absmax[seg], rfull_bar(rs), (kw0 / 64) & ~3, kl * 64);
-        } else {
-          for (int h = 0; h < C::BNC / 128; ++h) {
-            int src = 0, row = n0 + (int)rank * C::BNC + h * 128;
-            if (MODE == MODE_FWD_GLU) {
-              src = (CG == 1) ? h : (int)rank;
-              row = n0;
-            }
-            tma_load_2d(rc + h * 4096, &maps.codes[src], rfull_bar(rs), kl * 32, row);
-            tma_load_2d(ra + h * 2048, &maps.absmax[src], rfull_bar(rs), kl & ~3, row);
-          }
-        }
-        // A operand tile (completes on the leader's full barrier)
-        const int s = kb % C::S;
-        ok = mbar_wait(empty_bar(s), ((kb / C::S) & 1) ^ 1, args.status);
-        if (!ok) break;
-        if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
-        load(sbase + C::OFF_A + s * C::A_BYTES, &maps.a[seg], full_bar(s), kl * 64, m0);
       }
     }
   } else if (warp == 1) {
@@ -247,62 +277,75 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
     if (rank == 0 && lane == 0) {
       bool ok = true;
       const uint32_t idesc = idesc_bf16(C::BM * CG, C::BNT, false, MODE == MODE_BWD);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::S;
-        ok = mbar_wait<CG == 2>(full_bar(s), (kb / C::S) & 1, args.status);
+      int j = 0, tl = 0;
+      for (int t = cluster; t < total_tiles && ok; t += clusters, ++tl) {
+        const int b = tl & 1;
+        ok = mbar_wait<CG == 2>(acc_empty0 + 8u * b, ((tl >> 1) & 1) ^ 1, args.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a = sbase + C::OFF_A + s * C::A_BYTES;
-        const uint32_t b = sbase + C::OFF_B + s * C::B_BYTES;
+        const uint32_t acc = tmem + b * 256;
+        for (int kb = 0; kb < nk; ++kb, ++j) {
+          const int s = j % C::S;
+          ok = mbar_wait<CG == 2>(full_bar(s), (j / C::S) & 1, args.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a = sbase + C::OFF_A + s * C::A_BYTES;
+          const uint32_t bs = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, QL_SWZ_128B);
-          const uint64_t bd = (MODE == MODE_BWD) ? smem_desc(b + kk * 2048, 8192, 1024, QL_SWZ_128B)
-                                                 : smem_desc(b + kk * 32, 16, 1024, QL_SWZ_128B);
-          umma_bf16<CG>(tmem, ad, bd, idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, QL_SWZ_128B);
+            const uint64_t bd = (MODE == MODE_BWD) ? smem_desc(bs + kk * 2048, 8192, 1024, QL_SWZ_128B)
+                                                   : smem_desc(bs + kk * 32, 16, 1024, QL_SWZ_128B);
+            umma_bf16<CG>(acc, ad, bd, idesc, (kb | kk) != 0);
+          }
+          umma_commit<CG>(empty_bar(s));
         }
-        umma_commit<CG>(empty_bar(s));
-      }
-      if (ok && args.lora > 0) {
-        ok = mbar_wait<CG == 2>(lora_bar, 0, args.status);
-        if (ok) {
+        if (!ok) break;
+        if (args.lora > 0) {
+          ok = mbar_wait<CG == 2>(lora_full, tl & 1, args.status);
+          if (!ok) break;
           tc_fence_after();
           for (int i = 0; i < args.lora; ++i) {
             const uint64_t ad = smem_desc(sbase + C::OFF_LA + i * C::LA_BYTES, 16, 256, QL_SWZ_32B);
             if (MODE == MODE_FWD) {
               const uint64_t bd = smem_desc(sbase + C::OFF_LB, 2048, 1024, QL_SWZ_128B);
-              umma_bf16<CG>(tmem, ad, bd, idesc_bf16(C::BM * CG, 256, false, true), 1);
+              umma_bf16<CG>(acc, ad, bd, idesc_bf16(C::BM * CG, 256, false, true), 1);
             } else if (MODE == MODE_FWD_GLU) {
               const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 2048, 1024, QL_SWZ_128B);
-              umma_bf16<CG>(tmem + i * 128, ad, bd, idesc_bf16(C::BM * CG, 128, false, true), 1);
+              umma_bf16<CG>(acc + i * 128, ad, bd, idesc_bf16(C::BM * CG, 128, false, true), 1);
             } else {
               const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 16, 256, QL_SWZ_32B);
-              umma_bf16<CG>(tmem, ad, bd, idesc_bf16(C::BM * CG, 256, false, false), 1);
+              umma_bf16<CG>(acc, ad, bd, idesc_bf16(C::BM * CG, 256, false, false), 1);
             }
           }
+          umma_commit<CG>(lora_empty);
         }
+        umma_commit<CG>(acc_full0 + 8u * b);
       }
-      if (ok) {
-        umma_commit<CG>(acc_bar);
-      } else {
-        umma_commit<CG>(drain_bar);  // let issued MMAs finish before TMEM is released
-        mbar_wait(drain_bar, 0, args.status);
-      }
+      // let every issued MMA finish before TMEM can be released
+      umma_commit<CG>(drain_bar);
+      mbar_wait(drain_bar, 0, args.status);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + C::EPI_WARPS) {
     // ------------------------------------------------------ epilogue -----
-    const int lg = warp & 3;
+    const int ew = warp - 2;            // 0..7
+    const int lg = warp & 3;            // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;           // which half of the tile's columns
     const int row = lg * 32 + lane;
-    const int grow = m0 + row;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_bar, 0, args.status));
-    tc_fence_after();
-    if (ok) {
-      const uint32_t trow = tmem + (static_cast<uint32_t>(lg * 32) << 16);
+    int tl = 0;
+    for (int t = cluster; t < total_tiles; t += clusters, ++tl) {
+      int m0, n0;
+      tile_coords(t, m0, n0);
+      const int b = tl & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full0 + 8u * b, (tl >> 1) & 1, args.status))) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + b * 256 + (static_cast<uint32_t>(lg * 32) << 16);
+      const int grow = m0 + row;
       const bool row_ok = grow < args.M;
-      const size_t rbase = static_cast<size_t>(grow) * args.ldo;
-      if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
+      const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
+      if (EPI == EPI_STORE) {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = half * 4; c < half * 4 + 4; ++c) {
           float v[32];
           tmem_ld_32x32b_x32(trow + c * 32, v);
           if (!row_ok) continue;
@@ -310,40 +353,54 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
           for (int q = 0; q < 4; ++q) {
             const int col = n0 + c * 32 + q * 8;
             if (col >= args.N) break;
-            uint4 o0, o1;
-            if (EPI == EPI_STORE) {
-              o0.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-              o0.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-              o0.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-              o0.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              *reinterpret_cast<uint4*>(args.D + rbase + col) = o0;
-            } else {
-              const uint4 ev = *reinterpret_cast<const uint4*>(args.Ein + rbase + col);
-              const uint4 gv = *reinterpret_cast<const uint4*>(args.Gin + rbase + col);
-              const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-              uint32_t de[4], dg[4];
+            uint4 o;
+            o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+            o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+            o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+            o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            *reinterpret_cast<uint4*>(args.D + rbase + col) = o;
+          }
+        }
+      } else if (EPI == EPI_GLU_BWD) {
+        // the chunk's saved e, g are requested before its TMEM load so the two latencies overlap
+#pragma unroll 1
+        for (int c = half * 4; c < half * 4 + 4; ++c) {
+          uint4 ec[4], gc[4];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                float f0, d0, f1, d1;
-                const float e0 = bf16_lo(ew[j]), e1 = bf16_hi(ew[j]);
-                const float g0 = bf16_lo(gw[j]), g1 = bf16_hi(gw[j]);
-                act_fg(args.act, e0, f0, d0);
-                act_fg(args.act, e1, f1, d1);
-                const float h0 = v[q * 8 + 2 * j], h1 = v[q * 8 + 2 * j + 1];
-                de[j] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
-                dg[j] = pack_bf16x2(h0 * f0, h1 * f1);
-              }
-              o0 = make_uint4(de[0], de[1], de[2], de[3]);
-              o1 = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-              *reinterpret_cast<uint4*>(args.dE + rbase + col) = o0;
-              *reinterpret_cast<uint4*>(args.dG + rbase + col) = o1;
+          for (int q = 0; q < 4; ++q) {
+            const int col = n0 + c * 32 + q * 8;
+            const bool in = row_ok && col < args.N;
+            ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
+            gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+          }
+          float v[32];
+          tmem_ld_32x32b_x32(trow + c * 32, v);
+          if (!row_ok) continue;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = n0 + c * 32 + q * 8;
+            if (col >= args.N) break;
+            const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
+            const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
+            uint32_t de[4], dg[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float f0, d0, f1, d1;
+              const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
+              const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
+              act_fg(args.act, e0, f0, d0);
+              act_fg(args.act, e1, f1, d1);
+              const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
+              de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
+              dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
             }
+            *reinterpret_cast<uint4*>(args.dE + rbase + col) = make_uint4(de[0], de[1], de[2], de[3]);
+            *reinterpret_cast<uint4*>(args.dG + rbase + col) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
           }
         }
       } else {  // EPI_GLU_FWD: columns [0,128) hold e, [128,256) hold g
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = half * 2; c < half * 2 + 2; ++c) {
           float e[32], g[32];
           tmem_ld_32x32b_x32(trow + c * 32, e);
           tmem_ld_32x32b_x32(trow + 128 + c * 32, g);
@@ -352,82 +409,97 @@ __global__ void __launch_bounds__(14 * 32, 1) gemm_nf4_kernel(const __grid_const
           for (int q = 0; q < 4; ++q) {
             const int col = n0 + c * 32 + q * 8;
             if (col >= args.N) break;
-            uint32_t ew[4], gw[4], hw[4];
+            uint32_t ewv[4], gwv[4], hwv[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float e0 = e[q * 8 + 2 * j], e1 = e[q * 8 + 2 * j + 1];
-              const float g0 = g[q * 8 + 2 * j], g1 = g[q * 8 + 2 * j + 1];
-              ew[j] = pack_bf16x2(e0, e1);
-              gw[j] = pack_bf16x2(g0, g1);
-              hw[j] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
+            for (int i = 0; i < 4; ++i) {
+              const float e0 = e[q * 8 + 2 * i], e1 = e[q * 8 + 2 * i + 1];
+              const float g0 = g[q * 8 + 2 * i], g1 = g[q * 8 + 2 * i + 1];
+              ewv[i] = pack_bf16x2(e0, e1);
+              gwv[i] = pack_bf16x2(g0, g1);
+              hwv[i] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
             }
-            *reinterpret_cast<uint4*>(args.E + rbase + col) = make_uint4(ew[0], ew[1], ew[2], ew[3]);
-            *reinterpret_cast<uint4*>(args.G + rbase + col) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
-            *reinterpret_cast<uint4*>(args.H + rbase + col) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(args.E + rbase + col) = make_uint4(ewv[0], ewv[1], ewv[2], ewv[3]);
+            *reinterpret_cast<uint4*>(args.G + rbase + col) = make_uint4(gwv[0], gwv[1], gwv[2], gwv[3]);
+            *reinterpret_cast<uint4*>(args.H + rbase + col) = make_uint4(hwv[0], hwv[1], hwv[2], hwv[3]);
           }
         }
+      }
+      // accumulator b may be overwritten once every epilogue warp of the pair is done with it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(leader(acc_empty0 + 8u * b));
+        else mbar_arrive(acc_empty0 + 8u * b);
       }
     }
   } else {
     // --------------------------------------------------- dequantisers ----
-    const int dq = (warp - 6) * 32 + lane;  // 0..255
+    const int dq = (warp - 2 - C::EPI_WARPS) * 32 + lane;  // 0..255
     constexpr int groups = 256 / C::NB;
     const int grp = dq / C::NB;
-    const int t = dq % C::NB;
-    for (int kb = grp; kb < nk; kb += groups) {
-      const int seg = kb >= args.nkb0 ? 1 : 0;
-      const int kl = kb - seg * args.nkb0;
-      const int rs = kb % C::RS;
-      if (!__all_sync(0xffffffffu, mbar_wait(rfull_bar(rs), (kb / C::RS) & 1, args.status))) break;
-      const uint8_t* rc = sgen + C::OFF_RC + rs * C::RC_BYTES;
-      const float* ra = reinterpret_cast<const float*>(sgen + C::OFF_RA + rs * C::RA_BYTES);
-      uint4 w0, w1;
-      float amax;
-      int r = 0, cchunk = 0;
-      if (MODE == MODE_BWD) {
-        // raw tile: 64 rows x (BNC/2) bytes, swizzled 128B (CG=1) or 64B (CG=2)
-        r = t & 63;
-        cchunk = t >> 6;
-        constexpr int RB = C::BNC / 2;
-        constexpr int SHIFT = (RB == 128) ? 0 : 1;
-        constexpr int MASK = (RB == 128) ? 7 : 3;
-        const int x = (r >> SHIFT) & MASK;
-        w0 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk) ^ x) << 4));
-        w1 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk + 1) ^ x) << 4));
-        amax = ra[r * 4 + cchunk + (CG == 2 ? 2 * (int)rank : 0)];
-      } else {
-        // raw tile: NB rows x 32 bytes, 32B swizzle
-        r = t;
-        const int x = (r >> 2) & 1;
-        w0 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((0 ^ x) << 4));
-        w1 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((1 ^ x) << 4));
-        amax = ra[r * 4 + (kl & 3)];
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(rempty_bar(rs));
+    const int tq = dq % C::NB;
+    int j = 0;
+    bool ok = true;
+    for (int t = cluster; t < total_tiles && ok; t += clusters) {
+      for (int kb = 0; kb < nk; ++kb, ++j) {
+        if (j % groups != grp) continue;
+        const int seg = kb >= args.nkb0 ? 1 : 0;
+        const int kl = kb - seg * args.nkb0;
+        const int rs = j % C::RS;
+        ok = __all_sync(0xffffffffu, mbar_wait(rfull_bar(rs), (j / C::RS) & 1, args.status));
+        if (!ok) break;
+        const uint8_t* rc = sgen + C::OFF_RC + rs * C::RC_BYTES;
+        const float* ra = reinterpret_cast<const float*>(sgen + C::OFF_RA + rs * C::RA_BYTES);
+        uint4 w0, w1;
+        float amax;
+        int r = 0, cchunk = 0;
+        if (MODE == MODE_BWD) {
+          // raw tile: 64 rows x (BNC/2) bytes, swizzled 128B (CG=1) or 64B (CG=2)
+          r = tq & 63;
+          cchunk = tq >> 6;
+          constexpr int RB = C::BNC / 2;
+          constexpr int SHIFT = (RB == 128) ? 0 : 1;
+          constexpr int MASK = (RB == 128) ? 7 : 3;
+          const int x = (r >> SHIFT) & MASK;
+          w0 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk) ^ x) << 4));
+          w1 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk + 1) ^ x) << 4));
+          amax = ra[r * 4 + cchunk + (CG == 2 ? 2 * (int)rank : 0)];
+        } else {
+          // raw tile: NB rows x 32 bytes, 32B swizzle
+          r = tq;
+          const int x = (r >> 2) & 1;
+          w0 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((0 ^ x) << 4));
+          w1 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((1 ^ x) << 4));
+          amax = ra[r * 4 + (kl & 3)];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(rempty_bar(rs));
 
-      const int s = kb % C::S;
-      if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((kb / C::S) & 1) ^ 1, args.status))) break;
-      uint32_t tl[4], th[4];
-      nf4_block_table(amax, tl, th);
-      uint8_t* bt = sgen + C::OFF_B + s * C::B_BYTES;
-      uint8_t* dst = (MODE == MODE_BWD) ? bt + cchunk * 8192 + (r >> 3) * 1024 + (r & 7) * 128
-                                        : bt + (r >> 3) * 1024 + (r & 7) * 128;
-      const int x7 = r & 7;
-      const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const int s = j % C::S;
+        ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status));
+        if (!ok) break;
+        uint32_t tlo[4], thi[4];
+        nf4_block_table(amax, tlo, thi);
+        uint8_t* bt = sgen + C::OFF_B + s * C::B_BYTES;
+        uint8_t* dst = (MODE == MODE_BWD) ? bt + cchunk * 8192 + (r >> 3) * 1024 + (r & 7) * 128
+                                          : bt + (r >> 3) * 1024 + (r & 7) * 128;
+        const int x7 = r & 7;
+        const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(dst + ((j ^ x7) << 4)) = nf4_decode8(wv[j], tl, th);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (CG == 2) mbar_arrive_cluster(leader(full_bar(s)));
-        else mbar_arrive(full_bar(s));
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4*>(dst + ((i ^ x7) << 4)) = nf4_decode8(wv[i], tlo, thi);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 2) mbar_arrive_cluster(leader(full_bar(s)));
+          else mbar_arrive(full_bar(s));
+        }
       }
     }
   }
 
   // ------------------------------------------------------------ teardown --
+  __syncwarp();  // lanes that skipped a role's single-thread loop wait for it here
   tc_fence_before();
   if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   if (warp == 1) {
@@ -441,17 +513,14 @@ template <int MODE, int EPI, int CG>
 static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaStream_t stream) {
   using C = GemmCfg<MODE, CG>;
   auto kern = gemm_nf4_kernel<MODE, EPI, CG>;
-  static bool configured = false;  // per instantiation; attribute set once per process
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int resident[64] = {0};  // co-resident CTAs (multiple of CG) per device, per instantiation
   const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
   const int n_tiles = (args.N + bn_out - 1) / bn_out;
   const int m_tiles = (args.M + C::BM * CG - 1) / (C::BM * CG);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * n_tiles * CG), 1, 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -462,6 +531,26 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaSt
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!resident[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    int n = sms / CG;
+    if (CG > 1) {
+      cfg.gridDim = dim3(static_cast<unsigned>(sms - sms % CG), 1, 1);
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0 && clusters < n)
+        n = clusters;
+      cudaGetLastError();
+    }
+    resident[dev] = n * CG;
+  }
+  const int total = m_tiles * n_tiles;
+  const int ctas = (total * CG < resident[dev]) ? total * CG : resident[dev];
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
   return cudaLaunchKernelEx(&cfg, kern, maps, args);
 }
 
@@ -479,11 +568,6 @@ cudaError_t launch_gemm_nf4(int mode, int epi, int cg, const GemmMaps& maps, con
   QL_CASE(MODE_BWD, EPI_GLU_BWD, 2)
 #undef QL_CASE
   return cudaErrorInvalidValue;
-}
-
-int gemm_nf4_smem_bytes(int mode, int cg) {
-  if (mode == MODE_BWD) return cg == 1 ? GemmCfg<MODE_BWD, 1>::SMEM_BYTES : GemmCfg<MODE_BWD, 2>::SMEM_BYTES;
-  return cg == 1 ? GemmCfg<MODE_FWD, 1>::SMEM_BYTES : GemmCfg<MODE_FWD, 2>::SMEM_BYTES;
 }
 
 }  // namespace ql

@@ -52,8 +52,10 @@ QL_DEV void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 // Arrive on a barrier given by its shared::cluster address (may be a peer CTA's).
+// Default semantics (release at CTA scope): the data it publishes is this CTA's
+// shared memory, made visible to the async proxy by fence.proxy.async first.
 QL_DEV void mbar_arrive_cluster(uint32_t cbar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
 }
 QL_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -70,23 +72,11 @@ QL_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-QL_DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait.  Returns false (and flags the status word) on timeout, or if
 // another thread of the grid already flagged a timeout.
-template <bool kClusterScope = false>
+template <bool kUnused = false>
 QL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
-  auto probe = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  auto probe = [&]() { return mbar_try_wait(bar, parity); };
   if (probe()) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
