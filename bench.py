@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cta-group", type=int, default=2)
+    ap.add_argument("--tiles", type=int, default=2, help="GEMM tile configuration (1, 2 or 3)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override M (tokens per GPU) for small profiling cases; 0 = the workload's M")
     return ap.parse_args()
@@ -237,7 +237,7 @@ def run_ours(args, wl):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     ops.lib()
-    ops.qlora_set_cta_group(args.cta_group)
+    ops.qlora_set_tile_config(args.tiles)
     M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
 
     # Inputs: same seeded recipe as the tests; each rank draws its own batch.
@@ -376,7 +376,7 @@ def run_ours(args, wl):
         "frac_of_bf16_peak_sustained": value / world / pk["bf16_sustained"],
         "config": {"workload": args.workload, "M_per_gpu": M, "d": d, "h": h, "r": r, "act": act,
                    "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
-                   "cta_group": args.cta_group, "l2": L2_NOTE},
+                   "gemm_tiles": ops.TILE_CONFIGS[args.tiles], "l2": L2_NOTE},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": launches,

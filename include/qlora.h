@@ -173,10 +173,12 @@ QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t 
 /* Human-readable name of a status code (static string). */
 QLORA_API const char* qlora_status_string(qlora_status status);
 
-/* Selects the tensor-core tile shape of the NF4 GEMMs: 1 = one CTA per
- * 128-row tile, 2 = a CTA pair (cta_group::2) per 256-row tile (default).
- * Returns the previous value.  Not thread-safe. */
-QLORA_API int32_t qlora_set_cta_group(int32_t cta_group);
+/* Selects the tensor-core tile shape of the NF4 GEMMs (all give the same
+ * results): 1 = one CTA per 128 x 256 tile, 2 = a CTA pair (cta_group::2)
+ * per 256 x 256 tile (default), 3 = a CTA pair per 512 x 128 tile whose
+ * dequantised weight tile feeds two M = 256 MMAs.  Invalid values are
+ * ignored.  Returns the previous value.  Not thread-safe. */
+QLORA_API int32_t qlora_set_tile_config(int32_t tiles);
 
 /* Kernel tracing (host side, not thread-safe).  While enabled, every kernel
  * launch of the library is bracketed by CUDA events on its stream. */

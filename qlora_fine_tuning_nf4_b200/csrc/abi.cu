@@ -20,8 +20,9 @@ namespace ql {
 cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st);
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t numel, bf16* out,
                                   cudaStream_t st, int num_sms);
-cudaError_t launch_gemm_nf4(int mode, int epi, int cg, const GemmMaps& maps, const GemmArgs& args,
+cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
+int gemm_nf4_b_cols_per_cta(int tiles);
 cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1, float* part,
                            int M, int K, int splits, int kb_per_split, int* status, cudaStream_t st);
 cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, float* part, int M, int N, int splits,
@@ -54,7 +55,7 @@ struct TraceRec {
 std::vector<TraceRec> g_recs;
 std::vector<cudaEvent_t> g_pool;
 size_t g_pool_used = 0;
-int32_t g_cta_group = 2;
+int32_t g_tiles = 2;  // GEMM tile configuration (see qlora_set_tile_config)
 
 cudaEvent_t pool_event() {
   if (g_pool_used == g_pool.size()) {
@@ -245,21 +246,25 @@ ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0.f}, ReduceOut c
   return o;
 }
 
-// NF4 weight maps for the GEMM B operand (K-major for forward, MN-major for dX).
-bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const qlora_nf4& w, bool bwd, int cg) {
+// NF4 weight maps for the GEMM B operand (K-major for forward, MN-major for dX);
+// boxes follow the number of B columns each CTA dequantises (bnc).
+bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const qlora_nf4& w, bool bwd, int bnc) {
   const int64_t N = w.n_out, K = w.k_in;
   if (!bwd) {
-    return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, 32, 128,
+    const int rows = bnc < 128 ? bnc : 128;
+    return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, 32, rows,
                     CU_TENSOR_MAP_SWIZZLE_32B) &&
-           make_map(absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.absmax, K / 64, N, K / 64, 4, 128,
+           make_map(absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.absmax, K / 64, N, K / 64, 4, rows,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   }
-  const int rb = 128 / cg;  // bytes of codes per W row per CTA tile
-  return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, rb, 64,
-                  cg == 1 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
+  const int rb = bnc / 2;  // bytes of codes per W row per CTA tile
+  const CUtensorMapSwizzle swz = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                           : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  return make_map(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.codes, K / 2, N, K / 2, rb, 64, swz) &&
          make_map(absmax, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.absmax, K / 64, N, K / 64, 4, 64,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
+int lora_rows_box(int bnc) { return bnc < 128 ? bnc : 128; }
 
 qlora_status check_linear(const qlora_lora_linear* lin) {
   if (!lin || !lin->w.codes || !lin->w.absmax || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
@@ -275,12 +280,13 @@ qlora_status check_linear(const qlora_lora_linear* lin) {
 // Y-side GEMM launch helpers -------------------------------------------------
 qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, const bf16* XAs, bf16* Y, int* status,
                       cudaStream_t st) {
-  const int cg = g_cta_group;
+  const int tiles = g_tiles;
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int64_t K = lin.w.k_in, N = lin.w.n_out;
   if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin.w, false, cg)) return QLORA_ERR_CUDA;
+  if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin.w, false, bnc)) return QLORA_ERR_CUDA;
   if (!map_bf16(&maps.la[0], XAs, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&maps.lb[0], lin.B, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   maps.a[1] = maps.a[0];
@@ -299,7 +305,7 @@ qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, co
   a.D = Y;
   a.status = status;
   KScope k(K_GEMM_FWD, st);
-  return cuda_status(launch_gemm_nf4(MODE_FWD, EPI_STORE, cg, maps, a, st));
+  return cuda_status(launch_gemm_nf4(MODE_FWD, EPI_STORE, tiles, maps, a, st));
 }
 
 }  // namespace
@@ -327,9 +333,9 @@ qlora_status qlora_nf4_codebook(float out[16]) {
   return QLORA_OK;
 }
 
-int32_t qlora_set_cta_group(int32_t cg) {
-  const int32_t prev = g_cta_group;
-  if (cg == 1 || cg == 2) g_cta_group = cg;
+int32_t qlora_set_tile_config(int32_t tiles) {
+  const int32_t prev = g_tiles;
+  if (tiles >= 1 && tiles <= 3) g_tiles = tiles;
   return prev;
 }
 
@@ -406,7 +412,8 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
   if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int cg = g_cta_group;
+  const int tiles = g_tiles;
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   char* w = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(w);
   bf16* sG = reinterpret_cast<bf16*>(w + 256);
@@ -422,9 +429,10 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, N, M, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin->w, true, bnc)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[0], sG, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
@@ -440,7 +448,7 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     a.D = reinterpret_cast<bf16*>(dX);
     a.status = status;
     KScope k(K_GEMM_BWD, st);
-    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, cg, maps, a, st));
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
   }
   // dA = X^T (s G)
@@ -511,7 +519,8 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int cg = g_cta_group;
+  const int tiles = g_tiles;
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   MlpWs w = carve_mlp(ws, M, h);
   const bf16* x = reinterpret_cast<const bf16*>(X);
   bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
@@ -533,8 +542,8 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, false, cg)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, false, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, false, bnc)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, false, bnc)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[0], xags, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], xaus, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], gate->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -552,7 +561,7 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.H = reinterpret_cast<bf16*>(sv->H);
     a.status = w.status;
     KScope k(K_GEMM_GLU_FWD, st);
-    s = cuda_status(launch_gemm_nf4(MODE_FWD_GLU, EPI_GLU_FWD, cg, maps, a, st));
+    s = cuda_status(launch_gemm_nf4(MODE_FWD_GLU, EPI_GLU_FWD, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
   }
   // HA_d = H A_d
@@ -585,7 +594,8 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int cg = g_cta_group;
+  const int tiles = g_tiles;
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   MlpWs w = carve_mlp(ws, M, h);
   bf16* sGd = w.v0;
   // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
@@ -598,9 +608,10 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], down->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], down->w, true, bnc)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[0], sGd, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
@@ -620,7 +631,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.dG = w.dG;
     a.status = w.status;
     KScope k(K_GEMM_GLU_BWD, st);
-    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_GLU_BWD, cg, maps, a, st));
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_GLU_BWD, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
   }
   // 3. dA_d = H^T (s_d G_d)
@@ -642,12 +653,14 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, true, cg)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, true, cg)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, true, bnc)) return QLORA_ERR_CUDA;
+    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, true, bnc)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[0], w.gu, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], w.gu + 16, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[1], up->A, 16, d, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
+    if (!map_bf16(&maps.lb[1], up->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     a.M = (int)M;
@@ -659,7 +672,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.D = reinterpret_cast<bf16*>(dX);
     a.status = w.status;
     KScope k(K_GEMM_BWD, st);
-    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, cg, maps, a, st));
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
   }
   // 6. [dA_g | dA_u] = X^T [sG_g | sG_u]

@@ -94,46 +94,64 @@ QL_DEV void act_fg(int act, float e, float& f, float& g) {
   }
 }
 
-template <int MODE, int CG>
+// Tile configuration.  A CTA owns MH accumulators of 128 rows (TMEM lanes) x
+// BNT columns; with cta_group::2 a pair of CTAs issues each MMA with M = 256
+// and each CTA supplies BNC = BNT / 2 columns of the dequantised B operand.
+//   (CG, MH) = (1, 1): 128 x 256 per CTA
+//   (CG, MH) = (2, 1): 256 x 256 per pair
+//   (CG, MH) = (2, 2): 512 x 128 per pair -- each dequantised B tile feeds two
+//                      M = 256 MMAs, halving the dequantisation per MMA.
+template <int MODE, int CG, int MH>
 struct GemmCfg {
-  static constexpr int BM = 128;                 // rows per CTA (TMEM lanes)
-  static constexpr int BNT = 256;                // MMA N (whole pair)
+  static constexpr int BM = 128;                 // rows per CTA per M-half (TMEM lanes)
+  static constexpr int BNT = 256 / MH;           // MMA N (whole pair)
   static constexpr int BNC = BNT / CG;           // B columns produced per CTA
   static constexpr int BK = 64;                  // reduction block (one NF4 block, one 128B row)
   static constexpr int NB = BNC;                 // NF4 blocks dequantised per CTA per k-block
-  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int BOXR = BNC < 128 ? BNC : 128;  // rows per TMA box of codes / absmax / LoRA rows
+  static constexpr int A_TILE = BM * BK * 2;
+  static constexpr int A_BYTES = MH * A_TILE;
   static constexpr int B_BYTES = BNC * BK * 2;
   static constexpr int RC_BYTES = NB * 32;
   static constexpr int RA_BYTES = (MODE == MODE_BWD) ? 64 * 16 : BNC * 16;
-  static constexpr int S = (CG == 1) ? 3 : 5;    // operand stages
-  static constexpr int RS = (CG == 1) ? 4 : 6;   // raw stages
-  static constexpr int LA_BYTES = BM * 16 * 2;
-  static constexpr int LB_BYTES = 8192;
+  static constexpr int S = (CG == 1) ? 3 : (MH == 1 ? 5 : 4);   // operand stages
+  static constexpr int RS = (CG == 1) ? 4 : (MH == 1 ? 6 : 8);  // raw stages
+  static constexpr int LA_BYTES = BM * 16 * 2;   // one LoRA left operand tile (128 rows x 16)
+  static constexpr int LBOP = BNC * 32;          // one LoRA right operand (BNC x 16 bf16)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + S * A_BYTES;
   static constexpr int OFF_RC = OFF_B + S * B_BYTES;
   static constexpr int OFF_RA = OFF_RC + RS * RC_BYTES;
   static constexpr int OFF_LA = OFF_RA + RS * RA_BYTES;
-  static constexpr int OFF_LB = OFF_LA + 2 * LA_BYTES;
-  static constexpr int OFF_BAR = OFF_LB + 2 * LB_BYTES;
+  static constexpr int OFF_LB = OFF_LA + MH * 2 * LA_BYTES;
+  static constexpr int OFF_BAR = OFF_LB + 2 * LBOP;
   static constexpr int NBAR = 2 * S + 2 * RS + 7;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static constexpr int EPI_WARPS = 8;            // two per TMEM lane quadrant
   static constexpr int DQ_WARPS = 8;
-  static constexpr int THREADS = (2 + EPI_WARPS + DQ_WARPS) * 32;
-  static constexpr int TMEM_COLS = 512;          // two 256-column accumulators
+  static constexpr int EPI_WARP0 = 3;            // warps 0: A/LoRA TMA, 1: MMA, 2: raw-code TMA
+  static constexpr int DQ_WARP0 = EPI_WARP0 + EPI_WARPS;
+  static constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
+  static constexpr int TMEM_COLS = 512;          // two accumulators of MH x BNT = 256 columns
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0, "1024B alignment of swizzled regions");
+  static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0 && OFF_LB % 1024 == 0, "1024B alignment");
+  static_assert(256 % NB == 0 && NB % 64 == 0, "dequantiser mapping");
 };
 
+// Roles: warp 0 issues the TMA loads of the A operand and the LoRA operands,
+// warp 1 allocates TMEM and (leader CTA, one thread) issues tcgen05.mma,
+// warp 2 streams the raw NF4 codes + absmax, running up to RS k-blocks ahead
+// of the dequantisers independently of the MMA's progress, warps 3-10 drain
+// the accumulators (epilogue), warps 11-18 dequantise.
+//
 // Persistent kernel: each CTA (or CTA pair) walks the output tiles
 // t = cluster, cluster + clusters, ... (N tiles fastest).  Every role iterates
 // the same tile sequence; j counts 64-wide reduction blocks across tiles and
 // indexes the rings, so barrier phases follow from j and the tile counter.
-template <int MODE, int EPI, int CG>
-__global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
+template <int MODE, int EPI, int CG, int MH>
+__global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
     gemm_nf4_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
-  using C = GemmCfg<MODE, CG>;
+  using C = GemmCfg<MODE, CG, MH>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -142,9 +160,10 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
 
-  const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
+  const int bn_out = (EPI == EPI_GLU_FWD) ? C::BNT / 2 : C::BNT;  // output columns per tile
+  const int bm_pair = C::BM * CG * MH;                            // output rows per tile
   const int n_tiles = (args.N + bn_out - 1) / bn_out;
-  const int m_tiles = (args.M + C::BM * CG - 1) / (C::BM * CG);
+  const int m_tiles = (args.M + bm_pair - 1) / bm_pair;
   const int total_tiles = n_tiles * m_tiles;
   const int cluster = blockIdx.x / CG;
   const int clusters = gridDim.x / CG;
@@ -163,6 +182,19 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
   const uint32_t drain_bar = lora_full + 48u;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + C::OFF_BAR + C::NBAR * 8);
 
+  // Gated forward: the pair tile's B columns are [gate | up].  LoRA operand i
+  // (0 = gate, 1 = up) is loaded into the 64-column chunks of this CTA that
+  // belong to it; the other chunks stay zero, so both LoRA MMAs span all BNT
+  // columns and each only adds to its own half.
+  auto glu_chunk_is_gate = [&](int c) { return static_cast<int>(rank) * C::BNC + c * 64 < C::BNT / 2; };
+  if (EPI == EPI_GLU_FWD) {
+    for (int c = 0; c < C::BNC / 64; ++c) {
+      const int zero_op = glu_chunk_is_gate(c) ? 1 : 0;
+      uint4* z = reinterpret_cast<uint4*>(sgen + C::OFF_LB + zero_op * C::LBOP + c * 2048);
+      for (int i = threadIdx.x; i < 2048 / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       mbar_init(full_bar(s), 1 + CG * (C::NB / 32));
@@ -192,10 +224,12 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
 
   // shared::cluster address of a barrier in the pair's leader CTA
   auto leader = [&](uint32_t bar) { return (CG == 2) ? mapa_shared(bar, 0) : bar; };
-  auto tile_coords = [&](int t, int& m0, int& n0) {
-    m0 = (t / n_tiles) * (C::BM * CG) + static_cast<int>(rank) * C::BM;
+  // first output row of M-half h of tile t for this CTA, and the tile's first column
+  auto tile_coords = [&](int t, int& mb, int& n0) {
+    mb = (t / n_tiles) * bm_pair + static_cast<int>(rank) * C::BM;
     n0 = (t % n_tiles) * bn_out;
   };
+  auto half_row = [&](int mb, int h) { return mb + h * C::BM * CG; };
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -210,18 +244,62 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
         if constexpr (CG == 2) tma_load_2d_pair(dst, m, leader(bar_local), x, y);
         else tma_load_2d(dst, m, bar_local, x, y);
       };
-      int lora_bytes = args.lora * C::LA_BYTES;
-      if (MODE == MODE_FWD) lora_bytes += C::BNC * 32;
-      if (MODE == MODE_FWD_GLU) lora_bytes += 2 * (128 / CG) * 32;
-      if (MODE == MODE_BWD) lora_bytes += args.lora * C::BNC * 32;
+      int lora_bytes = MH * args.lora * C::LA_BYTES;
+      if (MODE == MODE_FWD || MODE == MODE_FWD_GLU) lora_bytes += C::LBOP;
+      if (MODE == MODE_BWD) lora_bytes += args.lora * C::LBOP;
       int j = 0, tl = 0;
       for (int t = cluster; t < total_tiles && ok; t += clusters, ++tl) {
-        int m0, n0;
-        tile_coords(t, m0, n0);
+        int mb, n0;
+        tile_coords(t, mb, n0);
         for (int kb = 0; kb < nk; ++kb, ++j) {
           const int seg = kb >= args.nkb0 ? 1 : 0;
           const int kl = kb - seg * args.nkb0;
-          // raw NF4 codes + absmax for the dequantisers (local barrier)
+          // A operand tiles (complete on the leader's full barrier)
+          const int s = j % C::S;
+          ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
+          if (!ok) break;
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
+          for (int h = 0; h < MH; ++h)
+            load(sbase + C::OFF_A + s * C::A_BYTES + h * C::A_TILE, &maps.a[seg], full_bar(s), kl * 64,
+                 half_row(mb, h));
+        }
+        if (!ok || args.lora == 0) continue;
+        // LoRA operands of this tile (single buffer, released by the MMA's commit)
+        ok = mbar_wait(lora_empty, (tl & 1) ^ 1, args.status);
+        if (!ok) break;
+        if (rank == 0) mbar_arrive_expect_tx(lora_full, lora_bytes * CG);
+        for (int h = 0; h < MH; ++h)
+          for (int i = 0; i < args.lora; ++i)
+            load(sbase + C::OFF_LA + (h * 2 + i) * C::LA_BYTES, &maps.la[i], lora_full, 0, half_row(mb, h));
+        if (MODE == MODE_FWD) {
+          for (int c = 0; c < C::BNC / 64; ++c)
+            load(sbase + C::OFF_LB + c * 2048, &maps.lb[0], lora_full, n0 + (int)rank * C::BNC + c * 64, 0);
+        } else if (MODE == MODE_FWD_GLU) {
+          for (int c = 0; c < C::BNC / 64; ++c) {
+            const int p = (int)rank * C::BNC + c * 64;
+            const int op = glu_chunk_is_gate(c) ? 0 : 1;
+            load(sbase + C::OFF_LB + op * C::LBOP + c * 2048, &maps.lb[op], lora_full,
+                 n0 + (op ? p - C::BNT / 2 : p), 0);
+          }
+        } else {
+          for (int i = 0; i < args.lora; ++i)
+            for (int bx = 0; bx < C::BNC / C::BOXR; ++bx)
+              load(sbase + C::OFF_LB + i * C::LBOP + bx * C::BOXR * 32, &maps.lb[i], lora_full, 0,
+                   n0 + (int)rank * C::BNC + bx * C::BOXR);
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ raw-code producer --
+    if (lane == 0) {
+      bool ok = true;
+      int j = 0;
+      for (int t = cluster; t < total_tiles && ok; t += clusters) {
+        int mb, n0;
+        tile_coords(t, mb, n0);
+        for (int kb = 0; kb < nk; ++kb, ++j) {
+          const int seg = kb >= args.nkb0 ? 1 : 0;
+          const int kl = kb - seg * args.nkb0;
           const int rs = j % C::RS;
           ok = mbar_wait(rempty_bar(rs), ((j / C::RS) & 1) ^ 1, args.status);
           if (!ok) break;
@@ -233,41 +311,16 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
             tma_load_2d(rc, &maps.codes[seg], rfull_bar(rs), kw0 / 2, kl * 64);
             tma_load_2d(ra, &maps.absmax[seg], rfull_bar(rs), (kw0 / 64) & ~3, kl * 64);
           } else {
-            for (int h = 0; h < C::BNC / 128; ++h) {
-              int src = 0, row = n0 + (int)rank * C::BNC + h * 128;
+            for (int bx = 0; bx < C::BNC / C::BOXR; ++bx) {
+              const int p = (int)rank * C::BNC + bx * C::BOXR;  // first B row of the box in the pair tile
+              int src = 0, row = n0 + p;
               if (MODE == MODE_FWD_GLU) {
-                src = (CG == 1) ? h : (int)rank;
-                row = n0;
+                src = p < C::BNT / 2 ? 0 : 1;
+                row = n0 + (src ? p - C::BNT / 2 : p);
               }
-              tma_load_2d(rc + h * 4096, &maps.codes[src], rfull_bar(rs), kl * 32, row);
-              tma_load_2d(ra + h * 2048, &maps.absmax[src], rfull_bar(rs), kl & ~3, row);
+              tma_load_2d(rc + bx * C::BOXR * 32, &maps.codes[src], rfull_bar(rs), kl * 32, row);
+              tma_load_2d(ra + bx * C::BOXR * 16, &maps.absmax[src], rfull_bar(rs), kl & ~3, row);
             }
-          }
-          // A operand tile (completes on the leader's full barrier)
-          const int s = j % C::S;
-          ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
-          if (!ok) break;
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
-          load(sbase + C::OFF_A + s * C::A_BYTES, &maps.a[seg], full_bar(s), kl * 64, m0);
-        }
-        if (!ok || args.lora == 0) continue;
-        // LoRA operands of this tile (single buffer, released by the MMA's commit)
-        ok = mbar_wait(lora_empty, (tl & 1) ^ 1, args.status);
-        if (!ok) break;
-        if (rank == 0) mbar_arrive_expect_tx(lora_full, lora_bytes * CG);
-        for (int i = 0; i < args.lora; ++i) {
-          load(sbase + C::OFF_LA + i * C::LA_BYTES, &maps.la[i], lora_full, 0, m0);
-          if (MODE == MODE_FWD) {
-            for (int c = 0; c < C::BNC / 64; ++c)
-              load(sbase + C::OFF_LB + c * 2048, &maps.lb[0], lora_full, n0 + (int)rank * C::BNC + c * 64, 0);
-          } else if (MODE == MODE_FWD_GLU) {
-            for (int c = 0; c < (128 / CG) / 64; ++c)
-              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 2048, &maps.lb[i], lora_full,
-                   n0 + (int)rank * (128 / CG) + c * 64, 0);
-          } else {
-            for (int c = 0; c < C::BNC / 128; ++c)
-              load(sbase + C::OFF_LB + i * C::LB_BYTES + c * 4096, &maps.lb[i], lora_full, 0,
-                   n0 + (int)rank * C::BNC + c * 128);
           }
         }
       }
@@ -277,45 +330,45 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
     if (rank == 0 && lane == 0) {
       bool ok = true;
       const uint32_t idesc = idesc_bf16(C::BM * CG, C::BNT, false, MODE == MODE_BWD);
+      const uint32_t idesc_lora = idesc_bf16(C::BM * CG, C::BNT, false, MODE != MODE_BWD);
       int j = 0, tl = 0;
       for (int t = cluster; t < total_tiles && ok; t += clusters, ++tl) {
         const int b = tl & 1;
-        ok = mbar_wait<CG == 2>(acc_empty0 + 8u * b, ((tl >> 1) & 1) ^ 1, args.status);
+        ok = mbar_wait(acc_empty0 + 8u * b, ((tl >> 1) & 1) ^ 1, args.status);
         if (!ok) break;
         tc_fence_after();
         const uint32_t acc = tmem + b * 256;
         for (int kb = 0; kb < nk; ++kb, ++j) {
           const int s = j % C::S;
-          ok = mbar_wait<CG == 2>(full_bar(s), (j / C::S) & 1, args.status);
+          ok = mbar_wait(full_bar(s), (j / C::S) & 1, args.status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a = sbase + C::OFF_A + s * C::A_BYTES;
           const uint32_t bs = sbase + C::OFF_B + s * C::B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, QL_SWZ_128B);
             const uint64_t bd = (MODE == MODE_BWD) ? smem_desc(bs + kk * 2048, 8192, 1024, QL_SWZ_128B)
                                                    : smem_desc(bs + kk * 32, 16, 1024, QL_SWZ_128B);
-            umma_bf16<CG>(acc, ad, bd, idesc, (kb | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < MH; ++h) {
+              const uint64_t ad = smem_desc(a + h * C::A_TILE + kk * 32, 16, 1024, QL_SWZ_128B);
+              umma_bf16<CG>(acc + h * C::BNT, ad, bd, idesc, (kb | kk) != 0);
+            }
           }
           umma_commit<CG>(empty_bar(s));
         }
         if (!ok) break;
         if (args.lora > 0) {
-          ok = mbar_wait<CG == 2>(lora_full, tl & 1, args.status);
+          ok = mbar_wait(lora_full, tl & 1, args.status);
           if (!ok) break;
           tc_fence_after();
-          for (int i = 0; i < args.lora; ++i) {
-            const uint64_t ad = smem_desc(sbase + C::OFF_LA + i * C::LA_BYTES, 16, 256, QL_SWZ_32B);
-            if (MODE == MODE_FWD) {
-              const uint64_t bd = smem_desc(sbase + C::OFF_LB, 2048, 1024, QL_SWZ_128B);
-              umma_bf16<CG>(acc, ad, bd, idesc_bf16(C::BM * CG, 256, false, true), 1);
-            } else if (MODE == MODE_FWD_GLU) {
-              const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 2048, 1024, QL_SWZ_128B);
-              umma_bf16<CG>(acc + i * 128, ad, bd, idesc_bf16(C::BM * CG, 128, false, true), 1);
-            } else {
-              const uint64_t bd = smem_desc(sbase + C::OFF_LB + i * C::LB_BYTES, 16, 256, QL_SWZ_32B);
-              umma_bf16<CG>(acc, ad, bd, idesc_bf16(C::BM * CG, 256, false, false), 1);
+          for (int h = 0; h < MH; ++h) {
+            for (int i = 0; i < args.lora; ++i) {
+              const uint64_t ad = smem_desc(sbase + C::OFF_LA + (h * 2 + i) * C::LA_BYTES, 16, 256, QL_SWZ_32B);
+              const uint64_t bd = (MODE == MODE_BWD)
+                                      ? smem_desc(sbase + C::OFF_LB + i * C::LBOP, 16, 256, QL_SWZ_32B)
+                                      : smem_desc(sbase + C::OFF_LB + i * C::LBOP, 2048, 1024, QL_SWZ_128B);
+              umma_bf16<CG>(acc + h * C::BNT, ad, bd, idesc_lora, 1);
             }
           }
           umma_commit<CG>(lora_empty);
@@ -326,84 +379,84 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
       umma_commit<CG>(drain_bar);
       mbar_wait(drain_bar, 0, args.status);
     }
-  } else if (warp < 2 + C::EPI_WARPS) {
+  } else if (warp < C::DQ_WARP0) {
     // ------------------------------------------------------ epilogue -----
-    const int ew = warp - 2;            // 0..7
+    const int ew = warp - C::EPI_WARP0;  // 0..7
     const int lg = warp & 3;            // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;           // which half of the tile's columns
+    const int half = ew >> 2;           // which half of the tile's column chunks
     const int row = lg * 32 + lane;
     int tl = 0;
     for (int t = cluster; t < total_tiles; t += clusters, ++tl) {
-      int m0, n0;
-      tile_coords(t, m0, n0);
+      int mb, n0;
+      tile_coords(t, mb, n0);
       const int b = tl & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full0 + 8u * b, (tl >> 1) & 1, args.status))) break;
       tc_fence_after();
-      const uint32_t trow = tmem + b * 256 + (static_cast<uint32_t>(lg * 32) << 16);
-      const int grow = m0 + row;
-      const bool row_ok = grow < args.M;
-      const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
-      if (EPI == EPI_STORE) {
+      const uint32_t tacc = tmem + b * 256 + (static_cast<uint32_t>(lg * 32) << 16);
+      if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
+        constexpr int CPH = C::BNT / 32;  // 32-column chunks per M-half
 #pragma unroll 1
-        for (int c = half * 4; c < half * 4 + 4; ++c) {
-          float v[32];
-          tmem_ld_32x32b_x32(trow + c * 32, v);
-          if (!row_ok) continue;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = n0 + c * 32 + q * 8;
-            if (col >= args.N) break;
-            uint4 o;
-            o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-            *reinterpret_cast<uint4*>(args.D + rbase + col) = o;
-          }
-        }
-      } else if (EPI == EPI_GLU_BWD) {
-        // the chunk's saved e, g are requested before its TMEM load so the two latencies overlap
-#pragma unroll 1
-        for (int c = half * 4; c < half * 4 + 4; ++c) {
+        for (int it = half * 4; it < half * 4 + 4; ++it) {
+          const int h = it / CPH, c = it % CPH;
+          const int grow = half_row(mb, h) + row;
+          const bool row_ok = grow < args.M;
+          const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
           uint4 ec[4], gc[4];
+          if (EPI == EPI_GLU_BWD) {
+            // the chunk's saved e, g are requested before its TMEM load so the two latencies overlap
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = n0 + c * 32 + q * 8;
-            const bool in = row_ok && col < args.N;
-            ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
-            gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+            for (int q = 0; q < 4; ++q) {
+              const int col = n0 + c * 32 + q * 8;
+              const bool in = row_ok && col < args.N;
+              ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
+              gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+            }
           }
           float v[32];
-          tmem_ld_32x32b_x32(trow + c * 32, v);
+          tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, v);
           if (!row_ok) continue;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int col = n0 + c * 32 + q * 8;
             if (col >= args.N) break;
-            const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
-            const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
-            uint32_t de[4], dg[4];
+            if (EPI == EPI_STORE) {
+              uint4 o;
+              o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              *reinterpret_cast<uint4*>(args.D + rbase + col) = o;
+            } else {
+              const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
+              const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
+              uint32_t de[4], dg[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float f0, d0, f1, d1;
-              const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
-              const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
-              act_fg(args.act, e0, f0, d0);
-              act_fg(args.act, e1, f1, d1);
-              const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
-              de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
-              dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
+              for (int i = 0; i < 4; ++i) {
+                float f0, d0, f1, d1;
+                const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
+                const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
+                act_fg(args.act, e0, f0, d0);
+                act_fg(args.act, e1, f1, d1);
+                const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
+                de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
+                dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
+              }
+              *reinterpret_cast<uint4*>(args.dE + rbase + col) = make_uint4(de[0], de[1], de[2], de[3]);
+              *reinterpret_cast<uint4*>(args.dG + rbase + col) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
             }
-            *reinterpret_cast<uint4*>(args.dE + rbase + col) = make_uint4(de[0], de[1], de[2], de[3]);
-            *reinterpret_cast<uint4*>(args.dG + rbase + col) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
           }
         }
-      } else {  // EPI_GLU_FWD: columns [0,128) hold e, [128,256) hold g
+      } else {  // EPI_GLU_FWD: per M-half, columns [0, BNT/2) hold e and [BNT/2, BNT) hold g
+        constexpr int CPH = C::BNT / 64;  // (e, g) chunk pairs per M-half
 #pragma unroll 1
-        for (int c = half * 2; c < half * 2 + 2; ++c) {
+        for (int it = half * 2; it < half * 2 + 2; ++it) {
+          const int h = it / CPH, c = it % CPH;
+          const int grow = half_row(mb, h) + row;
+          const bool row_ok = grow < args.M;
+          const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
           float e[32], g[32];
-          tmem_ld_32x32b_x32(trow + c * 32, e);
-          tmem_ld_32x32b_x32(trow + 128 + c * 32, g);
+          tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, e);
+          tmem_ld_32x32b_x32(tacc + h * C::BNT + C::BNT / 2 + c * 32, g);
           if (!row_ok) continue;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -434,13 +487,15 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
     }
   } else {
     // --------------------------------------------------- dequantisers ----
-    const int dq = (warp - 2 - C::EPI_WARPS) * 32 + lane;  // 0..255
+    const int dq = (warp - C::DQ_WARP0) * 32 + lane;  // 0..255
     constexpr int groups = 256 / C::NB;
     const int grp = dq / C::NB;
     const int tq = dq % C::NB;
     int j = 0;
     bool ok = true;
     for (int t = cluster; t < total_tiles && ok; t += clusters) {
+      int mb, n0;
+      tile_coords(t, mb, n0);
       for (int kb = 0; kb < nk; ++kb, ++j) {
         if (j % groups != grp) continue;
         const int seg = kb >= args.nkb0 ? 1 : 0;
@@ -454,16 +509,16 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
         float amax;
         int r = 0, cchunk = 0;
         if (MODE == MODE_BWD) {
-          // raw tile: 64 rows x (BNC/2) bytes, swizzled 128B (CG=1) or 64B (CG=2)
+          // raw tile: 64 rows x (BNC/2) bytes with the matching TMA swizzle (128B, 64B or 32B)
           r = tq & 63;
           cchunk = tq >> 6;
           constexpr int RB = C::BNC / 2;
-          constexpr int SHIFT = (RB == 128) ? 0 : 1;
-          constexpr int MASK = (RB == 128) ? 7 : 3;
+          constexpr int SHIFT = (RB == 128) ? 0 : (RB == 64 ? 1 : 2);
+          constexpr int MASK = RB / 16 - 1;
           const int x = (r >> SHIFT) & MASK;
           w0 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk) ^ x) << 4));
           w1 = *reinterpret_cast<const uint4*>(rc + r * RB + (((2 * cchunk + 1) ^ x) << 4));
-          amax = ra[r * 4 + cchunk + (CG == 2 ? 2 * (int)rank : 0)];
+          amax = ra[r * 4 + (((n0 + (int)rank * C::BNC) / 64) & 3) + cchunk];
         } else {
           // raw tile: NB rows x 32 bytes, 32B swizzle
           r = tq;
@@ -472,9 +527,6 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
           w1 = *reinterpret_cast<const uint4*>(rc + r * 32 + ((1 ^ x) << 4));
           amax = ra[r * 4 + (kl & 3)];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(rempty_bar(rs));
-
         const int s = j % C::S;
         ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status));
         if (!ok) break;
@@ -493,6 +545,11 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
         if (lane == 0) {
           if constexpr (CG == 2) mbar_arrive_cluster(leader(full_bar(s)));
           else mbar_arrive(full_bar(s));
+          // The raw slot is released only now: the stores above consumed every
+          // value loaded from it, so those shared-memory loads have returned
+          // before the TMA may overwrite the slot (an mbarrier arrive issued
+          // right after the loads could overtake them).
+          mbar_arrive(rempty_bar(rs));
         }
       }
     }
@@ -509,17 +566,18 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- launch --
-template <int MODE, int EPI, int CG>
+template <int MODE, int EPI, int CG, int MH>
 static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaStream_t stream) {
-  using C = GemmCfg<MODE, CG>;
-  auto kern = gemm_nf4_kernel<MODE, EPI, CG>;
+  using C = GemmCfg<MODE, CG, MH>;
+  auto kern = gemm_nf4_kernel<MODE, EPI, CG, MH>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static int resident[64] = {0};  // co-resident CTAs (multiple of CG) per device, per instantiation
-  const int bn_out = (EPI == EPI_GLU_FWD) ? 128 : 256;
+  const int bn_out = (EPI == EPI_GLU_FWD) ? C::BNT / 2 : C::BNT;
+  const int bm_pair = C::BM * CG * MH;
   const int n_tiles = (args.N + bn_out - 1) / bn_out;
-  const int m_tiles = (args.M + C::BM * CG - 1) / (C::BM * CG);
+  const int m_tiles = (args.M + bm_pair - 1) / bm_pair;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
@@ -554,20 +612,25 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaSt
   return cudaLaunchKernelEx(&cfg, kern, maps, args);
 }
 
-cudaError_t launch_gemm_nf4(int mode, int epi, int cg, const GemmMaps& maps, const GemmArgs& args,
+// Tile configurations: 1 = single CTA 128 x 256, 2 = CTA pair 256 x 256,
+// 3 = CTA pair 512 x 128.
+cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream) {
-#define QL_CASE(M_, E_, C_) \
-  if (mode == M_ && epi == E_ && cg == C_) return launch_one<M_, E_, C_>(maps, args, stream);
-  QL_CASE(MODE_FWD, EPI_STORE, 1)
-  QL_CASE(MODE_FWD, EPI_STORE, 2)
-  QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD, 1)
-  QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD, 2)
-  QL_CASE(MODE_BWD, EPI_STORE, 1)
-  QL_CASE(MODE_BWD, EPI_STORE, 2)
-  QL_CASE(MODE_BWD, EPI_GLU_BWD, 1)
-  QL_CASE(MODE_BWD, EPI_GLU_BWD, 2)
+#define QL_CASE(M_, E_)                                                          \
+  if (mode == M_ && epi == E_) {                                                 \
+    if (tiles == 1) return launch_one<M_, E_, 1, 1>(maps, args, stream);         \
+    if (tiles == 2) return launch_one<M_, E_, 2, 1>(maps, args, stream);         \
+    if (tiles == 3) return launch_one<M_, E_, 2, 2>(maps, args, stream);         \
+  }
+  QL_CASE(MODE_FWD, EPI_STORE)
+  QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD)
+  QL_CASE(MODE_BWD, EPI_STORE)
+  QL_CASE(MODE_BWD, EPI_GLU_BWD)
 #undef QL_CASE
   return cudaErrorInvalidValue;
 }
+
+// Columns of B each CTA dequantises for a tile configuration (host-side tensor map boxes).
+int gemm_nf4_b_cols_per_cta(int tiles) { return tiles == 1 ? 256 : (tiles == 2 ? 128 : 64); }
 
 }  // namespace ql

@@ -76,7 +76,7 @@ _SIGS = {
                                      ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_last_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
-    "qlora_set_cta_group": (ctypes.c_int32, [ctypes.c_int32]),
+    "qlora_set_tile_config": (ctypes.c_int32, [ctypes.c_int32]),
     "qlora_trace_begin": (ctypes.c_int, []),
     "qlora_trace_end": (ctypes.c_int32, [ctypes.POINTER(QloraTraceEntry), ctypes.c_int32]),
     "qlora_launch_count": (ctypes.c_uint64, []),
@@ -287,8 +287,11 @@ def qlora_status_string(status):
     return lib().qlora_status_string(status).decode()
 
 
-def qlora_set_cta_group(cg):
-    return int(lib().qlora_set_cta_group(cg))
+TILE_CONFIGS = {1: "1 CTA, 128x256", 2: "CTA pair, 256x256", 3: "CTA pair, 512x128"}
+
+
+def qlora_set_tile_config(tiles):
+    return int(lib().qlora_set_tile_config(tiles))
 
 
 def qlora_launch_count():

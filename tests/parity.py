@@ -92,8 +92,8 @@ def oracle_weight(w_bits):
     return codes, absmax, nf4_dequantize_f64(codes, absmax, n, k)
 
 
-def run_linear_gpu(p, cg=2, ws=None):
-    ops.qlora_set_cta_group(cg)
+def run_linear_gpu(p, tiles=2, ws=None):
+    ops.qlora_set_tile_config(tiles)
     w, codes, absmax = gpu_weight(p["W"])
     lin = ops.LoraLinear(w, dev(p["A"]), dev(p["B"]), p["s"])
     ws = ws or ops.Workspace()
@@ -114,8 +114,8 @@ def run_linear_oracle(p):
     return {"Y": Y, "XA": XA, "dX": dX, "dA": dA, "dB": dB, "codes": codes, "absmax": absmax}
 
 
-def run_mlp_gpu(p, act, cg=2, ws=None):
-    ops.qlora_set_cta_group(cg)
+def run_mlp_gpu(p, act, tiles=2, ws=None):
+    ops.qlora_set_tile_config(tiles)
     lins = {}
     qs = {}
     for k in ("g", "u", "d"):

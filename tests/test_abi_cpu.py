@@ -83,7 +83,8 @@ def test_host_side_rejections(lib):
     assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, 8, 16, ctypes.byref(sv), 16, 10, None) == 4
 
 
-def test_cta_group_setting(lib):
-    prev = ops.qlora_set_cta_group(1)
-    assert ops.qlora_set_cta_group(prev) == 1
-    assert ops.qlora_set_cta_group(3) == prev  # invalid values are ignored
+def test_tile_config_setting(lib):
+    prev = ops.qlora_set_tile_config(1)
+    assert ops.qlora_set_tile_config(prev) == 1
+    assert ops.qlora_set_tile_config(7) == prev  # invalid values are ignored
+    assert ops.qlora_set_tile_config(prev) == prev

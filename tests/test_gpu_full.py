@@ -61,7 +61,7 @@ def _quant(w_bits, g, tag):
 def test_full_size_linear(name):
     cfg = LINEAR_WORKLOADS[name]
     g = _golden(name)
-    ops.qlora_set_cta_group(2)
+    ops.qlora_set_tile_config(2)
     p = make_linear_problem(cfg["M"], cfg["K"], cfg["N"], cfg["r"], cfg["alpha"], cfg["seed"])
     w = _quant(p["W"], g, "W")
     lin = ops.LoraLinear(w, bits_to_torch(p["A"], "cuda"), bits_to_torch(p["B"], "cuda"), p["s"])
@@ -82,7 +82,7 @@ def test_full_size_linear(name):
 def test_full_size_mlp(name):
     cfg = MLP_WORKLOADS[name]
     g = _golden(name)
-    ops.qlora_set_cta_group(2)
+    ops.qlora_set_tile_config(2)
     p = make_mlp_problem(cfg["M"], cfg["d"], cfg["h"], cfg["r"], cfg["alpha"], cfg["seed"])
     lins = {}
     for k in ("g", "u", "d"):

@@ -2,8 +2,9 @@
 
 Bar: NF4 codes/absmax and dequantised weights bit-exact; every bf16 output and
 gradient within max|gpu - oracle| <= 2e-2 * RMS(oracle) per tensor.
-Sizes span several tiles of every kernel and ragged tails; both tensor-core
-tile shapes (single CTA and CTA pair) are covered.
+Sizes span several tiles of every kernel and ragged tails; all three
+tensor-core tile shapes (single CTA 128x256, CTA pair 256x256 and 512x128)
+are covered.
 """
 
 import numpy as np
@@ -106,11 +107,11 @@ LINEAR_CASES = [
 ]
 
 
-@pytest.mark.parametrize("cg", [1, 2])
+@pytest.mark.parametrize("tiles", [1, 2, 3])
 @pytest.mark.parametrize("M,K,N,alpha", LINEAR_CASES)
-def test_linear_fwd_bwd_parity(cg, M, K, N, alpha):
+def test_linear_fwd_bwd_parity(tiles, M, K, N, alpha):
     p = make_linear_problem(M, K, N, r=16, alpha=alpha, seed=M + K + N)
-    g = run_linear_gpu(p, cg)
+    g = run_linear_gpu(p, tiles)
     o = run_linear_oracle(p)
     assert g["status"] == 0
     assert np.array_equal(g["codes"], o["codes"]) and np.array_equal(g["absmax"], o["absmax"])
@@ -118,11 +119,11 @@ def test_linear_fwd_bwd_parity(cg, M, K, N, alpha):
         assert_close(k, g[k], o[k])
 
 
-@pytest.mark.parametrize("cg", [1, 2])
-def test_linear_zero_B_gives_zero_dA(cg):
+@pytest.mark.parametrize("tiles", [1, 2, 3])
+def test_linear_zero_B_gives_zero_dA(tiles):
     p = make_linear_problem(256, 512, 512, seed=5)
     p["B"] = np.zeros_like(p["B"])
-    g = run_linear_gpu(p, cg)
+    g = run_linear_gpu(p, tiles)
     o = run_linear_oracle(p)
     assert np.all(g["dA"] == 0)
     for k in ("Y", "dX", "dB"):
@@ -139,12 +140,12 @@ MLP_CASES = [
 ]
 
 
-@pytest.mark.parametrize("cg", [1, 2])
+@pytest.mark.parametrize("tiles", [1, 2, 3])
 @pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
 @pytest.mark.parametrize("M,d,h", MLP_CASES)
-def test_mlp_fwd_bwd_parity(cg, act, M, d, h):
+def test_mlp_fwd_bwd_parity(tiles, act, M, d, h):
     p = make_mlp_problem(M, d, h, seed=M + d + h)
-    g = run_mlp_gpu(p, act, cg)
+    g = run_mlp_gpu(p, act, tiles)
     o = run_mlp_oracle(p, act)
     assert g["status"] == 0
     for k in ("g", "u", "d"):

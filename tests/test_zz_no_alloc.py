@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("alpha", [16.0, 32.0])  # s = 1 and s = 2 (the scaled copy of X A lives in the scratch)
 def test_noalloc_forward_matches_workspace_forward_twice(alpha):
-    ops.qlora_set_cta_group(2)
+    ops.qlora_set_tile_config(2)
     p = make_linear_problem(1000, 1024, 768, r=16, alpha=alpha, seed=7)
     w = ops.nf4_quantize(bits_to_torch(p["W"], "cuda"))
     lin = ops.LoraLinear(w, bits_to_torch(p["A"], "cuda"), bits_to_torch(p["B"], "cuda"), p["s"])
