@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tiles", type=int, default=2, help="GEMM tile configuration (1, 2 or 3)")
+    ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override M (tokens per GPU) for small profiling cases; 0 = the workload's M")
     return ap.parse_args()

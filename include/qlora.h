@@ -117,7 +117,9 @@ QLORA_API qlora_status nf4_quantize(const qlora_bf16* w, int64_t n_out, int64_t 
 QLORA_API qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n_out, int64_t k_in, qlora_bf16* out,
                             qlora_stream_t stream);
 
-/* Workspace bytes needed by qlora_linear_fwd and qlora_linear_bwd. */
+/* Workspace bytes needed by qlora_linear_fwd and qlora_linear_bwd under the
+ * current tile configuration (the staged configuration 4 adds room for the
+ * dequantised bf16 weight, n_out * k_in * 2 bytes). */
 QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t k_in, int64_t n_out, int32_t r);
 
 /* Forward of one QLoRA projection (Mistral blog "10、11. 手动 Autograd"):
@@ -139,7 +141,8 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlor
                               void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* Workspace bytes needed by qlora_mlp_fwd and qlora_mlp_bwd (d = model
- * width, h = MLP width). */
+ * width, h = MLP width) under the current tile configuration (configuration 4
+ * adds room for two dequantised bf16 weights, 2 * h * d * 2 bytes). */
 QLORA_API size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r);
 
 /* Gated MLP forward (Gemma blog "GeGLU 与 Swiglu 激活函数"):
@@ -173,11 +176,17 @@ QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t 
 /* Human-readable name of a status code (static string). */
 QLORA_API const char* qlora_status_string(qlora_status status);
 
-/* Selects the tensor-core tile shape of the NF4 GEMMs (all give the same
- * results): 1 = one CTA per 128 x 256 tile, 2 = a CTA pair (cta_group::2)
- * per 256 x 256 tile (default), 3 = a CTA pair per 512 x 128 tile whose
- * dequantised weight tile feeds two M = 256 MMAs.  Invalid values are
- * ignored.  Returns the previous value.  Not thread-safe. */
+/* Selects how the NF4 GEMMs are tiled and fed (all give the same results).
+ * Configurations 1-3 dequantise the weight tile by tile in shared memory
+ * inside the GEMM mainloop: 1 = one CTA per 128 x 256 tile, 2 = a CTA pair
+ * (cta_group::2) per 256 x 256 tile, 3 = a CTA pair per 512 x 128 tile whose
+ * dequantised weight tile feeds two M = 256 MMAs.  Configuration 4 (default)
+ * = a CTA pair per 256 x 256 tile whose weight is first dequantised once per
+ * call into the workspace (the nf4_dequantize kernel) and then streamed by TMA:
+ * each weight element is decoded once instead of once per 256-row tile, at the
+ * price of that bf16 copy in the workspace.  The workspace size queries follow
+ * the configuration current when they are called.  Invalid values are ignored.
+ * Returns the previous value.  Not thread-safe. */
 QLORA_API int32_t qlora_set_tile_config(int32_t tiles);
 
 /* Kernel tracing (host side, not thread-safe).  While enabled, every kernel
@@ -208,7 +217,9 @@ QLORA_API uint64_t qlora_launch_count(void);
  * capture.  All calls share the one array: calls whose GPU work overlaps (on
  * different streams, or from different threads) race and must not be issued.
  * Each call zeroes the status word it uses; device-side timeouts are recorded
- * there and are not reported back through this call. */
+ * there and are not reported back through this call.  The fixed array has no
+ * room for a staged weight, so under tile configuration 4 this call uses
+ * configuration 2 (weight dequantised in the GEMM mainloop). */
 QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M,
                                                 qlora_bf16* Y, qlora_bf16* XA_saved, qlora_stream_t stream);
 

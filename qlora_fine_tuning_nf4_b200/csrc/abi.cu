@@ -55,7 +55,11 @@ struct TraceRec {
 std::vector<TraceRec> g_recs;
 std::vector<cudaEvent_t> g_pool;
 size_t g_pool_used = 0;
-int32_t g_tiles = 2;  // GEMM tile configuration (see qlora_set_tile_config)
+int32_t g_tiles = 4;  // GEMM tile configuration (see qlora_set_tile_config)
+#ifndef QL_GROUP_M
+#define QL_GROUP_M 8
+#endif
+constexpr int kGroupM = QL_GROUP_M;  // output-row tiles per group of the GEMM tile order
 
 cudaEvent_t pool_event() {
   if (g_pool_used == g_pool.size()) {
@@ -266,6 +270,32 @@ bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const qlora_nf4& w, bool b
 }
 int lora_rows_box(int bnc) { return bnc < 128 ? bnc : 128; }
 
+// Staged feed (tile configuration 4): the weight is dequantised once per call
+// into a bf16 [N, K] buffer of the workspace and its B tiles arrive by TMA in
+// the layout the in-mainloop dequantisers would have written.
+bool is_staged(int tiles) { return tiles == 4; }
+size_t stage_bytes(int64_t n_out, int64_t k_in) { return align256(static_cast<size_t>(n_out) * k_in * 2); }
+bool map_staged(CUtensorMap* m, const bf16* wq, const qlora_nf4& w, bool bwd, int bnc) {
+  const int64_t N = w.n_out, K = w.k_in;
+  if (!bwd) return map_bf16(m, wq, K, N, K, 64, bnc < 128 ? bnc : 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  return map_bf16(m, wq, K, N, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+qlora_status stage_weight(const qlora_nf4& w, bf16* dst, cudaStream_t st) {
+  KScope k(K_DEQUANT, st);
+  return cuda_status(launch_nf4_dequantize(w.codes, w.absmax, w.n_out * w.k_in, dst, st, num_sms()));
+}
+// B-operand maps of one weight for either feed (stage: its bf16 buffer when staged)
+qlora_status map_weight(GemmMaps& maps, int i, const qlora_nf4& w, bool bwd, int tiles, bf16* stage,
+                        cudaStream_t st) {
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
+  if (is_staged(tiles)) {
+    const qlora_status s = stage_weight(w, stage, st);
+    if (s != QLORA_OK) return s;
+    return map_staged(&maps.b[i], stage, w, bwd, bnc) ? QLORA_OK : QLORA_ERR_CUDA;
+  }
+  return map_nf4(&maps.codes[i], &maps.absmax[i], w, bwd, bnc) ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 qlora_status check_linear(const qlora_lora_linear* lin) {
   if (!lin || !lin->w.codes || !lin->w.absmax || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
   if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
@@ -279,19 +309,19 @@ qlora_status check_linear(const qlora_lora_linear* lin) {
 
 // Y-side GEMM launch helpers -------------------------------------------------
 qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, const bf16* XAs, bf16* Y, int* status,
-                      cudaStream_t st) {
-  const int tiles = g_tiles;
-  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
+                      int tiles, bf16* stage, cudaStream_t st) {
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int64_t K = lin.w.k_in, N = lin.w.n_out;
   if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin.w, false, bnc)) return QLORA_ERR_CUDA;
+  const qlora_status s = map_weight(maps, 0, lin.w, false, tiles, stage, st);
+  if (s != QLORA_OK) return s;
   if (!map_bf16(&maps.la[0], XAs, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&maps.lb[0], lin.B, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   maps.a[1] = maps.a[0];
   maps.codes[1] = maps.codes[0];
   maps.absmax[1] = maps.absmax[0];
+  maps.b[1] = maps.b[0];
   maps.la[1] = maps.la[0];
   maps.lb[1] = maps.lb[0];
   GemmArgs a;
@@ -304,6 +334,7 @@ qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, co
   a.ldo = (int)N;
   a.D = Y;
   a.status = status;
+  a.group_m = kGroupM;
   KScope k(K_GEMM_FWD, st);
   return cuda_status(launch_gemm_nf4(MODE_FWD, EPI_STORE, tiles, maps, a, st));
 }
@@ -335,7 +366,7 @@ qlora_status qlora_nf4_codebook(float out[16]) {
 
 int32_t qlora_set_tile_config(int32_t tiles) {
   const int32_t prev = g_tiles;
-  if (tiles >= 1 && tiles <= 3) g_tiles = tiles;
+  if (tiles >= 1 && tiles <= 4) g_tiles = tiles;
   return prev;
 }
 
@@ -369,8 +400,16 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) 
   size_t part = rowproj_part_bytes(M, K, 16);
   part = std::max(part, dypass_part_bytes(M, N));
   part = std::max(part, colproj_part_bytes(M, K, 16));
-  return 256 + vec + align256(part);
+  return 256 + vec + align256(part) + (is_staged(g_tiles) ? stage_bytes(N, K) : 0);
 }
+
+namespace {
+// the staged weight sits at the end of a linear workspace
+bf16* linear_stage(void* ws, int64_t M, int64_t K, int64_t N) {
+  return reinterpret_cast<bf16*>(static_cast<char*>(ws) + qlora_linear_workspace_bytes(M, K, N, 16) -
+                                 stage_bytes(N, K));
+}
+}  // namespace
 
 qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                               qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
@@ -394,7 +433,9 @@ qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
                    routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
   if (s != QLORA_OK) return s;
-  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, st);
+  const int tiles = g_tiles;
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, tiles,
+                  is_staged(tiles) ? linear_stage(ws, M, K, N) : nullptr, st);
 }
 
 qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
@@ -417,6 +458,7 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   char* w = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(w);
   bf16* sG = reinterpret_cast<bf16*>(w + 256);
+  bf16* stage = is_staged(tiles) ? linear_stage(ws, M, K, N) : nullptr;
   float* part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
   const float sc = lin->scale;
   // G = dY B^T (stored scaled: sG), dB = s (XA)^T dY
@@ -429,13 +471,14 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, N, M, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], lin->w, true, bnc)) return QLORA_ERR_CUDA;
+    if ((s = map_weight(maps, 0, lin->w, true, tiles, stage, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], sG, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
       return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
+    maps.b[1] = maps.b[0];
     maps.la[1] = maps.la[0];
     maps.lb[1] = maps.lb[0];
     GemmArgs a;
@@ -447,6 +490,7 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     a.ldo = (int)K;
     a.D = reinterpret_cast<bf16*>(dX);
     a.status = status;
+    a.group_m = kGroupM;
     KScope k(K_GEMM_BWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
@@ -466,7 +510,7 @@ size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
   part = std::max(part, dypass_part_bytes(M, h));
   part = std::max(part, colproj_part_bytes(M, h, 16));
   part = std::max(part, colproj_part_bytes(M, d, 32));
-  return 256 + 2 * big + 5 * vec + align256(part);
+  return 256 + 2 * big + 5 * vec + align256(part) + (is_staged(g_tiles) ? 2 * stage_bytes(h, d) : 0);
 }
 
 namespace {
@@ -474,8 +518,9 @@ struct MlpWs {
   int* status;
   bf16 *dE, *dG, *v0, *v1, *v2, *gu;  // v*: [M,16] vectors; gu: [M,32]
   float* part;
+  bf16 *stage0, *stage1;  // staged feed: room for two dequantised [h, d] weights (gate, up; or down)
 };
-MlpWs carve_mlp(void* ws, int64_t M, int64_t h) {
+MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h) {
   char* w = static_cast<char*>(ws);
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
   const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
@@ -489,6 +534,12 @@ MlpWs carve_mlp(void* ws, int64_t M, int64_t h) {
   m.v2 = reinterpret_cast<bf16*>(w + off); off += vec;
   m.gu = reinterpret_cast<bf16*>(w + off); off += 2 * vec;
   m.part = reinterpret_cast<float*>(w + off);
+  const size_t total = qlora_mlp_workspace_bytes(M, d, h, 16);
+  m.stage0 = m.stage1 = nullptr;
+  if (is_staged(g_tiles)) {
+    m.stage0 = reinterpret_cast<bf16*>(w + total - 2 * stage_bytes(h, d));
+    m.stage1 = reinterpret_cast<bf16*>(w + total - stage_bytes(h, d));
+  }
   return m;
 }
 qlora_status check_mlp(const qlora_lora_linear* g, const qlora_lora_linear* u, const qlora_lora_linear* d) {
@@ -520,8 +571,7 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
   if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int tiles = g_tiles;
-  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  MlpWs w = carve_mlp(ws, M, h);
+  MlpWs w = carve_mlp(ws, M, d, h);
   const bf16* x = reinterpret_cast<const bf16*>(X);
   bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
   bf16* xau = reinterpret_cast<bf16*>(sv->XA_u);
@@ -542,8 +592,8 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, false, bnc)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, false, bnc)) return QLORA_ERR_CUDA;
+    if ((s = map_weight(maps, 0, gate->w, false, tiles, w.stage0, st)) != QLORA_OK) return s;
+    if ((s = map_weight(maps, 1, up->w, false, tiles, w.stage1, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], xags, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], xaus, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], gate->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -560,6 +610,7 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.G = reinterpret_cast<bf16*>(sv->G);
     a.H = reinterpret_cast<bf16*>(sv->H);
     a.status = w.status;
+    a.group_m = kGroupM;
     KScope k(K_GEMM_GLU_FWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_FWD_GLU, EPI_GLU_FWD, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
@@ -570,7 +621,8 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
                    w.status, st);
   if (s != QLORA_OK) return s;
   // Y = H W_d^T + (s H A_d) B_d
-  return gemm_fwd(*down, reinterpret_cast<const bf16*>(sv->H), M, hads, reinterpret_cast<bf16*>(Y), w.status, st);
+  return gemm_fwd(*down, reinterpret_cast<const bf16*>(sv->H), M, hads, reinterpret_cast<bf16*>(Y), w.status, tiles,
+                  w.stage0, st);
 }
 
 qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
@@ -596,7 +648,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int tiles = g_tiles;
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  MlpWs w = carve_mlp(ws, M, h);
+  MlpWs w = carve_mlp(ws, M, d, h);
   bf16* sGd = w.v0;
   // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, d, reinterpret_cast<const bf16*>(sv->HA_d),
@@ -608,13 +660,14 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], down->w, true, bnc)) return QLORA_ERR_CUDA;
+    if ((s = map_weight(maps, 0, down->w, true, tiles, w.stage0, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], sGd, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
       return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
+    maps.b[1] = maps.b[0];
     maps.la[1] = maps.la[0];
     maps.lb[1] = maps.lb[0];
     GemmArgs a;
@@ -630,6 +683,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.dE = w.dE;
     a.dG = w.dG;
     a.status = w.status;
+    a.group_m = kGroupM;
     KScope k(K_GEMM_GLU_BWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_GLU_BWD, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
@@ -653,8 +707,8 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[0], &maps.absmax[0], gate->w, true, bnc)) return QLORA_ERR_CUDA;
-    if (!map_nf4(&maps.codes[1], &maps.absmax[1], up->w, true, bnc)) return QLORA_ERR_CUDA;
+    if ((s = map_weight(maps, 0, gate->w, true, tiles, w.stage0, st)) != QLORA_OK) return s;
+    if ((s = map_weight(maps, 1, up->w, true, tiles, w.stage1, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], w.gu, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], w.gu + 16, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
@@ -671,6 +725,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.ldo = (int)d;
     a.D = reinterpret_cast<bf16*>(dX);
     a.status = w.status;
+    a.group_m = kGroupM;
     KScope k(K_GEMM_BWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
@@ -786,7 +841,11 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_
   s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
                    routs(rout(xa, 0, 16, 0, 1.f), rout(XAs != xa ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
   if (s != QLORA_OK) return s;
-  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, st);
+  // The fixed scratch has no room for a staged weight: the staged configuration
+  // falls back to the pair tile that dequantises in the mainloop.
+  const int tiles = is_staged(g_tiles) ? 2 : g_tiles;
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, tiles, nullptr,
+                  st);
 }
 
 }  // extern "C"

@@ -9,16 +9,25 @@
 //   gate/up   e, g as above; h = act(e) g                  (MODE_FWD_GLU)
 //   backward  dX = dY dequant(W)   + (s dY B^T) A^T        (MODE_BWD)
 //   down bwd  dH as above; dE = dH g act'(e), dG = dH act(e) (EPI_GLU_BWD)
-// The dequantised weight never exists in HBM: each CTA expands the NF4 codes
-// of its B tile straight to bf16 in shared memory.
+// Two ways to feed the B operand (the weight), chosen per launch:
+//  * in-mainloop dequantisation: the dequantised weight never exists in HBM;
+//    each CTA expands the NF4 codes of its B tile straight to bf16 in shared
+//    memory, k-block by k-block, while the tensor cores consume earlier ones;
+//  * staged: the caller has expanded the whole weight once into a bf16 buffer
+//    (the HBM-bound dequantisation kernel) and the B tiles arrive by TMA like
+//    the A tiles.  Every B tile is then decoded once per call instead of once
+//    per output-row tile, and the shared-memory stores of the decoded tile
+//    leave the mainloop.
 //
-// Structure (one output tile per CTA, or per CTA pair with cta_group::2):
-//   warp 0      TMA producer: A tiles, raw NF4 codes + absmax, LoRA operands
-//   warp 1      TMEM allocation; lane 0 of the leader CTA issues tcgen05.mma
-//   warps 2-5   epilogue: TMEM -> registers -> activation -> global
-//   warps 6-13  dequantisers: raw codes -> bf16 B tile (128B-swizzled)
+// Structure (persistent; one output tile at a time per CTA, or per CTA pair
+// with cta_group::2):
+//   warp 0       TMA producer: A tiles (and staged B tiles), LoRA operands
+//   warp 1       TMEM allocation; lane 0 of the leader CTA issues tcgen05.mma
+//   warp 2       raw NF4 codes + absmax by TMA (in-mainloop feed only)
+//   warps 3-10   epilogue: TMEM -> registers -> activation -> global
+//   warps 11-18  dequantisers: raw codes -> bf16 B tile (in-mainloop feed only)
 // Pipelines: raw ring (TMA -> dequantisers), operand ring (A by TMA, B by the
-// dequantisers -> MMA), one accumulator barrier (MMA -> epilogue).
+// dequantisers or by TMA -> MMA), two accumulators (MMA -> epilogue).
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -101,7 +110,7 @@ QL_DEV void act_fg(int act, float e, float& f, float& g) {
 //   (CG, MH) = (2, 1): 256 x 256 per pair
 //   (CG, MH) = (2, 2): 512 x 128 per pair -- each dequantised B tile feeds two
 //                      M = 256 MMAs, halving the dequantisation per MMA.
-template <int MODE, int CG, int MH>
+template <int MODE, int CG, int MH, bool ST>
 struct GemmCfg {
   static constexpr int BM = 128;                 // rows per CTA per M-half (TMEM lanes)
   static constexpr int BNT = 256 / MH;           // MMA N (whole pair)
@@ -114,8 +123,8 @@ struct GemmCfg {
   static constexpr int B_BYTES = BNC * BK * 2;
   static constexpr int RC_BYTES = NB * 32;
   static constexpr int RA_BYTES = (MODE == MODE_BWD) ? 64 * 16 : BNC * 16;
-  static constexpr int S = (CG == 1) ? 3 : (MH == 1 ? 5 : 4);   // operand stages
-  static constexpr int RS = (CG == 1) ? 4 : (MH == 1 ? 6 : 8);  // raw stages
+  static constexpr int S = ST ? 6 : ((CG == 1) ? 3 : (MH == 1 ? 5 : 4));  // operand stages
+  static constexpr int RS = ST ? 0 : ((CG == 1) ? 4 : (MH == 1 ? 6 : 8));  // raw stages
   static constexpr int LA_BYTES = BM * 16 * 2;   // one LoRA left operand tile (128 rows x 16)
   static constexpr int LBOP = BNC * 32;          // one LoRA right operand (BNC x 16 bf16)
   static constexpr int OFF_A = 0;
@@ -128,7 +137,7 @@ struct GemmCfg {
   static constexpr int NBAR = 2 * S + 2 * RS + 7;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static constexpr int EPI_WARPS = 8;            // two per TMEM lane quadrant
-  static constexpr int DQ_WARPS = 8;
+  static constexpr int DQ_WARPS = ST ? 0 : 8;
   static constexpr int EPI_WARP0 = 3;            // warps 0: A/LoRA TMA, 1: MMA, 2: raw-code TMA
   static constexpr int DQ_WARP0 = EPI_WARP0 + EPI_WARPS;
   static constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
@@ -148,10 +157,10 @@ struct GemmCfg {
 // t = cluster, cluster + clusters, ... (N tiles fastest).  Every role iterates
 // the same tile sequence; j counts 64-wide reduction blocks across tiles and
 // indexes the rings, so barrier phases follow from j and the tile counter.
-template <int MODE, int EPI, int CG, int MH>
-__global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
+template <int MODE, int EPI, int CG, int MH, bool ST>
+__global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
     gemm_nf4_kernel(const __grid_constant__ GemmMaps maps, const GemmArgs args) {
-  using C = GemmCfg<MODE, CG, MH>;
+  using C = GemmCfg<MODE, CG, MH, ST>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -197,7 +206,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
-      mbar_init(full_bar(s), 1 + CG * (C::NB / 32));
+      mbar_init(full_bar(s), ST ? 1 : 1 + CG * (C::NB / 32));
       mbar_init(empty_bar(s), 1);
     }
     for (int s = 0; s < C::RS; ++s) {
@@ -225,9 +234,16 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
   // shared::cluster address of a barrier in the pair's leader CTA
   auto leader = [&](uint32_t bar) { return (CG == 2) ? mapa_shared(bar, 0) : bar; };
   // first output row of M-half h of tile t for this CTA, and the tile's first column
+  // Tiles are visited in groups of group_m row tiles: inside a group the row
+  // tile varies fastest, so the tiles in flight at any moment span a compact
+  // block of rows x columns and share their A and B panels through L2.
   auto tile_coords = [&](int t, int& mb, int& n0) {
-    mb = (t / n_tiles) * bm_pair + static_cast<int>(rank) * C::BM;
-    n0 = (t % n_tiles) * bn_out;
+    const int gsz = args.group_m * n_tiles;
+    const int first = (t / gsz) * args.group_m;
+    const int gm = min(m_tiles - first, args.group_m);
+    const int r = t - (first / args.group_m) * gsz;
+    mb = (first + r % gm) * bm_pair + static_cast<int>(rank) * C::BM;
+    n0 = (r / gm) * bn_out;
   };
   auto half_row = [&](int mb, int h) { return mb + h * C::BM * CG; };
 
@@ -237,8 +253,12 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
       bool ok = true;
       for (int i = 0; i < 2; ++i) {
         tma_prefetch_desc(&maps.a[i]);
-        tma_prefetch_desc(&maps.codes[i]);
-        tma_prefetch_desc(&maps.absmax[i]);
+        if constexpr (ST) {
+          tma_prefetch_desc(&maps.b[i]);
+        } else {
+          tma_prefetch_desc(&maps.codes[i]);
+          tma_prefetch_desc(&maps.absmax[i]);
+        }
       }
       auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar_local, int x, int y) {
         if constexpr (CG == 2) tma_load_2d_pair(dst, m, leader(bar_local), x, y);
@@ -258,10 +278,29 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
           const int s = j % C::S;
           ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
           if (!ok) break;
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::A_BYTES * CG);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), (C::A_BYTES + (ST ? C::B_BYTES : 0)) * CG);
           for (int h = 0; h < MH; ++h)
             load(sbase + C::OFF_A + s * C::A_BYTES + h * C::A_TILE, &maps.a[seg], full_bar(s), kl * 64,
                  half_row(mb, h));
+          if constexpr (ST) {
+            // staged weight: the B tile in the layout the dequantisers would write
+            const uint32_t bdst = sbase + C::OFF_B + s * C::B_BYTES;
+            if (MODE == MODE_BWD) {
+              // W rows kl*64.. (the reduction index) x this CTA's BNC output columns, 64 per box
+              for (int c = 0; c < C::BNC / 64; ++c)
+                load(bdst + c * 8192, &maps.b[seg], full_bar(s), n0 + (int)rank * C::BNC + c * 64, kl * 64);
+            } else {
+              for (int bx = 0; bx < C::BNC / C::BOXR; ++bx) {
+                const int p = (int)rank * C::BNC + bx * C::BOXR;  // first B row of the box in the pair tile
+                int src = 0, row = n0 + p;
+                if (MODE == MODE_FWD_GLU) {
+                  src = p < C::BNT / 2 ? 0 : 1;
+                  row = n0 + (src ? p - C::BNT / 2 : p);
+                }
+                load(bdst + bx * C::BOXR * 128, &maps.b[src], full_bar(s), kl * 64, row);
+              }
+            }
+          }
         }
         if (!ok || args.lora == 0) continue;
         // LoRA operands of this tile (single buffer, released by the MMA's commit)
@@ -291,7 +330,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------ raw-code producer --
-    if (lane == 0) {
+    if constexpr (!ST) if (lane == 0) {
       bool ok = true;
       int j = 0;
       for (int t = cluster; t < total_tiles && ok; t += clusters) {
@@ -485,7 +524,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
         else mbar_arrive(acc_empty0 + 8u * b);
       }
     }
-  } else {
+  } else if constexpr (!ST) {
     // --------------------------------------------------- dequantisers ----
     const int dq = (warp - C::DQ_WARP0) * 32 + lane;  // 0..255
     constexpr int groups = 256 / C::NB;
@@ -566,10 +605,10 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------- launch --
-template <int MODE, int EPI, int CG, int MH>
+template <int MODE, int EPI, int CG, int MH, bool ST>
 static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaStream_t stream) {
-  using C = GemmCfg<MODE, CG, MH>;
-  auto kern = gemm_nf4_kernel<MODE, EPI, CG, MH>;
+  using C = GemmCfg<MODE, CG, MH, ST>;
+  auto kern = gemm_nf4_kernel<MODE, EPI, CG, MH, ST>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -613,14 +652,16 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaSt
 }
 
 // Tile configurations: 1 = single CTA 128 x 256, 2 = CTA pair 256 x 256,
-// 3 = CTA pair 512 x 128.
+// 3 = CTA pair 512 x 128 (all three dequantising in the mainloop);
+// 4 = CTA pair 256 x 256 fed from a staged bf16 weight (maps.b).
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream) {
 #define QL_CASE(M_, E_)                                                          \
   if (mode == M_ && epi == E_) {                                                 \
-    if (tiles == 1) return launch_one<M_, E_, 1, 1>(maps, args, stream);         \
-    if (tiles == 2) return launch_one<M_, E_, 2, 1>(maps, args, stream);         \
-    if (tiles == 3) return launch_one<M_, E_, 2, 2>(maps, args, stream);         \
+    if (tiles == 1) return launch_one<M_, E_, 1, 1, false>(maps, args, stream);  \
+    if (tiles == 2) return launch_one<M_, E_, 2, 1, false>(maps, args, stream);  \
+    if (tiles == 3) return launch_one<M_, E_, 2, 2, false>(maps, args, stream);  \
+    if (tiles == 4) return launch_one<M_, E_, 2, 1, true>(maps, args, stream);   \
   }
   QL_CASE(MODE_FWD, EPI_STORE)
   QL_CASE(MODE_FWD_GLU, EPI_GLU_FWD)
@@ -631,6 +672,6 @@ cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, 
 }
 
 // Columns of B each CTA dequantises for a tile configuration (host-side tensor map boxes).
-int gemm_nf4_b_cols_per_cta(int tiles) { return tiles == 1 ? 256 : (tiles == 2 ? 128 : 64); }
+int gemm_nf4_b_cols_per_cta(int tiles) { return tiles == 1 ? 256 : (tiles == 3 ? 64 : 128); }
 
 }  // namespace ql

@@ -28,6 +28,7 @@ struct GemmMaps {
   CUtensorMap absmax[2];  // fp32 absmax, matching codes[]
   CUtensorMap la[2];      // LoRA left operand(s): bf16 [M, 16], box {16,128}, 32B swizzle
   CUtensorMap lb[2];      // LoRA right operand(s)
+  CUtensorMap b[2];       // staged feed only: the dequantised bf16 weight, matching codes[]
 };
 
 struct GemmArgs {
@@ -47,6 +48,7 @@ struct GemmArgs {
   bf16* dE;     // EPI_GLU_BWD outputs
   bf16* dG;
   int* status;  // device status word (timeouts)
+  int group_m;  // tile order: groups of group_m output-row tiles, rows fastest inside a group (>= 1)
 };
 
 // --------------------------------------------------------------- skinny ---

@@ -287,7 +287,8 @@ def qlora_status_string(status):
     return lib().qlora_status_string(status).decode()
 
 
-TILE_CONFIGS = {1: "1 CTA, 128x256", 2: "CTA pair, 256x256", 3: "CTA pair, 512x128"}
+TILE_CONFIGS = {1: "1 CTA, 128x256", 2: "CTA pair, 256x256", 3: "CTA pair, 512x128",
+                4: "CTA pair, 256x256, staged bf16 weight"}
 
 
 def qlora_set_tile_config(tiles):

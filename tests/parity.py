@@ -92,7 +92,7 @@ def oracle_weight(w_bits):
     return codes, absmax, nf4_dequantize_f64(codes, absmax, n, k)
 
 
-def run_linear_gpu(p, tiles=2, ws=None):
+def run_linear_gpu(p, tiles=4, ws=None):
     ops.qlora_set_tile_config(tiles)
     w, codes, absmax = gpu_weight(p["W"])
     lin = ops.LoraLinear(w, dev(p["A"]), dev(p["B"]), p["s"])
@@ -114,7 +114,7 @@ def run_linear_oracle(p):
     return {"Y": Y, "XA": XA, "dX": dX, "dA": dA, "dB": dB, "codes": codes, "absmax": absmax}
 
 
-def run_mlp_gpu(p, act, tiles=2, ws=None):
+def run_mlp_gpu(p, act, tiles=4, ws=None):
     ops.qlora_set_tile_config(tiles)
     lins = {}
     qs = {}

@@ -57,11 +57,12 @@ def _quant(w_bits, g, tag):
     return w
 
 
+@pytest.mark.parametrize("tiles", [4, 2])  # staged weight (default); dequantised in the mainloop
 @pytest.mark.parametrize("name", [n for n in LINEAR_WORKLOADS if n != "tiny_linear"])
-def test_full_size_linear(name):
+def test_full_size_linear(name, tiles):
     cfg = LINEAR_WORKLOADS[name]
     g = _golden(name)
-    ops.qlora_set_tile_config(2)
+    ops.qlora_set_tile_config(tiles)
     p = make_linear_problem(cfg["M"], cfg["K"], cfg["N"], cfg["r"], cfg["alpha"], cfg["seed"])
     w = _quant(p["W"], g, "W")
     lin = ops.LoraLinear(w, bits_to_torch(p["A"], "cuda"), bits_to_torch(p["B"], "cuda"), p["s"])
@@ -78,11 +79,12 @@ def test_full_size_linear(name):
         _check(k, gpu_f64(t).reshape(-1)[g[f"idx_{k}"]], g[f"val_{k}"], g[f"rms_{k}"])
 
 
+@pytest.mark.parametrize("tiles", [4, 2])
 @pytest.mark.parametrize("name", list(MLP_WORKLOADS))
-def test_full_size_mlp(name):
+def test_full_size_mlp(name, tiles):
     cfg = MLP_WORKLOADS[name]
     g = _golden(name)
-    ops.qlora_set_tile_config(2)
+    ops.qlora_set_tile_config(tiles)
     p = make_mlp_problem(cfg["M"], cfg["d"], cfg["h"], cfg["r"], cfg["alpha"], cfg["seed"])
     lins = {}
     for k in ("g", "u", "d"):

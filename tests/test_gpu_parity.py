@@ -2,9 +2,10 @@
 
 Bar: NF4 codes/absmax and dequantised weights bit-exact; every bf16 output and
 gradient within max|gpu - oracle| <= 2e-2 * RMS(oracle) per tensor.
-Sizes span several tiles of every kernel and ragged tails; all three
-tensor-core tile shapes (single CTA 128x256, CTA pair 256x256 and 512x128)
-are covered.
+Sizes span several tiles of every kernel and ragged tails; every GEMM
+configuration is covered: the three tile shapes that dequantise in the
+mainloop (single CTA 128x256, CTA pair 256x256 and 512x128) and the CTA pair
+256x256 fed from a staged bf16 weight.
 """
 
 import numpy as np
@@ -107,7 +108,7 @@ LINEAR_CASES = [
 ]
 
 
-@pytest.mark.parametrize("tiles", [1, 2, 3])
+@pytest.mark.parametrize("tiles", [1, 2, 3, 4])
 @pytest.mark.parametrize("M,K,N,alpha", LINEAR_CASES)
 def test_linear_fwd_bwd_parity(tiles, M, K, N, alpha):
     p = make_linear_problem(M, K, N, r=16, alpha=alpha, seed=M + K + N)
@@ -119,7 +120,7 @@ def test_linear_fwd_bwd_parity(tiles, M, K, N, alpha):
         assert_close(k, g[k], o[k])
 
 
-@pytest.mark.parametrize("tiles", [1, 2, 3])
+@pytest.mark.parametrize("tiles", [1, 2, 3, 4])
 def test_linear_zero_B_gives_zero_dA(tiles):
     p = make_linear_problem(256, 512, 512, seed=5)
     p["B"] = np.zeros_like(p["B"])
@@ -140,7 +141,7 @@ MLP_CASES = [
 ]
 
 
-@pytest.mark.parametrize("tiles", [1, 2, 3])
+@pytest.mark.parametrize("tiles", [1, 2, 3, 4])
 @pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
 @pytest.mark.parametrize("M,d,h", MLP_CASES)
 def test_mlp_fwd_bwd_parity(tiles, act, M, d, h):
