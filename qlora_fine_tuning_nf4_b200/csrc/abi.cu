@@ -23,13 +23,13 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes, const float* absmax, int
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
 int gemm_nf4_b_cols_per_cta(int tiles);
-cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1, float* part,
-                           int M, int K, int splits, int kb_per_split, int* status, cudaStream_t st);
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, float* part, int M, int N, int splits,
-                           int mb_per_split, int* status, cudaStream_t st);
-cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, float* gpart,
-                          float* qpart, int M, int N, int rc_per_cta, int* status, cudaStream_t st);
-cudaError_t launch_reduce(const float* part, int S, int rows, int R, const ReduceOuts& outs, cudaStream_t st);
+cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
+                           const ReduceJob& job, int nkc, int* status, cudaStream_t st);
+cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+                           int* status, cudaStream_t st);
+cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
+                          const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
+cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st);
 extern const uint32_t h_nf4_bits[16];
 }  // namespace ql
 
@@ -143,38 +143,61 @@ bool map_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t
 }
 
 // ---------------------------------------------------------- planning ----
-constexpr int kTargetCtas = 2 * 148;
+// Skinny passes run kTargetCtas persistent CTAs (four per SM on B200).
+constexpr int kTargetCtas = 4 * 148;
 
-struct RowPlan { int splits, kb_per; };
-RowPlan plan_rowproj(int64_t M, int64_t K) {
-  const int64_t mblocks = cdiv(M, 64), kbs = K / 64;
-  int64_t splits = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, mblocks), 1), kbs);
-  const int64_t per = cdiv(kbs, splits);
-  return {static_cast<int>(cdiv(kbs, per)), static_cast<int>(per)};
+// Partition of `groups` output groups of `upg` units each over the CTAs:
+// unit granularity while there are fewer groups than CTAs (every CTA streams
+// the same number of tiles), whole groups otherwise (one partial per group).
+struct SkPlan {
+  SkPart sp;
+  int slot_cap;
+};
+SkPlan plan_skinny(int64_t groups, int64_t upg) {
+  SkPlan p;
+  const int64_t units = groups * upg;
+  int64_t align = groups >= kTargetCtas ? upg : 1;
+  while (cdiv(units, align) > (int64_t(1) << 30)) align *= 2;  // keep the unit count in int range
+  const int64_t U = cdiv(units, align);
+  p.sp.U = static_cast<int>(U);
+  p.sp.P = static_cast<int>(std::min<int64_t>(kTargetCtas, U));
+  p.sp.align = static_cast<int>(align);
+  p.sp.upg = static_cast<int>(upg);
+  p.slot_cap = 1;
+  for (int64_t g = 0; g < groups; ++g) p.slot_cap = std::max(p.slot_cap, sk_slots(p.sp, static_cast<int>(g)));
+  return p;
 }
-struct ColPlan { int splits, mb_per; };
-ColPlan plan_colproj(int64_t M, int64_t ncols) {
-  const int64_t nblocks = cdiv(ncols, 64), mbs = cdiv(M, 64);
-  int64_t splits = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, nblocks), 1), mbs);
-  const int64_t per = cdiv(mbs, splits);
-  return {static_cast<int>(cdiv(mbs, per)), static_cast<int>(per)};
-}
-struct DyPlan { int gsplits, qsplits, rc; };
-DyPlan plan_dypass(int64_t M, int64_t N) {
-  const int64_t gx = cdiv(N, 256), mch = cdiv(M, 64);
-  int64_t gy = std::min<int64_t>(std::max<int64_t>(cdiv(kTargetCtas, gx), 1), mch);
-  const int64_t rc = cdiv(mch, gy);
-  return {static_cast<int>(gx), static_cast<int>(cdiv(mch, rc)), static_cast<int>(rc)};
-}
+constexpr int kDyCC = 4;  // column chunks of 64 per dypass unit (matches the kernel)
+SkPlan plan_rowproj(int64_t M, int64_t K) { return plan_skinny(cdiv(M, 64), K / 64); }
+SkPlan plan_colproj(int64_t M, int64_t ncols) { return plan_skinny(cdiv(ncols, 64), cdiv(M, 64)); }
+SkPlan plan_dypass(int64_t M, int64_t N) { return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64)); }
 size_t rowproj_part_bytes(int64_t M, int64_t K, int R) {
-  return static_cast<size_t>(plan_rowproj(M, K).splits) * M * R * 4;
+  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K).slot_cap * 64 * R * 4;
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
-  return static_cast<size_t>(plan_colproj(M, ncols).splits) * ncols * R * 4;
+  return static_cast<size_t>(cdiv(ncols, 64)) * plan_colproj(M, ncols).slot_cap * 64 * R * 4;
+}
+size_t dypass_gpart_bytes(int64_t M, int64_t N) {
+  return align256(static_cast<size_t>(cdiv(M, 64)) * cdiv(cdiv(N, 64), kDyCC) * 64 * 16 * 4);
 }
 size_t dypass_part_bytes(int64_t M, int64_t N) {
-  const DyPlan p = plan_dypass(M, N);
-  return align256(static_cast<size_t>(p.gsplits) * M * 16 * 4) + static_cast<size_t>(p.qsplits) * N * 16 * 4;
+  const int64_t ncb = cdiv(cdiv(N, 64), kDyCC);
+  return dypass_gpart_bytes(M, N) + static_cast<size_t>(ncb) * plan_dypass(M, N).slot_cap * kDyCC * 64 * 16 * 4;
+}
+ReduceJob reduce_job(float* part, int64_t groups, int grows, int64_t rows, int R, int slot_cap, int nslots,
+                     const SkPart& sp, const ReduceOuts& outs) {
+  ReduceJob j;
+  std::memset(&j, 0, sizeof(j));
+  j.part = part;
+  j.groups = static_cast<int>(groups);
+  j.grows = grows;
+  j.rows = static_cast<int>(rows);
+  j.R = R;
+  j.slot_cap = slot_cap;
+  j.nslots = nslots;
+  j.sp = sp;
+  j.outs = outs;
+  return j;
 }
 
 // ------------------------------------------------------------ passes ----
@@ -188,14 +211,16 @@ qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, c
   if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mv0, V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mv1, V1 ? V1 : V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
-  const RowPlan p = plan_rowproj(M, K);
+  const SkPlan p = plan_rowproj(M, K);
+  const int64_t nrc = cdiv(M, 64);
+  const ReduceJob j = reduce_job(part, nrc, 64, M, 16 * nv, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_ROWPROJ, st);
-    qlora_status s = cuda_status(launch_rowproj(nv, mt, mv0, mv1, part, (int)M, (int)K, p.splits, p.kb_per, status, st));
+    const qlora_status s = cuda_status(launch_rowproj(nv, mt, mv0, mv1, j, (int)(K / 64), status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(part, p.splits, (int)M, 16 * nv, outs, st));
+  return cuda_status(launch_reduce(j, nullptr, st));
 }
 
 // Q = T^T U (U [M, R]) -> outs
@@ -204,14 +229,16 @@ qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U
   CUtensorMap mt, mu;
   if (!map_bf16(&mt, T, ncols, M, ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mu, U, R, M, R, R, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
-  const ColPlan p = plan_colproj(M, ncols);
+  const SkPlan p = plan_colproj(M, ncols);
+  const int64_t ncc = cdiv(ncols, 64);
+  const ReduceJob j = reduce_job(part, ncc, 64, ncols, R, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_COLPROJ, st);
-    qlora_status s = cuda_status(launch_colproj(R, mt, mu, part, (int)M, (int)ncols, p.splits, p.mb_per, status, st));
+    const qlora_status s = cuda_status(launch_colproj(R, mt, mu, j, (int)cdiv(M, 64), status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(part, p.splits, (int)ncols, R, outs, st));
+  return cuda_status(launch_reduce(j, nullptr, st));
 }
 
 // G = T Bl^T ([M,16]) and Q = T^T U ([N,16]) from one read of T [M, N].
@@ -221,22 +248,19 @@ qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, con
   if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mu, U, 16, M, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mb, Bl, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  const DyPlan p = plan_dypass(M, N);
+  const SkPlan p = plan_dypass(M, N);
+  const int64_t nrc = cdiv(M, 64), nch = cdiv(N, 64), ncb = cdiv(nch, kDyCC);
   float* gpart = part;
-  float* qpart = reinterpret_cast<float*>(reinterpret_cast<char*>(part) +
-                                          align256(static_cast<size_t>(p.gsplits) * M * 16 * 4));
+  float* qpart = reinterpret_cast<float*>(reinterpret_cast<char*>(part) + dypass_gpart_bytes(M, N));
+  const ReduceJob jg = reduce_job(gpart, nrc, 64, M, 16, (int)ncb, (int)ncb, p.sp, gouts);
+  const ReduceJob jq = reduce_job(qpart, ncb, kDyCC * 64, N, 16, p.slot_cap, 0, p.sp, qouts);
   {
     KScope k(K_DYPASS, st);
-    qlora_status s = cuda_status(launch_dypass(mt, mu, mb, gpart, qpart, (int)M, (int)N, p.rc, status, st));
-    if (s != QLORA_OK) return s;
-  }
-  {
-    KScope k(K_REDUCE, st);
-    qlora_status s = cuda_status(launch_reduce(gpart, p.gsplits, (int)M, 16, gouts, st));
+    const qlora_status s = cuda_status(launch_dypass(mt, mu, mb, jg, jq, (int)nch, status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(qpart, p.qsplits, (int)N, 16, qouts, st));
+  return cuda_status(launch_reduce(jg, &jq, st));
 }
 
 ReduceOut rout(bf16* p, int col0, int ld, int transpose, float scale) { return {p, col0, ld, transpose, scale}; }
@@ -404,10 +428,23 @@ size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) 
 }
 
 namespace {
-// the staged weight sits at the end of a linear workspace
-bf16* linear_stage(void* ws, int64_t M, int64_t K, int64_t N) {
-  return reinterpret_cast<bf16*>(static_cast<char*>(ws) + qlora_linear_workspace_bytes(M, K, N, 16) -
-                                 stage_bytes(N, K));
+// Linear workspace: [status word | 256 B][M x 16 vector][partials][staged weight]
+struct LinearWs {
+  int* status;
+  bf16* vec;
+  float* part;
+  bf16* stage;
+};
+LinearWs carve_linear(void* ws, int64_t M, int64_t K, int64_t N) {
+  char* w = static_cast<char*>(ws);
+  LinearWs l;
+  l.status = reinterpret_cast<int*>(w);
+  l.vec = reinterpret_cast<bf16*>(w + 256);
+  l.part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
+  l.stage = is_staged(g_tiles) ? reinterpret_cast<bf16*>(w + qlora_linear_workspace_bytes(M, K, N, 16) -
+                                                         stage_bytes(N, K))
+                               : nullptr;
+  return l;
 }
 }  // namespace
 
@@ -423,19 +460,16 @@ qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
   if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(ws);
-  int* status = reinterpret_cast<int*>(w);
-  bf16* XAs = reinterpret_cast<bf16*>(w + 256);
-  float* part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
+  LinearWs l = carve_linear(ws, M, K, N);
   bf16* xa = reinterpret_cast<bf16*>(XA_saved);
   const bool scaled = lin->scale != 1.0f;
-  if (!scaled) XAs = xa;
-  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
-                   routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
+  bf16* XAs = scaled ? l.vec : xa;
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, l.part,
+                   routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)),
+                   l.status, st);
   if (s != QLORA_OK) return s;
-  const int tiles = g_tiles;
-  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, tiles,
-                  is_staged(tiles) ? linear_stage(ws, M, K, N) : nullptr, st);
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), l.status, g_tiles,
+                  l.stage, st);
 }
 
 qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
@@ -455,11 +489,11 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int tiles = g_tiles;
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  char* w = static_cast<char*>(ws);
-  int* status = reinterpret_cast<int*>(w);
-  bf16* sG = reinterpret_cast<bf16*>(w + 256);
-  bf16* stage = is_staged(tiles) ? linear_stage(ws, M, K, N) : nullptr;
-  float* part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
+  LinearWs l = carve_linear(ws, M, K, N);
+  int* status = l.status;
+  bf16* sG = l.vec;
+  bf16* stage = l.stage;
+  float* part = l.part;
   const float sc = lin->scale;
   // G = dY B^T (stored scaled: sG), dB = s (XA)^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, N, reinterpret_cast<const bf16*>(XA_saved),

@@ -52,13 +52,33 @@ struct GemmArgs {
 };
 
 // --------------------------------------------------------------- skinny ---
-// Rank-r products on warp-level mma.sync, split into fp32 partials that a
-// reduction kernel sums in a fixed order (deterministic).
-struct SkinnyMaps {
-  CUtensorMap t;   // main operand T: bf16 [rows, cols], box {64, 64}, 128B swizzle
-  CUtensorMap u;   // row-side factor U: bf16 [rows, R], box {R, 64}
-  CUtensorMap v;   // column-side factor: A-like [cols, R] box {R,64} or B-like [R, cols] box {64,R}
+// Rank-r products on warp-level mma.sync.  Each skinny kernel is persistent:
+// its P CTAs split the work units (64 x 64 tiles, or 64-row x 256-column
+// blocks) into P contiguous, equally sized ranges, so every CTA streams the
+// same number of bytes.  A CTA writes one fp32 partial per output group
+// (a 64-row or 256-column block of the result) it touches; a reduction kernel
+// adds each group's partials in slot order (deterministic).
+
+// Balanced contiguous partition of U units over P parts: part c owns
+// [part_begin(c), part_begin(c + 1)); part_owner(u) is the part that owns u.
+__host__ __device__ inline int part_begin(int c, int U, int P) {
+  return static_cast<int>(static_cast<int64_t>(c) * U / P);
+}
+__host__ __device__ inline int part_owner(int u, int U, int P) {
+  return static_cast<int>(((static_cast<int64_t>(u) + 1) * P - 1) / U);
+}
+
+// Partition of a skinny pass: U super-units of `align` units each over P CTAs;
+// output group g covers units [g * upg, (g + 1) * upg).
+struct SkPart {
+  int U, P, align, upg;
 };
+// CTA owning unit u, first slot CTA of group g, and number of slots of group g
+__host__ __device__ inline int sk_owner(const SkPart& p, int u) { return part_owner(u / p.align, p.U, p.P); }
+__host__ __device__ inline int sk_first(const SkPart& p, int g) { return sk_owner(p, g * p.upg); }
+__host__ __device__ inline int sk_slots(const SkPart& p, int g) {
+  return sk_owner(p, g * p.upg + p.upg - 1) - sk_first(p, g) + 1;
+}
 
 // Output of the partial-sum reduction: 16 of the R partial columns, scaled,
 // rounded to bf16 and written row-major or transposed.
@@ -71,6 +91,17 @@ struct ReduceOut {
 };
 struct ReduceOuts {
   ReduceOut o[4];
+};
+
+// Partials of one output of a skinny pass: part[g][slot][row in group][R] for
+// `groups` groups of `grows` rows (the last may extend past `rows`), slot_cap
+// slots per group; group g has `nslots` slots if nslots > 0, else
+// sk_slots(sp, g).  The reduction adds them in slot order and stores `outs`.
+struct ReduceJob {
+  float* part;
+  int groups, grows, rows, R, slot_cap, nslots;
+  SkPart sp;
+  ReduceOuts outs;
 };
 
 }  // namespace ql

@@ -6,17 +6,22 @@
 //   rowproj   P[m, :]  = T[m, :] V          V = [K, 16*NV] (LoRA A)     X A, H A_d
 //   colproj   Q[n, :]  = T[:, n]^T U        U = [M, R]                   X^T G (dA)
 //   dypass    G[m, :]  = T[m, :] B^T  and  Q[n, :] = T[:, n]^T U          dY B^T, (X A)^T dY
-// Each CTA streams 64x64 bf16 tiles of T through a TMA/mbarrier ring (the
-// kernels are HBM-bound on T) and writes fp32 partial sums over its slice of
-// the reduction; `reduce_partials_kernel` adds the slices in a fixed order,
-// applies the LoRA scale and rounds to bf16, so results are deterministic.
+// They are HBM-bound on T.  Each is persistent: its CTAs take equal
+// contiguous ranges of the work units; one producer warp streams 64x64 bf16
+// tiles of T (128B-swizzled) and the small factors through a 4-deep
+// TMA/mbarrier ring, four consumer warps contract them (16 rows or columns of
+// the tile each) and release each slot as soon as they are done with it.
+// Every CTA writes one fp32 partial per output group it touched;
+// `reduce_kernel` adds a group's partials in slot order, applies the LoRA
+// scale and rounds to bf16, so results are deterministic.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
+#include <cstring>
+
+
 namespace ql {
 
-constexpr int SK_THREADS = 128;
-constexpr int SK_STAGES = 4;
 constexpr int T_TILE = 64 * 64 * 2;  // bytes
 
 // A-fragment (16x16) of rows [r0, r0+16) and cols [c0, c0+16) of a 64x64
@@ -48,19 +53,80 @@ QL_DEV void frag_b_nk(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[2])
   ldsm_x2(tile + n * 128 + ((chunk ^ (n & 7)) << 4), b[0], b[1]);
 }
 
-// Uniform bounded wait for all threads of the CTA.
-QL_DEV bool cta_wait(uint32_t bar, uint32_t parity, int* status) {
-  const bool ok = mbar_wait(bar, parity, status);
-  return __syncthreads_and(ok) != 0;
+// ------------------------------------------------------------ pipeline ---
+constexpr int SK_CWARPS = 4;                         // consumer warps
+constexpr int SK_THREADS = 32 * (SK_CWARPS + 1);     // + the producer warp
+constexpr int SK_STAGES = 4;                         // 4 CTAs per SM: 16 consumer warps
+
+QL_DEV uint32_t sk_full(uint32_t bars, int s) { return bars + 8u * s; }
+QL_DEV uint32_t sk_empty(uint32_t bars, int s) { return bars + 8u * (SK_STAGES + s); }
+
+QL_DEV void sk_init(uint32_t bars) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SK_STAGES; ++s) {
+      mbar_init(sk_full(bars, s), 1);
+      mbar_init(sk_empty(bars, s), SK_CWARPS);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+}
+
+// Producer (one thread): issue(i, s, full_bar) loads tile i of the CTA's range
+// into slot s once the consumers released it; afterwards waits (bounded) until
+// every load it issued has landed, so no copy is in flight when the CTA exits.
+template <typename Issue>
+QL_DEV void sk_produce(int ntiles, uint32_t bars, int* status, Issue issue) {
+  int i = 0;
+  for (; i < ntiles; ++i) {
+    const int s = i % SK_STAGES;
+    if (!mbar_wait(sk_empty(bars, s), ((i / SK_STAGES) & 1) ^ 1, status)) break;
+    issue(i, s, sk_full(bars, s));
+  }
+  for (int j = i > SK_STAGES ? i - SK_STAGES : 0; j < i; ++j)
+    mbar_wait(sk_full(bars, j % SK_STAGES), (j / SK_STAGES) & 1, status);
+}
+
+// Consumer side of tile i: wait until it has landed (uniform over the warp).
+// After a failed wait the warp stops waiting (the status word holds the
+// timeout) and walks the rest of its tiles without touching them.
+QL_DEV bool sk_acquire(uint32_t bars, int i, bool ok, int* status) {
+  return ok && __all_sync(0xffffffffu, mbar_wait(sk_full(bars, i % SK_STAGES), (i / SK_STAGES) & 1, status));
+}
+// ... and hand the slot back (the fragments read from it are consumed by then).
+QL_DEV void sk_release(uint32_t bars, int i, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(sk_empty(bars, i % SK_STAGES));
+}
+
+// Tile range [t0, t1) of CTA c.
+QL_DEV void sk_range(const SkPart& sp, int units, int c, int& t0, int& t1) {
+  t0 = part_begin(c, sp.U, sp.P) * sp.align;
+  t1 = min(part_begin(c + 1, sp.U, sp.P) * sp.align, units);
+}
+
+// Store a warp's 16 x (8 * NB) accumulator block (mma C layout) at rows
+// [r0, r0 + 16) of a row-major fp32 [rows][ld] array, then clear it.
+template <int NB>
+QL_DEV void store_acc(float* base, int ld, int r0, int lane, float (&acc)[NB][4]) {
+  const int r = r0 + (lane >> 2);
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int c = nb * 8 + (lane & 3) * 2;
+    *reinterpret_cast<float2*>(base + static_cast<size_t>(r) * ld + c) = make_float2(acc[nb][0], acc[nb][1]);
+    *reinterpret_cast<float2*>(base + static_cast<size_t>(r + 8) * ld + c) = make_float2(acc[nb][2], acc[nb][3]);
+    acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+  }
 }
 
 // ------------------------------------------------------------- rowproj ---
-// part[ks][m][16*NV] = sum over this CTA's k-slice of T[m,k] * V_j[k, :]
+// Units: 64x64 tiles (rc, kc), kc fastest; group = row block rc (nkc units).
+// job.part[rc][slot][64][R]: T V over the CTA's tiles of row block rc.
 template <int NV>
 __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_v0,
                                                              const __grid_constant__ CUtensorMap tmap_v1,
-                                                             float* __restrict__ part, int M, int K, int kb_per_split,
+                                                             const __grid_constant__ ReduceJob job, int nkc,
                                                              int* status) {
   constexpr int R = 16 * NV;
   constexpr int V_TILE = 64 * 16 * 2;
@@ -69,64 +135,58 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bars = sbase + SK_STAGES * STAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 64;
-  const int ks = blockIdx.y;
-  const int kb0 = ks * kb_per_split;
-  const int nkb = min(K / 64 - kb0, kb_per_split);
+  const int c = blockIdx.x;
+  int t0, t1;
+  sk_range(job.sp, job.groups * nkc, c, t0, t1);
+  const int nt = t1 - t0;
+  sk_init(bars);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SK_STAGES; ++s) mbar_init(bars + 8 * s, 1);
-    fence_mbar_init();
+  if (warp == SK_CWARPS) {
+    if (lane == 0)
+      sk_produce(nt, bars, status, [&](int i, int s, uint32_t fb) {
+        const int t = t0 + i, rc = t / nkc, kc = t % nkc;
+        const uint32_t st = sbase + s * STAGE;
+        mbar_arrive_expect_tx(fb, STAGE);
+        tma_load_2d(st, &tmap_t, fb, kc * 64, rc * 64);
+        tma_load_2d(st + T_TILE, &tmap_v0, fb, 0, kc * 64);
+        if (NV == 2) tma_load_2d(st + T_TILE + V_TILE, &tmap_v1, fb, 0, kc * 64);
+      });
+    return;
   }
-  __syncthreads();
-  auto issue = [&](int it) {
-    const int s = it % SK_STAGES;
-    const uint32_t st = sbase + s * STAGE;
-    mbar_arrive_expect_tx(bars + 8 * s, STAGE);
-    const int k = (kb0 + it) * 64;
-    tma_load_2d(st, &tmap_t, bars + 8 * s, k, m0);
-    tma_load_2d(st + T_TILE, &tmap_v0, bars + 8 * s, 0, k);
-    if (NV == 2) tma_load_2d(st + T_TILE + V_TILE, &tmap_v1, bars + 8 * s, 0, k);
-  };
-  if (threadIdx.x == 0)
-    for (int it = 0; it < SK_STAGES && it < nkb; ++it) issue(it);
-
   float acc[R / 8][4] = {};
-  for (int it = 0; it < nkb; ++it) {
-    const int s = it % SK_STAGES;
-    if (!cta_wait(bars + 8 * s, (it / SK_STAGES) & 1, status)) return;
-    const uint32_t t = sbase + s * STAGE;
+  bool ok = true;
+  for (int i = 0; i < nt; ++i) {
+    const int t = t0 + i, rc = t / nkc, kc = t % nkc;
+    ok = sk_acquire(bars, i, ok, status);
+    if (ok) {
+      const uint32_t tb = sbase + (i % SK_STAGES) * STAGE;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t a[4];
-      frag_a_rows(t, warp * 16, kk * 16, lane, a);
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4];
+        frag_a_rows(tb, warp * 16, kk * 16, lane, a);
 #pragma unroll
-      for (int nb = 0; nb < R / 8; ++nb) {
-        uint32_t b[2];
-        frag_b_kn(t + T_TILE + (nb >> 1) * V_TILE, 32, kk * 16, (nb & 1) * 8, lane, b);
-        mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+        for (int nb = 0; nb < R / 8; ++nb) {
+          uint32_t b[2];
+          frag_b_kn(tb + T_TILE + (nb >> 1) * V_TILE, 32, kk * 16, (nb & 1) * 8, lane, b);
+          mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+        }
       }
+      sk_release(bars, i, lane);
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && it + SK_STAGES < nkb) issue(it + SK_STAGES);
-  }
-  const int r_lo = m0 + warp * 16 + (lane >> 2);
-  float* base = part + static_cast<size_t>(ks) * M * R;
-#pragma unroll
-  for (int nb = 0; nb < R / 8; ++nb) {
-    const int c = nb * 8 + (lane & 3) * 2;
-    if (r_lo < M) *reinterpret_cast<float2*>(base + static_cast<size_t>(r_lo) * R + c) = make_float2(acc[nb][0], acc[nb][1]);
-    if (r_lo + 8 < M)
-      *reinterpret_cast<float2*>(base + static_cast<size_t>(r_lo + 8) * R + c) = make_float2(acc[nb][2], acc[nb][3]);
+    if (kc == nkc - 1 || i == nt - 1) {
+      const int slot = c - sk_first(job.sp, rc);
+      store_acc(job.part + static_cast<size_t>(rc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
+    }
   }
 }
 
 // ------------------------------------------------------------- colproj ---
-// part[ms][n][R] = sum over this CTA's m-slice of T[m,n] * U[m, :]
+// Units: 64x64 tiles (cc, mc), mc fastest; group = column block cc (nmc units).
+// job.part[cc][slot][64][R]: T^T U over the CTA's tiles of column block cc.
 template <int R>
 __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_u,
-                                                             float* __restrict__ part, int M, int N, int mb_per_split,
+                                                             const __grid_constant__ ReduceJob job, int nmc,
                                                              int* status) {
   constexpr int U_TILE = 64 * R * 2;
   constexpr int STAGE = T_TILE + U_TILE;
@@ -134,68 +194,65 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bars = sbase + SK_STAGES * STAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * 64;
-  const int ms = blockIdx.y;
-  const int mb0 = ms * mb_per_split;
-  const int nmb = min((M + 63) / 64 - mb0, mb_per_split);
+  const int c = blockIdx.x;
+  int t0, t1;
+  sk_range(job.sp, job.groups * nmc, c, t0, t1);
+  const int nt = t1 - t0;
+  sk_init(bars);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SK_STAGES; ++s) mbar_init(bars + 8 * s, 1);
-    fence_mbar_init();
+  if (warp == SK_CWARPS) {
+    if (lane == 0)
+      sk_produce(nt, bars, status, [&](int i, int s, uint32_t fb) {
+        const int t = t0 + i, cc = t / nmc, mc = t % nmc;
+        const uint32_t st = sbase + s * STAGE;
+        mbar_arrive_expect_tx(fb, STAGE);
+        tma_load_2d(st, &tmap_t, fb, cc * 64, mc * 64);
+        tma_load_2d(st + T_TILE, &tmap_u, fb, 0, mc * 64);
+      });
+    return;
   }
-  __syncthreads();
-  auto issue = [&](int it) {
-    const int s = it % SK_STAGES;
-    const uint32_t st = sbase + s * STAGE;
-    mbar_arrive_expect_tx(bars + 8 * s, STAGE);
-    const int m = (mb0 + it) * 64;
-    tma_load_2d(st, &tmap_t, bars + 8 * s, n0, m);
-    tma_load_2d(st + T_TILE, &tmap_u, bars + 8 * s, 0, m);
-  };
-  if (threadIdx.x == 0)
-    for (int it = 0; it < SK_STAGES && it < nmb; ++it) issue(it);
-
   float acc[R / 8][4] = {};
-  for (int it = 0; it < nmb; ++it) {
-    const int s = it % SK_STAGES;
-    if (!cta_wait(bars + 8 * s, (it / SK_STAGES) & 1, status)) return;
-    const uint32_t t = sbase + s * STAGE;
+  bool ok = true;
+  for (int i = 0; i < nt; ++i) {
+    const int t = t0 + i, cc = t / nmc, mc = t % nmc;
+    ok = sk_acquire(bars, i, ok, status);
+    if (ok) {
+      const uint32_t tb = sbase + (i % SK_STAGES) * STAGE;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t a[4];
-      frag_a_cols(t, kk * 16, warp * 16, lane, a);
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4];
+        frag_a_cols(tb, kk * 16, warp * 16, lane, a);
 #pragma unroll
-      for (int nb = 0; nb < R / 8; ++nb) {
-        uint32_t b[2];
-        frag_b_kn(t + T_TILE, R * 2, kk * 16, nb * 8, lane, b);
-        mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+        for (int nb = 0; nb < R / 8; ++nb) {
+          uint32_t b[2];
+          frag_b_kn(tb + T_TILE, R * 2, kk * 16, nb * 8, lane, b);
+          mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+        }
       }
+      sk_release(bars, i, lane);
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && it + SK_STAGES < nmb) issue(it + SK_STAGES);
-  }
-  const int n_lo = n0 + warp * 16 + (lane >> 2);
-  float* base = part + static_cast<size_t>(ms) * N * R;
-#pragma unroll
-  for (int nb = 0; nb < R / 8; ++nb) {
-    const int c = nb * 8 + (lane & 3) * 2;
-    if (n_lo < N) *reinterpret_cast<float2*>(base + static_cast<size_t>(n_lo) * R + c) = make_float2(acc[nb][0], acc[nb][1]);
-    if (n_lo + 8 < N)
-      *reinterpret_cast<float2*>(base + static_cast<size_t>(n_lo + 8) * R + c) = make_float2(acc[nb][2], acc[nb][3]);
+    if (mc == nmc - 1 || i == nt - 1) {
+      const int slot = c - sk_first(job.sp, cc);
+      store_acc(job.part + static_cast<size_t>(cc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
+    }
   }
 }
 
 // -------------------------------------------------------------- dypass ---
 // One read of T = dY [M, N] gives both
-//   gpart[ns][m][16] = sum over this CTA's columns of T[m,n] * Bl[:, n]   (Bl = LoRA B, [16, N])
-//   qpart[ms][n][16] = sum over this CTA's rows    of T[m,n] * U[m, :]    (U = X A, [M, 16])
-// CTA tile: RC x 64 rows by CC x 64 columns, visited row-chunk major.
-template <int CC>
+//   G[m, :] = sum_n T[m,n] Bl[:, n]   (Bl = LoRA B, [16, N])
+//   Q[n, :] = sum_m T[m,n] U[m, :]    (U = X A, [M, 16])
+// Units: (cb, rc) = 64 rows x DY_CC column chunks of 64, rc fastest.
+//   gjob.part[rc][cb][64][16]: G over the unit's columns (one writer per unit);
+//   qjob.part[cb][slot][DY_CC * 64][16]: Q of column block cb over the CTA's rows.
+constexpr int DY_CC = 4;
 __global__ void __launch_bounds__(SK_THREADS) dypass_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                             const __grid_constant__ CUtensorMap tmap_u,
                                                             const __grid_constant__ CUtensorMap tmap_b,
-                                                            float* __restrict__ gpart, float* __restrict__ qpart,
-                                                            int M, int N, int rc_per_cta, int* status) {
+                                                            const __grid_constant__ ReduceJob gjob,
+                                                            const __grid_constant__ ReduceJob qjob, int nch,
+                                                            int* status) {
+  constexpr int CC = DY_CC;
   constexpr int U_TILE = 64 * 16 * 2;
   constexpr int B_TILE = 16 * 64 * 2;
   constexpr int STAGE = T_TILE + U_TILE + B_TILE;
@@ -203,111 +260,138 @@ __global__ void __launch_bounds__(SK_THREADS) dypass_kernel(const __grid_constan
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bars = sbase + SK_STAGES * STAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ns = blockIdx.x, ms = blockIdx.y;
-  const int n0 = ns * CC * 64;
-  const int m0 = ms * rc_per_cta * 64;
-  const int nrc = min((M - m0 + 63) / 64, rc_per_cta);
-  const int ncc = min((N - n0 + 63) / 64, CC);
-  const int total = nrc * ncc;
+  const int c = blockIdx.x;
+  const int nrc = gjob.groups, ncb = qjob.groups;
+  const SkPart& sp = qjob.sp;
+  int u0, u1;
+  sk_range(sp, ncb * nrc, c, u0, u1);
+  auto chunks = [&](int cb) { return min(CC, nch - cb * CC); };
+  int nt = 0;
+  for (int u = u0; u < u1; ++u) nt += chunks(u / nrc);
+  sk_init(bars);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SK_STAGES; ++s) mbar_init(bars + 8 * s, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  auto issue = [&](int it) {
-    const int s = it % SK_STAGES;
-    const uint32_t st = sbase + s * STAGE;
-    const int rc = it / ncc, cc = it % ncc;
-    mbar_arrive_expect_tx(bars + 8 * s, STAGE);
-    tma_load_2d(st, &tmap_t, bars + 8 * s, n0 + cc * 64, m0 + rc * 64);
-    tma_load_2d(st + T_TILE, &tmap_u, bars + 8 * s, 0, m0 + rc * 64);
-    tma_load_2d(st + T_TILE + U_TILE, &tmap_b, bars + 8 * s, n0 + cc * 64, 0);
-  };
-  if (threadIdx.x == 0)
-    for (int it = 0; it < SK_STAGES && it < total; ++it) issue(it);
-
-  float gacc[2][4];
-  float qacc[CC][2][4] = {};
-  for (int it = 0; it < total; ++it) {
-    const int rc = it / ncc, cc = it % ncc;
-    if (cc == 0) {
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) gacc[i][j] = 0.f;
-    }
-    const int s = it % SK_STAGES;
-    if (!cta_wait(bars + 8 * s, (it / SK_STAGES) & 1, status)) return;
-    const uint32_t t = sbase + s * STAGE;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t a[4];
-      // G += T[rows 16w.., cols kk*16..] * Bl^T
-      frag_a_rows(t, warp * 16, kk * 16, lane, a);
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        uint32_t b[2];
-        frag_b_nk(t + T_TILE + U_TILE, kk * 16, nb * 8, lane, b);
-        mma_bf16_16816(gacc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
-      }
-      // Q += T[rows kk*16.., cols 16w..]^T * U
-      frag_a_cols(t, kk * 16, warp * 16, lane, a);
-#pragma unroll
-      for (int c = 0; c < CC; ++c) {
-        if (c != cc) continue;
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          uint32_t b[2];
-          frag_b_kn(t + T_TILE, 32, kk * 16, nb * 8, lane, b);
-          mma_bf16_16816(qacc[c][nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+  if (warp == SK_CWARPS) {
+    if (lane == 0) {
+      int u = u0, cc = 0;
+      sk_produce(nt, bars, status, [&](int, int s, uint32_t fb) {
+        const int cb = u / nrc, rc = u % nrc, col = (cb * CC + cc) * 64;
+        const uint32_t st = sbase + s * STAGE;
+        mbar_arrive_expect_tx(fb, STAGE);
+        tma_load_2d(st, &tmap_t, fb, col, rc * 64);
+        tma_load_2d(st + T_TILE, &tmap_u, fb, 0, rc * 64);
+        tma_load_2d(st + T_TILE + U_TILE, &tmap_b, fb, col, 0);
+        if (++cc == chunks(cb)) {
+          cc = 0;
+          ++u;
         }
-      }
+      });
     }
-    __syncthreads();
-    if (threadIdx.x == 0 && it + SK_STAGES < total) issue(it + SK_STAGES);
-    if (cc == ncc - 1) {
-      const int r_lo = m0 + rc * 64 + warp * 16 + (lane >> 2);
-      float* base = gpart + static_cast<size_t>(ns) * M * 16;
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const int c = nb * 8 + (lane & 3) * 2;
-        if (r_lo < M) *reinterpret_cast<float2*>(base + static_cast<size_t>(r_lo) * 16 + c) = make_float2(gacc[nb][0], gacc[nb][1]);
-        if (r_lo + 8 < M)
-          *reinterpret_cast<float2*>(base + static_cast<size_t>(r_lo + 8) * 16 + c) = make_float2(gacc[nb][2], gacc[nb][3]);
-      }
-    }
+    return;
   }
-  float* qbase = qpart + static_cast<size_t>(ms) * N * 16;
+  float qacc[CC][2][4] = {};
+  int i = 0;
+  bool ok = true;
+  for (int u = u0; u < u1; ++u) {
+    const int cb = u / nrc, rc = u % nrc, ncc = chunks(cb);
+    float gacc[2][4] = {};
 #pragma unroll
-  for (int c = 0; c < CC; ++c) {
-    if (c >= ncc) break;
-    const int n_lo = n0 + c * 64 + warp * 16 + (lane >> 2);
+    for (int cc = 0; cc < CC; ++cc) {
+      if (cc >= ncc) break;
+      ok = sk_acquire(bars, i, ok, status);
+      if (ok) {
+        const uint32_t tb = sbase + (i % SK_STAGES) * STAGE;
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      const int col = nb * 8 + (lane & 3) * 2;
-      if (n_lo < N) *reinterpret_cast<float2*>(qbase + static_cast<size_t>(n_lo) * 16 + col) = make_float2(qacc[c][nb][0], qacc[c][nb][1]);
-      if (n_lo + 8 < N)
-        *reinterpret_cast<float2*>(qbase + static_cast<size_t>(n_lo + 8) * 16 + col) = make_float2(qacc[c][nb][2], qacc[c][nb][3]);
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t a[4];
+          // G += T[rows 16w.., cols kk*16..] * Bl^T
+          frag_a_rows(tb, warp * 16, kk * 16, lane, a);
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            uint32_t b[2];
+            frag_b_nk(tb + T_TILE + U_TILE, kk * 16, nb * 8, lane, b);
+            mma_bf16_16816(gacc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+          }
+          // Q += T[rows kk*16.., cols 16w..]^T * U
+          frag_a_cols(tb, kk * 16, warp * 16, lane, a);
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            uint32_t b[2];
+            frag_b_kn(tb + T_TILE, 32, kk * 16, nb * 8, lane, b);
+            mma_bf16_16816(qacc[cc][nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+          }
+        }
+        sk_release(bars, i, lane);
+      }
+      ++i;
+    }
+    store_acc(gjob.part + static_cast<size_t>(rc * ncb + cb) * 64 * 16, 16, warp * 16, lane, gacc);
+    if (u == u1 - 1 || (u + 1) / nrc != cb) {
+      float* qb = qjob.part + static_cast<size_t>(cb * qjob.slot_cap + c - sk_first(sp, cb)) * (CC * 64) * 16;
+#pragma unroll
+      for (int q = 0; q < CC; ++q) store_acc(qb + q * 64 * 16, 16, warp * 16, lane, qacc[q]);
     }
   }
 }
 
 // ------------------------------------------------------------- reduce ----
-// out = bf16(scale * sum_{s < S} part[s][row][c]), summed in s order.
-__global__ void reduce_partials_kernel(const float* __restrict__ part, int S, int rows, int R, ReduceOuts outs) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * R) return;
-  const int row = idx / R, c = idx % R;
-  float acc = 0.f;
-  for (int s = 0; s < S; ++s) acc += part[(static_cast<size_t>(s) * rows + row) * R + c];
+// out = bf16(scale * sum over the group's slots of part), summed in slot
+// order.  One thread per four consecutive partial columns; its slot loads are
+// issued sixteen at a time.  One launch serves up to two reductions.
+struct ReduceJobs {
+  ReduceJob j[2];
+  int n0, n1;  // float4 elements (rows * R / 4) of each job
+};
+__global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ ReduceJobs js) {
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = idx < js.n0 ? 0 : 1;
+  if (k == 1) idx -= js.n0;
+  if (idx >= (k ? js.n1 : js.n0)) return;
+  const ReduceJob& j = js.j[k];
+  const int row = (idx * 4) / j.R, c = (idx * 4) % j.R;
+  const int g = row / j.grows, r = row % j.grows;
+  const int ns = j.nslots > 0 ? j.nslots : sk_slots(j.sp, g);
+  const size_t slot_stride = static_cast<size_t>(j.grows) * j.R;
+  const float* p = j.part + static_cast<size_t>(g) * j.slot_cap * slot_stride + static_cast<size_t>(r) * j.R + c;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < ns; s += 16) {
+    float4 v[16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const ReduceOut& o = outs.o[j];
+    for (int q = 0; q < 16; ++q)
+      if (s + q < ns) v[q] = __ldg(reinterpret_cast<const float4*>(p + (s + q) * slot_stride));
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if (s + q < ns) {
+        acc.x += v[q].x;
+        acc.y += v[q].y;
+        acc.z += v[q].z;
+        acc.w += v[q].w;
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const ReduceOut& o = j.outs.o[q];
     if (o.ptr == nullptr || c < o.col0 || c >= o.col0 + 16) continue;
     const int cc = c - o.col0;
-    const size_t off = o.transpose ? static_cast<size_t>(cc) * o.ld + row : static_cast<size_t>(row) * o.ld + cc;
-    o.ptr[off] = __float2bfloat16_rn(o.scale * acc);
+    const bf16 b0 = __float2bfloat16_rn(o.scale * acc.x), b1 = __float2bfloat16_rn(o.scale * acc.y);
+    const bf16 b2 = __float2bfloat16_rn(o.scale * acc.z), b3 = __float2bfloat16_rn(o.scale * acc.w);
+    if (o.transpose) {
+      bf16* d = o.ptr + static_cast<size_t>(cc) * o.ld + row;
+      d[0] = b0;
+      d[o.ld] = b1;
+      d[2 * static_cast<size_t>(o.ld)] = b2;
+      d[3 * static_cast<size_t>(o.ld)] = b3;
+    } else {
+      __nv_bfloat162 lo, hi;
+      lo.x = b0;
+      lo.y = b1;
+      hi.x = b2;
+      hi.y = b3;
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&lo);
+      w.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(o.ptr + static_cast<size_t>(row) * o.ld + cc) = w;
+    }
   }
 }
 
@@ -315,54 +399,58 @@ __global__ void reduce_partials_kernel(const float* __restrict__ part, int S, in
 static cudaError_t set_smem(const void* f, int bytes) {
   return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
+static int sk_smem(int stage) { return SK_STAGES * stage + 2 * SK_STAGES * 8 + 1024; }
 
-cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1, float* part,
-                           int M, int K, int splits, int kb_per_split, int* status, cudaStream_t st) {
-  const dim3 grid((M + 63) / 64, splits);
+cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
+                           const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
+  const int smem = sk_smem(T_TILE + nv * 2048);
   if (nv == 1) {
-    const int smem = SK_STAGES * (T_TILE + 2048) + 64 + 1024;
     cudaError_t e = set_smem((const void*)rowproj_kernel<1>, smem);
     if (e != cudaSuccess) return e;
-    rowproj_kernel<1><<<grid, SK_THREADS, smem, st>>>(t, v0, v1, part, M, K, kb_per_split, status);
+    rowproj_kernel<1><<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
   } else {
-    const int smem = SK_STAGES * (T_TILE + 4096) + 64 + 1024;
     cudaError_t e = set_smem((const void*)rowproj_kernel<2>, smem);
     if (e != cudaSuccess) return e;
-    rowproj_kernel<2><<<grid, SK_THREADS, smem, st>>>(t, v0, v1, part, M, K, kb_per_split, status);
+    rowproj_kernel<2><<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, float* part, int M, int N, int splits,
-                           int mb_per_split, int* status, cudaStream_t st) {
-  const dim3 grid((N + 63) / 64, splits);
-  const int smem = SK_STAGES * (T_TILE + 64 * R * 2) + 64 + 1024;
+cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+                           int* status, cudaStream_t st) {
+  const int smem = sk_smem(T_TILE + 64 * R * 2);
   if (R == 16) {
     cudaError_t e = set_smem((const void*)colproj_kernel<16>, smem);
     if (e != cudaSuccess) return e;
-    colproj_kernel<16><<<grid, SK_THREADS, smem, st>>>(t, u, part, M, N, mb_per_split, status);
+    colproj_kernel<16><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
   } else {
     cudaError_t e = set_smem((const void*)colproj_kernel<32>, smem);
     if (e != cudaSuccess) return e;
-    colproj_kernel<32><<<grid, SK_THREADS, smem, st>>>(t, u, part, M, N, mb_per_split, status);
+    colproj_kernel<32><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
   }
   return cudaGetLastError();
 }
 
-constexpr int DY_CC = 4;
-cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, float* gpart, float* qpart,
-                          int M, int N, int rc_per_cta, int* status, cudaStream_t st) {
-  const dim3 grid((N + DY_CC * 64 - 1) / (DY_CC * 64), (M + rc_per_cta * 64 - 1) / (rc_per_cta * 64));
-  const int smem = SK_STAGES * (T_TILE + 2048 + 2048) + 64 + 1024;
-  cudaError_t e = set_smem((const void*)dypass_kernel<DY_CC>, smem);
+cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
+                          const ReduceJob& qjob, int nch, int* status, cudaStream_t st) {
+  const int smem = sk_smem(T_TILE + 2048 + 2048);
+  cudaError_t e = set_smem((const void*)dypass_kernel, smem);
   if (e != cudaSuccess) return e;
-  dypass_kernel<DY_CC><<<grid, SK_THREADS, smem, st>>>(t, u, b, gpart, qpart, M, N, rc_per_cta, status);
+  dypass_kernel<<<qjob.sp.P, SK_THREADS, smem, st>>>(t, u, b, gjob, qjob, nch, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_reduce(const float* part, int S, int rows, int R, const ReduceOuts& outs, cudaStream_t st) {
-  const int n = rows * R;
-  reduce_partials_kernel<<<(n + 255) / 256, 256, 0, st>>>(part, S, rows, R, outs);
+cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st) {
+  ReduceJobs js;
+  std::memset(&js, 0, sizeof(js));
+  js.j[0] = j0;
+  js.n0 = j0.rows * j0.R / 4;
+  if (j1) {
+    js.j[1] = *j1;
+    js.n1 = j1->rows * j1->R / 4;
+  }
+  const int n = js.n0 + js.n1;
+  reduce_kernel<<<(n + 255) / 256, 256, 0, st>>>(js);
   return cudaGetLastError();
 }
 
