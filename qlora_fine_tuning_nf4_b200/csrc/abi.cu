@@ -308,6 +308,16 @@ qlora_status stage_weight(const qlora_nf4& w, bf16* dst, cudaStream_t st) {
   KScope k(K_DEQUANT, st);
   return cuda_status(launch_nf4_dequantize(w.codes, w.absmax, w.n_out * w.k_in, dst, st, num_sms()));
 }
+// Output maps of the staged configuration's TMA-store epilogue: bf16 [rows, cols]
+// with row stride ld, written in 32 x 32 boxes (64B swizzle).  No-ops otherwise.
+bool map_outs(GemmMaps& maps, int tiles, int64_t rows, int64_t cols, int64_t ld, const void* o0,
+              const void* o1 = nullptr, const void* o2 = nullptr) {
+  if (!is_staged(tiles)) return true;
+  const void* o[3] = {o0, o1, o2};
+  for (int i = 0; i < 3; ++i)
+    if (o[i] && !map_bf16(&maps.out[i], o[i], cols, rows, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
+  return true;
+}
 // B-operand maps of one weight for either feed (stage: its bf16 buffer when staged)
 qlora_status map_weight(GemmMaps& maps, int i, const qlora_nf4& w, bool bwd, int tiles, bf16* stage,
                         cudaStream_t st) {
@@ -348,6 +358,7 @@ qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, co
   maps.b[1] = maps.b[0];
   maps.la[1] = maps.la[0];
   maps.lb[1] = maps.lb[0];
+  if (!map_outs(maps, tiles, M, N, N, Y)) return QLORA_ERR_CUDA;
   GemmArgs a;
   std::memset(&a, 0, sizeof(a));
   a.M = (int)M;
@@ -523,6 +534,7 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     a.lora = 1;
     a.ldo = (int)K;
     a.D = reinterpret_cast<bf16*>(dX);
+    if (!map_outs(maps, tiles, M, K, K, dX)) return QLORA_ERR_CUDA;
     a.status = status;
     a.group_m = kGroupM;
     KScope k(K_GEMM_BWD, st);
@@ -643,6 +655,7 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.E = reinterpret_cast<bf16*>(sv->E);
     a.G = reinterpret_cast<bf16*>(sv->G);
     a.H = reinterpret_cast<bf16*>(sv->H);
+    if (!map_outs(maps, tiles, M, h, h, sv->E, sv->G, sv->H)) return QLORA_ERR_CUDA;
     a.status = w.status;
     a.group_m = kGroupM;
     KScope k(K_GEMM_GLU_FWD, st);
@@ -716,6 +729,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.Gin = reinterpret_cast<const bf16*>(sv->G);
     a.dE = w.dE;
     a.dG = w.dG;
+    if (!map_outs(maps, tiles, M, h, h, w.dE, w.dG)) return QLORA_ERR_CUDA;
     a.status = w.status;
     a.group_m = kGroupM;
     KScope k(K_GEMM_GLU_BWD, st);
@@ -758,6 +772,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     a.lora = 2;
     a.ldo = (int)d;
     a.D = reinterpret_cast<bf16*>(dX);
+    if (!map_outs(maps, tiles, M, d, d, dX)) return QLORA_ERR_CUDA;
     a.status = w.status;
     a.group_m = kGroupM;
     KScope k(K_GEMM_BWD, st);

@@ -123,7 +123,7 @@ struct GemmCfg {
   static constexpr int B_BYTES = BNC * BK * 2;
   static constexpr int RC_BYTES = NB * 32;
   static constexpr int RA_BYTES = (MODE == MODE_BWD) ? 64 * 16 : BNC * 16;
-  static constexpr int S = ST ? 6 : ((CG == 1) ? 3 : (MH == 1 ? 5 : 4));  // operand stages
+  static constexpr int S = ST ? 5 : ((CG == 1) ? 3 : (MH == 1 ? 5 : 4));  // operand stages
   static constexpr int RS = ST ? 0 : ((CG == 1) ? 4 : (MH == 1 ? 6 : 8));  // raw stages
   static constexpr int LA_BYTES = BM * 16 * 2;   // one LoRA left operand tile (128 rows x 16)
   static constexpr int LBOP = BNC * 32;          // one LoRA right operand (BNC x 16 bf16)
@@ -133,7 +133,11 @@ struct GemmCfg {
   static constexpr int OFF_RA = OFF_RC + RS * RC_BYTES;
   static constexpr int OFF_LA = OFF_RA + RS * RA_BYTES;
   static constexpr int OFF_LB = OFF_LA + MH * 2 * LA_BYTES;
-  static constexpr int OFF_BAR = OFF_LB + 2 * LBOP;
+  static constexpr int OFF_EPI = OFF_LB + 2 * LBOP;
+  // staged feed: per epilogue warp three 32 x 32 bf16 output slots (64B-swizzled) for TMA stores
+  static constexpr int EPI_SLOT = 32 * 32 * 2;
+  static constexpr int EPI_BYTES = ST ? 8 * 3 * EPI_SLOT : 0;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int NBAR = 2 * S + 2 * RS + 7;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;  // + alignment slack
   static constexpr int EPI_WARPS = 8;            // two per TMEM lane quadrant
@@ -143,7 +147,8 @@ struct GemmCfg {
   static constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
   static constexpr int TMEM_COLS = 512;          // two accumulators of MH x BNT = 256 columns
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0 && OFF_LB % 1024 == 0, "1024B alignment");
+  static_assert(OFF_LA % 1024 == 0 && OFF_RA % 1024 == 0 && OFF_LB % 1024 == 0 && OFF_EPI % 1024 == 0,
+                "1024B alignment");
   static_assert(256 % NB == 0 && NB % 64 == 0, "dequantiser mapping");
 };
 
@@ -432,87 +437,198 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full0 + 8u * b, (tl >> 1) & 1, args.status))) break;
       tc_fence_after();
       const uint32_t tacc = tmem + b * 256 + (static_cast<uint32_t>(lg * 32) << 16);
-      if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
-        constexpr int CPH = C::BNT / 32;  // 32-column chunks per M-half
+      if constexpr (ST) {
+        // Output chunks (32 rows x 32 columns) go through this warp's shared
+        // slots and leave by TMA store, which writes whole lines and clips at
+        // the tensor's edges.
+        const uint32_t stg = sbase + C::OFF_EPI + ew * 3 * C::EPI_SLOT;
+        const uint64_t pol = l2_policy_evict_first();
+        uint8_t* stg_g = sgen + C::OFF_EPI + ew * 3 * C::EPI_SLOT;
+        // byte offset of 16-byte chunk q of this lane's row (64B swizzle)
+        auto soff = [&](int q) { return lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4); };
+        auto put = [&](int slot, int q, uint4 v) {
+          *reinterpret_cast<uint4*>(stg_g + slot * C::EPI_SLOT + soff(q)) = v;
+        };
+        if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
+          constexpr int CPH = C::BNT / 32;  // 32-column chunks per M-half
 #pragma unroll 1
-        for (int it = half * 4; it < half * 4 + 4; ++it) {
-          const int h = it / CPH, c = it % CPH;
-          const int grow = half_row(mb, h) + row;
-          const bool row_ok = grow < args.M;
-          const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
-          uint4 ec[4], gc[4];
-          if (EPI == EPI_GLU_BWD) {
-            // the chunk's saved e, g are requested before its TMEM load so the two latencies overlap
+          for (int it = half * 4; it < half * 4 + 4; ++it) {
+            const int h = it / CPH, c = it % CPH;
+            const int grow0 = half_row(mb, h) + lg * 32;
+            const int grow = grow0 + lane;
+            const int col0 = n0 + c * 32;
+            uint4 ec[4], gc[4];
+            if (EPI == EPI_GLU_BWD) {
+              const bool row_ok = grow < args.M;
+              const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int col = col0 + q * 8;
+                const bool in = row_ok && col < args.N;
+                ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
+                gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+              }
+            }
+            float v[32];
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, v);
+            if (lane == 0) bulk_wait_group_read<0>();  // the previous chunk's stores have read the slots
+            __syncwarp();
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const int col = n0 + c * 32 + q * 8;
-              const bool in = row_ok && col < args.N;
-              ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
-              gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+              if (EPI == EPI_STORE) {
+                uint4 o;
+                o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                put(0, q, o);
+              } else {
+                const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
+                const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
+                uint32_t de[4], dg[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float f0, d0, f1, d1;
+                  const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
+                  const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
+                  act_fg(args.act, e0, f0, d0);
+                  act_fg(args.act, e1, f1, d1);
+                  const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
+                  de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
+                  dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
+                }
+                put(0, q, make_uint4(de[0], de[1], de[2], de[3]));
+                put(1, q, make_uint4(dg[0], dg[1], dg[2], dg[3]));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out[0], stg, col0, grow0, pol);
+              if (EPI == EPI_GLU_BWD) tma_store_2d(&maps.out[1], stg + C::EPI_SLOT, col0, grow0, pol);
+              bulk_commit_group();
             }
           }
-          float v[32];
-          tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, v);
-          if (!row_ok) continue;
+        } else {  // EPI_GLU_FWD: per M-half, columns [0, BNT/2) hold e and [BNT/2, BNT) hold g
+          constexpr int CPH = C::BNT / 64;
+#pragma unroll 1
+          for (int it = half * 2; it < half * 2 + 2; ++it) {
+            const int h = it / CPH, c = it % CPH;
+            const int grow0 = half_row(mb, h) + lg * 32;
+            const int col0 = n0 + c * 32;
+            float e[32], g[32];
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, e);
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + C::BNT / 2 + c * 32, g);
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = n0 + c * 32 + q * 8;
-            if (col >= args.N) break;
-            if (EPI == EPI_STORE) {
-              uint4 o;
-              o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-              o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-              o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-              o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              *reinterpret_cast<uint4*>(args.D + rbase + col) = o;
-            } else {
-              const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
-              const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
-              uint32_t de[4], dg[4];
+            for (int q = 0; q < 4; ++q) {
+              uint32_t ewv[4], gwv[4], hwv[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                float f0, d0, f1, d1;
-                const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
-                const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
-                act_fg(args.act, e0, f0, d0);
-                act_fg(args.act, e1, f1, d1);
-                const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
-                de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
-                dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
+                const float e0 = e[q * 8 + 2 * i], e1 = e[q * 8 + 2 * i + 1];
+                const float g0 = g[q * 8 + 2 * i], g1 = g[q * 8 + 2 * i + 1];
+                ewv[i] = pack_bf16x2(e0, e1);
+                gwv[i] = pack_bf16x2(g0, g1);
+                hwv[i] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
               }
-              *reinterpret_cast<uint4*>(args.dE + rbase + col) = make_uint4(de[0], de[1], de[2], de[3]);
-              *reinterpret_cast<uint4*>(args.dG + rbase + col) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              put(0, q, make_uint4(ewv[0], ewv[1], ewv[2], ewv[3]));
+              put(1, q, make_uint4(gwv[0], gwv[1], gwv[2], gwv[3]));
+              put(2, q, make_uint4(hwv[0], hwv[1], hwv[2], hwv[3]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out[0], stg, col0, grow0, pol);
+              tma_store_2d(&maps.out[1], stg + C::EPI_SLOT, col0, grow0, pol);
+              tma_store_2d(&maps.out[2], stg + 2 * C::EPI_SLOT, col0, grow0, pol);
+              bulk_commit_group();
             }
           }
         }
-      } else {  // EPI_GLU_FWD: per M-half, columns [0, BNT/2) hold e and [BNT/2, BNT) hold g
-        constexpr int CPH = C::BNT / 64;  // (e, g) chunk pairs per M-half
-#pragma unroll 1
-        for (int it = half * 2; it < half * 2 + 2; ++it) {
-          const int h = it / CPH, c = it % CPH;
-          const int grow = half_row(mb, h) + row;
-          const bool row_ok = grow < args.M;
-          const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
-          float e[32], g[32];
-          tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, e);
-          tmem_ld_32x32b_x32(tacc + h * C::BNT + C::BNT / 2 + c * 32, g);
-          if (!row_ok) continue;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = n0 + c * 32 + q * 8;
-            if (col >= args.N) break;
-            uint32_t ewv[4], gwv[4], hwv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float e0 = e[q * 8 + 2 * i], e1 = e[q * 8 + 2 * i + 1];
-              const float g0 = g[q * 8 + 2 * i], g1 = g[q * 8 + 2 * i + 1];
-              ewv[i] = pack_bf16x2(e0, e1);
-              gwv[i] = pack_bf16x2(g0, g1);
-              hwv[i] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
+      } else {
+        if (EPI == EPI_STORE || EPI == EPI_GLU_BWD) {
+          constexpr int CPH = C::BNT / 32;  // 32-column chunks per M-half
+  #pragma unroll 1
+          for (int it = half * 4; it < half * 4 + 4; ++it) {
+            const int h = it / CPH, c = it % CPH;
+            const int grow = half_row(mb, h) + row;
+            const bool row_ok = grow < args.M;
+            const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
+            uint4 ec[4], gc[4];
+            if (EPI == EPI_GLU_BWD) {
+              // the chunk's saved e, g are requested before its TMEM load so the two latencies overlap
+  #pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int col = n0 + c * 32 + q * 8;
+                const bool in = row_ok && col < args.N;
+                ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
+                gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+              }
             }
-            *reinterpret_cast<uint4*>(args.E + rbase + col) = make_uint4(ewv[0], ewv[1], ewv[2], ewv[3]);
-            *reinterpret_cast<uint4*>(args.G + rbase + col) = make_uint4(gwv[0], gwv[1], gwv[2], gwv[3]);
-            *reinterpret_cast<uint4*>(args.H + rbase + col) = make_uint4(hwv[0], hwv[1], hwv[2], hwv[3]);
+            float v[32];
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, v);
+            if (!row_ok) continue;
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = n0 + c * 32 + q * 8;
+              if (col >= args.N) break;
+              if (EPI == EPI_STORE) {
+                uint4 o;
+                o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                *reinterpret_cast<uint4*>(args.D + rbase + col) = o;
+              } else {
+                const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
+                const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
+                uint32_t de[4], dg[4];
+  #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float f0, d0, f1, d1;
+                  const float e0 = bf16_lo(ewv[i]), e1 = bf16_hi(ewv[i]);
+                  const float g0 = bf16_lo(gwv[i]), g1 = bf16_hi(gwv[i]);
+                  act_fg(args.act, e0, f0, d0);
+                  act_fg(args.act, e1, f1, d1);
+                  const float h0 = v[q * 8 + 2 * i], h1 = v[q * 8 + 2 * i + 1];
+                  de[i] = pack_bf16x2(h0 * g0 * d0, h1 * g1 * d1);
+                  dg[i] = pack_bf16x2(h0 * f0, h1 * f1);
+                }
+                *reinterpret_cast<uint4*>(args.dE + rbase + col) = make_uint4(de[0], de[1], de[2], de[3]);
+                *reinterpret_cast<uint4*>(args.dG + rbase + col) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+              }
+            }
+          }
+        } else {  // EPI_GLU_FWD: per M-half, columns [0, BNT/2) hold e and [BNT/2, BNT) hold g
+          constexpr int CPH = C::BNT / 64;  // (e, g) chunk pairs per M-half
+  #pragma unroll 1
+          for (int it = half * 2; it < half * 2 + 2; ++it) {
+            const int h = it / CPH, c = it % CPH;
+            const int grow = half_row(mb, h) + row;
+            const bool row_ok = grow < args.M;
+            const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
+            float e[32], g[32];
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, e);
+            tmem_ld_32x32b_x32(tacc + h * C::BNT + C::BNT / 2 + c * 32, g);
+            if (!row_ok) continue;
+  #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = n0 + c * 32 + q * 8;
+              if (col >= args.N) break;
+              uint32_t ewv[4], gwv[4], hwv[4];
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float e0 = e[q * 8 + 2 * i], e1 = e[q * 8 + 2 * i + 1];
+                const float g0 = g[q * 8 + 2 * i], g1 = g[q * 8 + 2 * i + 1];
+                ewv[i] = pack_bf16x2(e0, e1);
+                gwv[i] = pack_bf16x2(g0, g1);
+                hwv[i] = pack_bf16x2(act_f(args.act, e0) * g0, act_f(args.act, e1) * g1);
+              }
+              *reinterpret_cast<uint4*>(args.E + rbase + col) = make_uint4(ewv[0], ewv[1], ewv[2], ewv[3]);
+              *reinterpret_cast<uint4*>(args.G + rbase + col) = make_uint4(gwv[0], gwv[1], gwv[2], gwv[3]);
+              *reinterpret_cast<uint4*>(args.H + rbase + col) = make_uint4(hwv[0], hwv[1], hwv[2], hwv[3]);
+            }
           }
         }
       }
@@ -524,6 +640,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
         else mbar_arrive(acc_empty0 + 8u * b);
       }
     }
+    if (ST && lane == 0) bulk_wait_group<0>();  // output stores complete before the CTA exits
   } else if constexpr (!ST) {
     // --------------------------------------------------- dequantisers ----
     const int dq = (warp - C::DQ_WARP0) * 32 + lane;  // 0..255

@@ -29,6 +29,7 @@ struct GemmMaps {
   CUtensorMap la[2];      // LoRA left operand(s): bf16 [M, 16], box {16,128}, 32B swizzle
   CUtensorMap lb[2];      // LoRA right operand(s)
   CUtensorMap b[2];       // staged feed only: the dequantised bf16 weight, matching codes[]
+  CUtensorMap out[3];     // staged feed only: outputs (D | E, G, H | dE, dG), box {32,32}, 64B swizzle
 };
 
 struct GemmArgs {

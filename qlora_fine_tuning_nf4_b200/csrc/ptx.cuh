@@ -113,6 +113,32 @@ QL_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, uint32_t cbar, 
       : "memory");
 }
 QL_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// L2 policy that marks lines as the first to evict (streaming outputs that
+// should not displace operands other CTAs still re-read).
+QL_DEV uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// 2-D tiled store from this CTA's shared memory (bulk-group completion) with
+// an L2 cache policy; parts of the box outside the tensor are not written.
+QL_DEV void tma_store_2d(const CUtensorMap* m, uint32_t src, int x, int y, uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(src), "r"(x), "r"(y), "l"(policy)
+               : "memory");
+}
+QL_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed bulk groups still read their shared-memory source
+template <int N>
+QL_DEV void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// wait until at most N committed bulk groups are still in flight
+template <int N>
+QL_DEV void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // -------------------------------------------------------------- tcgen05 ---
 template <int CG>
