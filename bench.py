@@ -14,6 +14,7 @@ instead (rank 0 only) on a bounded row sample of the same workload.
 """
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -37,7 +38,7 @@ L2_NOTE = "inputs larger than L2 (saved E/G/H and dE/dG are 5 x 172 MiB per step
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
@@ -100,8 +101,8 @@ def smi_device_id(local):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle sampling during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi clocks/throttle sampling; only samples stamped inside the timed window count."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
@@ -112,32 +113,38 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                          "-lms", "50", "-i", str(self.dev)], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0, t1):
+        """Summary of the samples stamped in [t0, t1] (host wall-clock seconds)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        sm, mx, reasons = [], None, set()
+        sm, pw, mx, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, top, power = float(f[2]), float(f[3]), float(f[4])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            if not t0 <= ts <= t1:
+                continue
+            sm.append(clk)
+            pw.append(power)
+            mx = top
+            for n, v in zip(names, f[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w": statistics.median(pw) if pw else None, "samples": len(sm)}
 
 
 # ------------------------------------------------------------ oracle arm ---
@@ -269,6 +276,9 @@ def run_ours(args, wl):
             dist.all_reduce(flat)
 
     stream = torch.cuda.current_stream()
+    clk = ClockSampler(smi_device_id(local))
+    clk.start()
+    time.sleep(0.5)  # the sampler's first sample lands before the timed window
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -280,11 +290,9 @@ def run_ours(args, wl):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    clk = ClockSampler(smi_device_id(local))
     launches0 = ops.qlora_launch_count()
     barrier()
-    clk.start()
-    time.sleep(0.3)
+    t_begin = time.time()
     ops.qlora_trace_begin()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -292,9 +300,10 @@ def run_ours(args, wl):
         step()
     e1.record(stream)
     barrier()
+    t_end = time.time()
     ms = e0.elapsed_time(e1)
     trace = ops.qlora_trace_end()
-    clocks = clk.stop()
+    clocks = clk.stop(t_begin, t_end)
     launches = ops.qlora_launch_count() - launches0
     if ops.qlora_last_device_status(ws) != 0:
         raise RuntimeError("device status error during the timed region")
@@ -356,6 +365,14 @@ def run_ours(args, wl):
                 "share_of_step": tot / ms}
     kernels = {k: {"launches": v[0], "ms_total": round(v[1], 4), "share": round(v[1] / ms, 4)}
                for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])}
+    # HBM-bound staging dequantisation: algorithmic bytes (codes + absmax read, bf16 written) per step
+    dq = None
+    if "nf4_dequantize" in trace:
+        n_l, tot = trace["nf4_dequantize"]
+        dq_bytes = args.steps * 2 * (2 * h * d + h * d) * (0.5 + 4 / 64 + 2)  # gate, up, down in fwd and in bwd
+        gbs = dq_bytes / (tot / 1e3) / 1e9
+        dq = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+              "launches": n_l, "ms_per_step": tot / args.steps}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -381,6 +398,7 @@ def run_ours(args, wl):
                 "steps": e2e_steps},
         "gpu_launches": launches,
         "roofline": roof,
+        "dequant": dq,
         "kernels": kernels,
         "cpu_baseline": cpu,
         "clocks": clocks,

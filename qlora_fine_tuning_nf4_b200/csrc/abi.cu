@@ -18,7 +18,8 @@
 namespace ql {
 // kernels implemented in the other translation units
 cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st);
-cudaError_t launch_nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t numel, bf16* out,
+cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
+                                  const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
                                   cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
@@ -304,9 +305,12 @@ bool map_staged(CUtensorMap* m, const bf16* wq, const qlora_nf4& w, bool bwd, in
   if (!bwd) return map_bf16(m, wq, K, N, K, 64, bnc < 128 ? bnc : 128, CU_TENSOR_MAP_SWIZZLE_128B);
   return map_bf16(m, wq, K, N, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-qlora_status stage_weight(const qlora_nf4& w, bf16* dst, cudaStream_t st) {
+// Dequantises one weight (w1 == nullptr) or two in one launch into their staging buffers.
+qlora_status stage_weights(const qlora_nf4& w0, bf16* dst0, const qlora_nf4* w1, bf16* dst1, cudaStream_t st) {
   KScope k(K_DEQUANT, st);
-  return cuda_status(launch_nf4_dequantize(w.codes, w.absmax, w.n_out * w.k_in, dst, st, num_sms()));
+  return cuda_status(launch_nf4_dequantize(w0.codes, w0.absmax, w0.n_out * w0.k_in, dst0, w1 ? w1->codes : nullptr,
+                                           w1 ? w1->absmax : nullptr, w1 ? w1->n_out * w1->k_in : 0, dst1, st,
+                                           num_sms()));
 }
 // Output maps of the staged configuration's TMA-store epilogue: bf16 [rows, cols]
 // with row stride ld, written in 32 x 32 boxes (64B swizzle).  No-ops otherwise.
@@ -318,16 +322,21 @@ bool map_outs(GemmMaps& maps, int tiles, int64_t rows, int64_t cols, int64_t ld,
     if (o[i] && !map_bf16(&maps.out[i], o[i], cols, rows, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
   return true;
 }
-// B-operand maps of one weight for either feed (stage: its bf16 buffer when staged)
-qlora_status map_weight(GemmMaps& maps, int i, const qlora_nf4& w, bool bwd, int tiles, bf16* stage,
-                        cudaStream_t st) {
+// B-operand maps of one weight (w1 == nullptr) or two (GEMM segments / gate-up halves 0 and 1) for
+// either feed; under the staged feed the weights are first dequantised into stage0 / stage1.
+qlora_status map_weights(GemmMaps& maps, const qlora_nf4& w0, const qlora_nf4* w1, bool bwd, int tiles,
+                         bf16* stage0, bf16* stage1, cudaStream_t st) {
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   if (is_staged(tiles)) {
-    const qlora_status s = stage_weight(w, stage, st);
+    const qlora_status s = stage_weights(w0, stage0, w1, stage1, st);
     if (s != QLORA_OK) return s;
-    return map_staged(&maps.b[i], stage, w, bwd, bnc) ? QLORA_OK : QLORA_ERR_CUDA;
+    if (!map_staged(&maps.b[0], stage0, w0, bwd, bnc)) return QLORA_ERR_CUDA;
+    if (w1 && !map_staged(&maps.b[1], stage1, *w1, bwd, bnc)) return QLORA_ERR_CUDA;
+    return QLORA_OK;
   }
-  return map_nf4(&maps.codes[i], &maps.absmax[i], w, bwd, bnc) ? QLORA_OK : QLORA_ERR_CUDA;
+  if (!map_nf4(&maps.codes[0], &maps.absmax[0], w0, bwd, bnc)) return QLORA_ERR_CUDA;
+  if (w1 && !map_nf4(&maps.codes[1], &maps.absmax[1], *w1, bwd, bnc)) return QLORA_ERR_CUDA;
+  return QLORA_OK;
 }
 
 qlora_status check_linear(const qlora_lora_linear* lin) {
@@ -348,7 +357,7 @@ qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, co
   std::memset(&maps, 0, sizeof(maps));
   const int64_t K = lin.w.k_in, N = lin.w.n_out;
   if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  const qlora_status s = map_weight(maps, 0, lin.w, false, tiles, stage, st);
+  const qlora_status s = map_weights(maps, lin.w, nullptr, false, tiles, stage, nullptr, st);
   if (s != QLORA_OK) return s;
   if (!map_bf16(&maps.la[0], XAs, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&maps.lb[0], lin.B, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -426,7 +435,8 @@ qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n
   if (misaligned(codes) || misaligned(absmax) || misaligned(out)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   KScope k(K_DEQUANT, st);
-  return cuda_status(launch_nf4_dequantize(codes, absmax, n_out * k_in, reinterpret_cast<bf16*>(out), st, num_sms()));
+  return cuda_status(launch_nf4_dequantize(codes, absmax, n_out * k_in, reinterpret_cast<bf16*>(out), nullptr, nullptr,
+                                           0, nullptr, st, num_sms()));
 }
 
 size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
@@ -516,7 +526,7 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, N, M, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if ((s = map_weight(maps, 0, lin->w, true, tiles, stage, st)) != QLORA_OK) return s;
+    if ((s = map_weights(maps, lin->w, nullptr, true, tiles, stage, nullptr, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], sG, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
       return QLORA_ERR_CUDA;
@@ -638,8 +648,7 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
-    if ((s = map_weight(maps, 0, gate->w, false, tiles, w.stage0, st)) != QLORA_OK) return s;
-    if ((s = map_weight(maps, 1, up->w, false, tiles, w.stage1, st)) != QLORA_OK) return s;
+    if ((s = map_weights(maps, gate->w, &up->w, false, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], xags, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], xaus, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], gate->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -707,7 +716,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if ((s = map_weight(maps, 0, down->w, true, tiles, w.stage0, st)) != QLORA_OK) return s;
+    if ((s = map_weights(maps, down->w, nullptr, true, tiles, w.stage0, nullptr, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], sGd, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
       return QLORA_ERR_CUDA;
@@ -755,8 +764,7 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if ((s = map_weight(maps, 0, gate->w, true, tiles, w.stage0, st)) != QLORA_OK) return s;
-    if ((s = map_weight(maps, 1, up->w, true, tiles, w.stage1, st)) != QLORA_OK) return s;
+    if ((s = map_weights(maps, gate->w, &up->w, true, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
     if (!map_bf16(&maps.la[0], w.gu, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.la[1], w.gu + 16, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))

@@ -53,18 +53,32 @@ __global__ void nf4_quantize_kernel(const bf16* __restrict__ w, int64_t nblocks,
   if (lane == 0) absmax[blk] = m;
 }
 
-// Each warp handles runs of 1024 elements: lane l takes 8 consecutive
-// elements at offsets 8l + 256i (i = 0..3), so every warp-wide load of codes
-// is 128 contiguous bytes and every store of bf16 is 512 contiguous bytes.
-__global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes, const float* __restrict__ absmax,
-                                      int64_t numel, bf16* __restrict__ out) {
+// Dequantisation of up to two tensors in one launch.  A warp takes runs of
+// 1024 elements: lane l expands the 8 elements at 8l + 256i (i = 0..3), so
+// each warp-wide load of codes is 128 contiguous bytes and each bf16 store
+// 512 contiguous bytes.  The 16 levels sit in shared memory (lanes reading
+// the same level are served by one broadcast).
+struct DqJob {
+  const uint8_t* codes;
+  const float* absmax;
+  bf16* out;
+  int64_t runs;  // numel / 1024, rounded up
+  int64_t numel;
+};
+__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, const DqJob j1) {
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = __uint_as_float(c_nf4_bits[threadIdx.x]);
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  for (int64_t base = wid * 1024; base < numel; base += warps * 1024) {
+  const int64_t total = j0.runs + j1.runs;
+  for (int64_t run = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; run < total; run += warps) {
+    const bool second = run >= j0.runs;
+    const int64_t base = (second ? run - j0.runs : run) * 1024;
+    const uint8_t* codes = second ? j1.codes : j0.codes;
+    const float* absmax = second ? j1.absmax : j0.absmax;
+    bf16* out = second ? j1.out : j0.out;
+    const int64_t numel = second ? j1.numel : j0.numel;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t e = base + i * 256 + lane * 8;
@@ -90,14 +104,17 @@ cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t numel, bf16* out,
+// Dequantises one tensor, or two (codes1 != nullptr) in the same launch.
+cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
+                                  const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
                                   cudaStream_t st, int num_sms) {
-  const int64_t chunks = (numel + 1023) / 1024;  // one warp-run each
-  int64_t grid = (chunks + 7) / 8;               // 8 warps per CTA
-  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  DqJob j0 = {codes0, absmax0, out0, (numel0 + 1023) / 1024, numel0};
+  DqJob j1 = {codes1, absmax1, out1, codes1 ? (numel1 + 1023) / 1024 : 0, codes1 ? numel1 : 0};
+  int64_t grid = (j0.runs + j1.runs + 7) / 8;             // one run per warp, 8 warps per CTA
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 CTAs of 256 threads per SM
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  nf4_dequantize_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(codes, absmax, numel, out);
+  nf4_dequantize_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(j0, j1);
   return cudaGetLastError();
 }
 
