@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
+    ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
+                    help="frozen base format: NF4 (QLoRA, the metric) or bf16 (plain LoRA, for comparison)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override M (tokens per GPU) for small profiling cases; 0 = the workload's M")
     return ap.parse_args()
@@ -251,8 +253,13 @@ def run_ours(args, wl):
     p = make_mlp_problem(M, d, h, r, wl["alpha"], wl["seed"] + 1000 * rank)
     lins = {}
     for k in ("g", "u", "d"):
-        w = ops.nf4_quantize(bits_to_torch(p["W_" + k], dev))
-        lins[k] = ops.LoraLinear(w, bits_to_torch(p["A_" + k], dev), bits_to_torch(p["B_" + k], dev), p["s"])
+        A, B = bits_to_torch(p["A_" + k], dev), bits_to_torch(p["B_" + k], dev)
+        if args.weights == "nf4":
+            lins[k] = ops.LoraLinear(ops.nf4_quantize(bits_to_torch(p["W_" + k], dev)), A, B, p["s"])
+        else:
+            lins[k] = ops.LoraLinear16(bits_to_torch(p["W_" + k], dev), A, B, p["s"])
+    mlp_fwd = ops.qlora_mlp_fwd if args.weights == "nf4" else ops.qlora_mlp16_fwd
+    mlp_bwd = ops.qlora_mlp_bwd if args.weights == "nf4" else ops.qlora_mlp16_bwd
     X = bits_to_torch(p["X"], dev)
     dY = bits_to_torch(p["dY"], dev)
     del p
@@ -270,8 +277,8 @@ def run_ours(args, wl):
     grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
 
     def step():
-        ops.qlora_mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws, Y=Y, saved=saved)
-        ops.qlora_mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads)
+        mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws, Y=Y, saved=saved)
+        mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads)
         if world > 1:
             dist.all_reduce(flat)
 
@@ -393,7 +400,8 @@ def run_ours(args, wl):
         "frac_of_bf16_peak_sustained": value / world / pk["bf16_sustained"],
         "config": {"workload": args.workload, "M_per_gpu": M, "d": d, "h": h, "r": r, "act": act,
                    "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
-                   "gemm_tiles": ops.TILE_CONFIGS[args.tiles], "l2": L2_NOTE},
+                   "gemm_tiles": ops.TILE_CONFIGS[4 if args.weights == "bf16" else args.tiles],
+                   "base_weights": args.weights, "l2": L2_NOTE},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": launches,

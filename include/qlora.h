@@ -86,6 +86,20 @@ typedef struct {
   float scale; /* s = alpha / r */
 } qlora_lora_linear;
 
+/* One projection with a frozen bf16 base W [n_out, k_in] (row-major) instead
+ * of NF4: plain LoRA rather than QLoRA (Mistral blog FAQ, "load_in_4bit set
+ * to False"; Show HN highlight 7, 4-bit and 16-bit LoRA).  Same LoRA factors
+ * and scale as qlora_lora_linear. */
+typedef struct {
+  const qlora_bf16* w;
+  int64_t n_out;
+  int64_t k_in;
+  const qlora_bf16* A;
+  const qlora_bf16* B;
+  int32_t r;   /* must be 16 */
+  float scale; /* s = alpha / r */
+} qlora_lora_linear16;
+
 /* Tensors the MLP forward saves for its backward (caller-allocated):
  * E, G, H [M, h] (e = gate projection, g = up projection, h = act(e) * g),
  * XA_g, XA_u [M, r] (X A_g, X A_u) and HA_d [M, r] (H A_d). */
@@ -167,6 +181,33 @@ QLORA_API qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gat
                            const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
                            qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* workspace,
                            size_t workspace_bytes, qlora_stream_t stream);
+
+/* The same four computations with bf16 base weights (qlora_lora_linear16):
+ * outputs, saved tensors, shapes, workspace rules and errors as the NF4 calls
+ * above, with dequant(W) replaced by W itself.  They always run the CTA-pair
+ * GEMM that streams the weight by TMA (tile configuration 4), whatever
+ * qlora_set_tile_config selected, and need no room for a staged weight: the
+ * *16_workspace_bytes queries give their sizes.  The three weights of an MLP
+ * call must all be bf16. */
+QLORA_API size_t qlora_linear16_workspace_bytes(int64_t M, int64_t k_in, int64_t n_out, int32_t r);
+QLORA_API size_t qlora_mlp16_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r);
+QLORA_API qlora_status qlora_linear16_fwd(const qlora_lora_linear16* lin, const qlora_bf16* X, int64_t M,
+                                          qlora_bf16* Y, qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes,
+                                          qlora_stream_t stream);
+QLORA_API qlora_status qlora_linear16_bwd(const qlora_lora_linear16* lin, const qlora_bf16* X,
+                                          const qlora_bf16* XA_saved, const qlora_bf16* dY, int64_t M, qlora_bf16* dX,
+                                          qlora_bf16* dA, qlora_bf16* dB, void* workspace, size_t workspace_bytes,
+                                          qlora_stream_t stream);
+QLORA_API qlora_status qlora_mlp16_fwd(qlora_act act, const qlora_lora_linear16* gate,
+                                       const qlora_lora_linear16* up, const qlora_lora_linear16* down,
+                                       const qlora_bf16* X, int64_t M, qlora_bf16* Y, const qlora_mlp_saved* saved,
+                                       void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+QLORA_API qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16* gate,
+                                       const qlora_lora_linear16* up, const qlora_lora_linear16* down,
+                                       const qlora_bf16* X, const qlora_mlp_saved* saved, const qlora_bf16* dY,
+                                       int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                                       qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
+                                       void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* Reads the device status word in `workspace` (synchronising `stream`),
  * clears it, and maps it to a status: QLORA_OK, QLORA_ERR_TIMEOUT or

@@ -62,6 +62,24 @@ int32_t g_tiles = 4;  // GEMM tile configuration (see qlora_set_tile_config)
 #endif
 constexpr int kGroupM = QL_GROUP_M;  // output-row tiles per group of the GEMM tile order
 
+// Internal view of one projection: a frozen NF4 base (codes + absmax) or a
+// frozen bf16 base (w16), plus its LoRA factors.
+struct Wt {
+  const uint8_t* codes;
+  const float* absmax;
+  const qlora_bf16* w16;
+  int64_t n_out, k_in;
+};
+struct Lin {
+  Wt w;
+  const qlora_bf16* A;
+  const qlora_bf16* B;
+  int32_t r;
+  float scale;
+};
+Lin lin_of(const qlora_lora_linear& l) { return {{l.w.codes, l.w.absmax, nullptr, l.w.n_out, l.w.k_in}, l.A, l.B, l.r, l.scale}; }
+Lin lin_of(const qlora_lora_linear16& l) { return {{nullptr, nullptr, l.w, l.n_out, l.k_in}, l.A, l.B, l.r, l.scale}; }
+
 cudaEvent_t pool_event() {
   if (g_pool_used == g_pool.size()) {
     cudaEvent_t e;
@@ -277,7 +295,7 @@ ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0.f}, ReduceOut c
 
 // NF4 weight maps for the GEMM B operand (K-major for forward, MN-major for dX);
 // boxes follow the number of B columns each CTA dequantises (bnc).
-bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const qlora_nf4& w, bool bwd, int bnc) {
+bool map_nf4(CUtensorMap* codes, CUtensorMap* absmax, const Wt& w, bool bwd, int bnc) {
   const int64_t N = w.n_out, K = w.k_in;
   if (!bwd) {
     const int rows = bnc < 128 ? bnc : 128;
@@ -300,13 +318,13 @@ int lora_rows_box(int bnc) { return bnc < 128 ? bnc : 128; }
 // the layout the in-mainloop dequantisers would have written.
 bool is_staged(int tiles) { return tiles == 4; }
 size_t stage_bytes(int64_t n_out, int64_t k_in) { return align256(static_cast<size_t>(n_out) * k_in * 2); }
-bool map_staged(CUtensorMap* m, const bf16* wq, const qlora_nf4& w, bool bwd, int bnc) {
+bool map_staged(CUtensorMap* m, const void* wq, const Wt& w, bool bwd, int bnc) {
   const int64_t N = w.n_out, K = w.k_in;
   if (!bwd) return map_bf16(m, wq, K, N, K, 64, bnc < 128 ? bnc : 128, CU_TENSOR_MAP_SWIZZLE_128B);
   return map_bf16(m, wq, K, N, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // Dequantises one weight (w1 == nullptr) or two in one launch into their staging buffers.
-qlora_status stage_weights(const qlora_nf4& w0, bf16* dst0, const qlora_nf4* w1, bf16* dst1, cudaStream_t st) {
+qlora_status stage_weights(const Wt& w0, bf16* dst0, const Wt* w1, bf16* dst1, cudaStream_t st) {
   KScope k(K_DEQUANT, st);
   return cuda_status(launch_nf4_dequantize(w0.codes, w0.absmax, w0.n_out * w0.k_in, dst0, w1 ? w1->codes : nullptr,
                                            w1 ? w1->absmax : nullptr, w1 ? w1->n_out * w1->k_in : 0, dst1, st,
@@ -323,10 +341,16 @@ bool map_outs(GemmMaps& maps, int tiles, int64_t rows, int64_t cols, int64_t ld,
   return true;
 }
 // B-operand maps of one weight (w1 == nullptr) or two (GEMM segments / gate-up halves 0 and 1) for
-// either feed; under the staged feed the weights are first dequantised into stage0 / stage1.
-qlora_status map_weights(GemmMaps& maps, const qlora_nf4& w0, const qlora_nf4* w1, bool bwd, int tiles,
-                         bf16* stage0, bf16* stage1, cudaStream_t st) {
+// either feed; under the staged feed NF4 weights are first dequantised into stage0 / stage1, and
+// bf16 weights are read where they are (they always use the staged feed).
+qlora_status map_weights(GemmMaps& maps, const Wt& w0, const Wt* w1, bool bwd, int tiles, bf16* stage0,
+                         bf16* stage1, cudaStream_t st) {
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
+  if (w0.w16) {
+    if (!is_staged(tiles) || !map_staged(&maps.b[0], w0.w16, w0, bwd, bnc)) return QLORA_ERR_CUDA;
+    if (w1 && !map_staged(&maps.b[1], w1->w16, *w1, bwd, bnc)) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
   if (is_staged(tiles)) {
     const qlora_status s = stage_weights(w0, stage0, w1, stage1, st);
     if (s != QLORA_OK) return s;
@@ -339,19 +363,21 @@ qlora_status map_weights(GemmMaps& maps, const qlora_nf4& w0, const qlora_nf4* w
   return QLORA_OK;
 }
 
-qlora_status check_linear(const qlora_lora_linear* lin) {
-  if (!lin || !lin->w.codes || !lin->w.absmax || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
+qlora_status check_linear(const Lin* lin) {
+  if (!lin || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
+  if (lin->w.w16 ? false : (!lin->w.codes || !lin->w.absmax)) return QLORA_ERR_INVALID_ARG;
   if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
   if (lin->r != 16) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in % 256 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in > (1 << 30) || lin->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->A) || misaligned(lin->B))
+  if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->w.w16) || misaligned(lin->A) ||
+      misaligned(lin->B))
     return QLORA_ERR_MISALIGNED;
   return QLORA_OK;
 }
 
 // Y-side GEMM launch helpers -------------------------------------------------
-qlora_status gemm_fwd(const qlora_lora_linear& lin, const bf16* X, int64_t M, const bf16* XAs, bf16* Y, int* status,
+qlora_status gemm_fwd(const Lin& lin, const bf16* X, int64_t M, const bf16* XAs, bf16* Y, int* status,
                       int tiles, bf16* stage, cudaStream_t st) {
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -439,38 +465,42 @@ qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n
                                            0, nullptr, st, num_sms()));
 }
 
-size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
-  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
+namespace {
+// Linear workspace: [status word | 256 B][M x 16 vector][partials][staged weight, if `stage`]
+size_t linear_ws(int64_t M, int64_t K, int64_t N, bool stage) {
   const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
   size_t part = rowproj_part_bytes(M, K, 16);
   part = std::max(part, dypass_part_bytes(M, N));
   part = std::max(part, colproj_part_bytes(M, K, 16));
-  return 256 + vec + align256(part) + (is_staged(g_tiles) ? stage_bytes(N, K) : 0);
+  return 256 + vec + align256(part) + (stage ? stage_bytes(N, K) : 0);
+}
+}  // namespace
+
+size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
+  return linear_ws(M, K, N, is_staged(g_tiles));
 }
 
 namespace {
-// Linear workspace: [status word | 256 B][M x 16 vector][partials][staged weight]
 struct LinearWs {
   int* status;
   bf16* vec;
   float* part;
   bf16* stage;
 };
-LinearWs carve_linear(void* ws, int64_t M, int64_t K, int64_t N) {
+LinearWs carve_linear(void* ws, int64_t M, int64_t K, int64_t N, bool stage) {
   char* w = static_cast<char*>(ws);
   LinearWs l;
   l.status = reinterpret_cast<int*>(w);
   l.vec = reinterpret_cast<bf16*>(w + 256);
   l.part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
-  l.stage = is_staged(g_tiles) ? reinterpret_cast<bf16*>(w + qlora_linear_workspace_bytes(M, K, N, 16) -
-                                                         stage_bytes(N, K))
-                               : nullptr;
+  l.stage = stage ? reinterpret_cast<bf16*>(w + linear_ws(M, K, N, true) - stage_bytes(N, K)) : nullptr;
   return l;
 }
 }  // namespace
 
-qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
-                              qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+static qlora_status linear_fwd(const Lin* lin, int tiles, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                               qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
   qlora_status s = check_linear(lin);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
@@ -479,9 +509,10 @@ qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X,
   if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
-  if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  const bool stage = is_staged(tiles) && !lin->w.w16;
+  if (ws_bytes < linear_ws(M, K, N, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  LinearWs l = carve_linear(ws, M, K, N);
+  LinearWs l = carve_linear(ws, M, K, N, stage);
   bf16* xa = reinterpret_cast<bf16*>(XA_saved);
   const bool scaled = lin->scale != 1.0f;
   bf16* XAs = scaled ? l.vec : xa;
@@ -489,13 +520,13 @@ qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X,
                    routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)),
                    l.status, st);
   if (s != QLORA_OK) return s;
-  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), l.status, g_tiles,
+  return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), l.status, tiles,
                   l.stage, st);
 }
 
-qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
-                              const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB,
-                              void* ws, size_t ws_bytes, qlora_stream_t stream) {
+static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                        const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws,
+                        size_t ws_bytes, qlora_stream_t stream) {
   qlora_status s = check_linear(lin);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
@@ -506,11 +537,11 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
     return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
-  if (ws_bytes < qlora_linear_workspace_bytes(M, K, N, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  const bool stage_w = is_staged(tiles) && !lin->w.w16;
+  if (ws_bytes < linear_ws(M, K, N, stage_w)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int tiles = g_tiles;
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  LinearWs l = carve_linear(ws, M, K, N);
+  LinearWs l = carve_linear(ws, M, K, N, stage_w);
   int* status = l.status;
   bf16* sG = l.vec;
   bf16* stage = l.stage;
@@ -556,8 +587,9 @@ qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X,
                       routs(rout(reinterpret_cast<bf16*>(dA), 0, 16, 0, 1.f)), status, st);
 }
 
-size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
-  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
+namespace {
+// MLP workspace: [status | 256 B][dE][dG][5 rank vectors][partials][two staged weights, if `stage`]
+size_t mlp_ws(int64_t M, int64_t d, int64_t h, bool stage) {
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
   const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
   size_t part = rowproj_part_bytes(M, d, 32);
@@ -566,7 +598,13 @@ size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
   part = std::max(part, dypass_part_bytes(M, h));
   part = std::max(part, colproj_part_bytes(M, h, 16));
   part = std::max(part, colproj_part_bytes(M, d, 32));
-  return 256 + 2 * big + 5 * vec + align256(part) + (is_staged(g_tiles) ? 2 * stage_bytes(h, d) : 0);
+  return 256 + 2 * big + 5 * vec + align256(part) + (stage ? 2 * stage_bytes(h, d) : 0);
+}
+}  // namespace
+
+size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
+  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
+  return mlp_ws(M, d, h, is_staged(g_tiles));
 }
 
 namespace {
@@ -576,7 +614,7 @@ struct MlpWs {
   float* part;
   bf16 *stage0, *stage1;  // staged feed: room for two dequantised [h, d] weights (gate, up; or down)
 };
-MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h) {
+MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h, bool stage) {
   char* w = static_cast<char*>(ws);
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
   const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
@@ -590,28 +628,29 @@ MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h) {
   m.v2 = reinterpret_cast<bf16*>(w + off); off += vec;
   m.gu = reinterpret_cast<bf16*>(w + off); off += 2 * vec;
   m.part = reinterpret_cast<float*>(w + off);
-  const size_t total = qlora_mlp_workspace_bytes(M, d, h, 16);
+  const size_t total = mlp_ws(M, d, h, true);
   m.stage0 = m.stage1 = nullptr;
-  if (is_staged(g_tiles)) {
+  if (stage) {
     m.stage0 = reinterpret_cast<bf16*>(w + total - 2 * stage_bytes(h, d));
     m.stage1 = reinterpret_cast<bf16*>(w + total - stage_bytes(h, d));
   }
   return m;
 }
-qlora_status check_mlp(const qlora_lora_linear* g, const qlora_lora_linear* u, const qlora_lora_linear* d) {
+qlora_status check_mlp(const Lin* g, const Lin* u, const Lin* d) {
   qlora_status s;
   if ((s = check_linear(g)) != QLORA_OK || (s = check_linear(u)) != QLORA_OK || (s = check_linear(d)) != QLORA_OK)
     return s;
   if (g->w.n_out != u->w.n_out || g->w.k_in != u->w.k_in || d->w.k_in != g->w.n_out || d->w.n_out != g->w.k_in)
     return QLORA_ERR_INVALID_ARG;
   if (g->w.n_out % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!g->w.w16 != !u->w.w16 || !g->w.w16 != !d->w.w16) return QLORA_ERR_INVALID_ARG;  // one base format
   return QLORA_OK;
 }
 }  // namespace
 
-qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                           const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
-                           const qlora_mlp_saved* sv, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const Lin* down, int tiles, const qlora_bf16* X,
+                     int64_t M, qlora_bf16* Y, const qlora_mlp_saved* sv, void* ws, size_t ws_bytes,
+                     qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
   qlora_status s = check_mlp(gate, up, down);
   if (s != QLORA_OK) return s;
@@ -624,10 +663,10 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
     return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
-  if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  const bool stage = is_staged(tiles) && !gate->w.w16;
+  if (ws_bytes < mlp_ws(M, d, h, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int tiles = g_tiles;
-  MlpWs w = carve_mlp(ws, M, d, h);
+  MlpWs w = carve_mlp(ws, M, d, h, stage);
   const bf16* x = reinterpret_cast<const bf16*>(X);
   bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
   bf16* xau = reinterpret_cast<bf16*>(sv->XA_u);
@@ -681,11 +720,10 @@ qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const q
                   w.stage0, st);
 }
 
-qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                           const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
-                           const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
-                           qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
-                           size_t ws_bytes, qlora_stream_t stream) {
+static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const Lin* down, int tiles, const qlora_bf16* X,
+                     const qlora_mlp_saved* sv, const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g,
+                     qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
+                     void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
   qlora_status s = check_mlp(gate, up, down);
   if (s != QLORA_OK) return s;
@@ -700,11 +738,11 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
     if (misaligned(p)) return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
-  if (ws_bytes < qlora_mlp_workspace_bytes(M, d, h, 16)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  const bool stage = is_staged(tiles) && !gate->w.w16;
+  if (ws_bytes < mlp_ws(M, d, h, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int tiles = g_tiles;
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  MlpWs w = carve_mlp(ws, M, d, h);
+  MlpWs w = carve_mlp(ws, M, d, h, stage);
   bf16* sGd = w.v0;
   // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, d, reinterpret_cast<const bf16*>(sv->HA_d),
@@ -794,6 +832,80 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
                       w.status, st);
 }
 
+// NF4 entry points: the current tile configuration.
+qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                              qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!lin) return QLORA_ERR_INVALID_ARG;
+  const Lin l = lin_of(*lin);
+  return linear_fwd(&l, g_tiles, X, M, Y, XA_saved, ws, ws_bytes, stream);
+}
+qlora_status qlora_linear_bwd(const qlora_lora_linear* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                              const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!lin) return QLORA_ERR_INVALID_ARG;
+  const Lin l = lin_of(*lin);
+  return linear_bwd(&l, g_tiles, X, XA_saved, dY, M, dX, dA, dB, ws, ws_bytes, stream);
+}
+qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                           const qlora_mlp_saved* sv, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!gate || !up || !down) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_fwd(act, &g, &u, &d, g_tiles, X, M, Y, sv, ws, ws_bytes, stream);
+}
+qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                           const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
+                           const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                           qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
+                           size_t ws_bytes, qlora_stream_t stream) {
+  if (!gate || !up || !down) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_bwd(act, &g, &u, &d, g_tiles, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes,
+                 stream);
+}
+
+// 16-bit entry points: bf16 base weights, always the staged-feed pair tile
+// (the weight is already what the GEMM streams; nothing is dequantised).
+size_t qlora_linear16_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
+  return linear_ws(M, K, N, false);
+}
+size_t qlora_mlp16_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
+  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
+  return mlp_ws(M, d, h, false);
+}
+qlora_status qlora_linear16_fwd(const qlora_lora_linear16* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                                qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!lin) return QLORA_ERR_INVALID_ARG;
+  const Lin l = lin_of(*lin);
+  if (!l.w.w16) return QLORA_ERR_INVALID_ARG;
+  return linear_fwd(&l, 4, X, M, Y, XA_saved, ws, ws_bytes, stream);
+}
+qlora_status qlora_linear16_bwd(const qlora_lora_linear16* lin, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                                const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB,
+                                void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!lin) return QLORA_ERR_INVALID_ARG;
+  const Lin l = lin_of(*lin);
+  if (!l.w.w16) return QLORA_ERR_INVALID_ARG;
+  return linear_bwd(&l, 4, X, XA_saved, dY, M, dX, dA, dB, ws, ws_bytes, stream);
+}
+qlora_status qlora_mlp16_fwd(qlora_act act, const qlora_lora_linear16* gate, const qlora_lora_linear16* up,
+                             const qlora_lora_linear16* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                             const qlora_mlp_saved* sv, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!gate || !up || !down || !gate->w || !up->w || !down->w) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_fwd(act, &g, &u, &d, 4, X, M, Y, sv, ws, ws_bytes, stream);
+}
+qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16* gate, const qlora_lora_linear16* up,
+                             const qlora_lora_linear16* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
+                             const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                             qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
+                             size_t ws_bytes, qlora_stream_t stream) {
+  if (!gate || !up || !down || !gate->w || !up->w || !down->w) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_bwd(act, &g, &u, &d, 4, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes, stream);
+}
+
 qlora_status qlora_last_device_status(void* ws, qlora_stream_t stream) {
   if (!ws) return QLORA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -872,8 +984,11 @@ static qlora_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
-                                      qlora_bf16* XA_saved, qlora_stream_t stream) {
+qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const qlora_bf16* X, int64_t M,
+                                      qlora_bf16* Y, qlora_bf16* XA_saved, qlora_stream_t stream) {
+  if (!lin_nf4) return QLORA_ERR_INVALID_ARG;
+  const Lin lv = lin_of(*lin_nf4);
+  const Lin* lin = &lv;
   qlora_status s = check_linear(lin);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;

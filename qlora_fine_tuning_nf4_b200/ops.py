@@ -33,6 +33,11 @@ class QloraLoraLinear(ctypes.Structure):
                 ("r", ctypes.c_int32), ("scale", ctypes.c_float)]
 
 
+class QloraLoraLinear16(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("r", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
 class QloraMlpSaved(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("E", "G", "H", "XA_g", "XA_u", "HA_d")]
 
@@ -82,6 +87,25 @@ _SIGS = {
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_linear16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                         ctypes.c_int32]),
+    "qlora_mlp16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                      ctypes.c_int32]),
+    "qlora_linear16_fwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear16), ctypes.c_void_p, ctypes.c_int64,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                          ctypes.c_void_p]),
+    "qlora_linear16_bwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear16), ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_mlp16_fwd": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear16),
+                                       ctypes.POINTER(QloraLoraLinear16), ctypes.POINTER(QloraLoraLinear16),
+                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                       ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p, ctypes.c_size_t,
+                                       ctypes.c_void_p]),
+    "qlora_mlp16_bwd": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear16),
+                                       ctypes.POINTER(QloraLoraLinear16), ctypes.POINTER(QloraLoraLinear16),
+                                       ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
+                                       ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
 }
 
 
@@ -169,6 +193,32 @@ class LoraLinear:
         return QloraLoraLinear(self.w.c(), self.A.data_ptr(), self.B.data_ptr(), self.A.shape[1], self.scale)
 
 
+@dataclass
+class LoraLinear16:
+    """A projection with a frozen bf16 base weight (LoRA rather than QLoRA)."""
+    w: torch.Tensor  # bf16 [n_out, k_in]
+    A: torch.Tensor  # bf16 [k_in, r]
+    B: torch.Tensor  # bf16 [r, n_out]
+    scale: float
+
+    @property
+    def n_out(self):
+        return self.w.shape[0]
+
+    @property
+    def k_in(self):
+        return self.w.shape[1]
+
+    def c(self):
+        return QloraLoraLinear16(self.w.data_ptr(), self.n_out, self.k_in, self.A.data_ptr(), self.B.data_ptr(),
+                                 self.A.shape[1], self.scale)
+
+
+def _dims(lin):
+    """(n_out, k_in) of an NF4 or a bf16 projection."""
+    return (lin.w.n_out, lin.w.k_in) if isinstance(lin, LoraLinear) else (lin.n_out, lin.k_in)
+
+
 class Workspace:
     """Caller-owned device workspace (zeroed once; grows on demand)."""
 
@@ -190,18 +240,33 @@ def qlora_mlp_workspace_bytes(M, d, h, r=16):
     return int(lib().qlora_mlp_workspace_bytes(M, d, h, r))
 
 
-def qlora_linear_fwd(lin: LoraLinear, X, ws: Workspace, Y=None, XA=None):
+def qlora_linear16_workspace_bytes(M, K, N, r=16):
+    return int(lib().qlora_linear16_workspace_bytes(M, K, N, r))
+
+
+def qlora_mlp16_workspace_bytes(M, d, h, r=16):
+    return int(lib().qlora_mlp16_workspace_bytes(M, d, h, r))
+
+
+def _linear_fwd(fn, wsq, lin, X, ws, Y, XA):
     M = X.shape[0]
+    n_out, k_in = _dims(lin)
     if Y is None:
-        Y = torch.empty(M, lin.w.n_out, dtype=torch.bfloat16, device=X.device)
+        Y = torch.empty(M, n_out, dtype=torch.bfloat16, device=X.device)
     if XA is None:
         XA = torch.empty(M, lin.A.shape[1], dtype=torch.bfloat16, device=X.device)
-    nb = qlora_linear_workspace_bytes(M, lin.w.k_in, lin.w.n_out, lin.A.shape[1])
-    buf = ws.get(nb)
+    buf = ws.get(wsq(M, k_in, n_out, lin.A.shape[1]))
     c = lin.c()
-    _check("qlora_linear_fwd", lib().qlora_linear_fwd(ctypes.byref(c), _p(X), M, _p(Y), _p(XA), _p(buf),
-                                                      buf.numel(), _stream()))
+    _check(fn, getattr(lib(), fn)(ctypes.byref(c), _p(X), M, _p(Y), _p(XA), _p(buf), buf.numel(), _stream()))
     return Y, XA
+
+
+def qlora_linear_fwd(lin: LoraLinear, X, ws: Workspace, Y=None, XA=None):
+    return _linear_fwd("qlora_linear_fwd", qlora_linear_workspace_bytes, lin, X, ws, Y, XA)
+
+
+def qlora_linear16_fwd(lin: LoraLinear16, X, ws: Workspace, Y=None, XA=None):
+    return _linear_fwd("qlora_linear16_fwd", qlora_linear16_workspace_bytes, lin, X, ws, Y, XA)
 
 
 def qlora_linear_fwd_noalloc(lin: LoraLinear, X, Y=None, XA=None):
@@ -219,21 +284,28 @@ def qlora_linear_fwd_noalloc(lin: LoraLinear, X, Y=None, XA=None):
     return Y, XA
 
 
-def qlora_linear_bwd(lin: LoraLinear, X, XA, dY, ws: Workspace, dX=None, dA=None, dB=None):
+def _linear_bwd(fn, wsq, lin, X, XA, dY, ws, dX, dA, dB):
     M = X.shape[0]
-    dev = X.device
+    n_out, k_in = _dims(lin)
     if dX is None:
-        dX = torch.empty(M, lin.w.k_in, dtype=torch.bfloat16, device=dev)
+        dX = torch.empty(M, k_in, dtype=torch.bfloat16, device=X.device)
     if dA is None:
         dA = torch.empty_like(lin.A)
     if dB is None:
         dB = torch.empty_like(lin.B)
-    nb = qlora_linear_workspace_bytes(M, lin.w.k_in, lin.w.n_out, lin.A.shape[1])
-    buf = ws.get(nb)
+    buf = ws.get(wsq(M, k_in, n_out, lin.A.shape[1]))
     c = lin.c()
-    _check("qlora_linear_bwd", lib().qlora_linear_bwd(ctypes.byref(c), _p(X), _p(XA), _p(dY), M, _p(dX), _p(dA),
-                                                      _p(dB), _p(buf), buf.numel(), _stream()))
+    _check(fn, getattr(lib(), fn)(ctypes.byref(c), _p(X), _p(XA), _p(dY), M, _p(dX), _p(dA), _p(dB), _p(buf),
+                                  buf.numel(), _stream()))
     return dX, dA, dB
+
+
+def qlora_linear_bwd(lin: LoraLinear, X, XA, dY, ws: Workspace, dX=None, dA=None, dB=None):
+    return _linear_bwd("qlora_linear_bwd", qlora_linear_workspace_bytes, lin, X, XA, dY, ws, dX, dA, dB)
+
+
+def qlora_linear16_bwd(lin: LoraLinear16, X, XA, dY, ws: Workspace, dX=None, dA=None, dB=None):
+    return _linear_bwd("qlora_linear16_bwd", qlora_linear16_workspace_bytes, lin, X, XA, dY, ws, dX, dA, dB)
 
 
 def make_mlp_saved(M, h, r, device):
@@ -245,36 +317,53 @@ def _saved_c(sv):
     return QloraMlpSaved(*[sv[k].data_ptr() for k in ("E", "G", "H", "XA_g", "XA_u", "HA_d")])
 
 
-def qlora_mlp_fwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, ws: Workspace, Y=None, saved=None):
+def _mlp_fwd(fn, wsq, act, gate, up, down, X, ws, Y, saved):
     M, d = X.shape
-    h = gate.w.n_out
+    h = _dims(gate)[0]
     r = gate.A.shape[1]
     if Y is None:
         Y = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
     if saved is None:
         saved = make_mlp_saved(M, h, r, X.device)
-    buf = ws.get(qlora_mlp_workspace_bytes(M, d, h, r))
+    buf = ws.get(wsq(M, d, h, r))
     g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
-    _check("qlora_mlp_fwd", lib().qlora_mlp_fwd(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn),
-                                                _p(X), M, _p(Y), ctypes.byref(sv), _p(buf), buf.numel(), _stream()))
+    _check(fn, getattr(lib(), fn)(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X), M,
+                                  _p(Y), ctypes.byref(sv), _p(buf), buf.numel(), _stream()))
     return Y, saved
 
 
-def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, dY, ws: Workspace, grads=None):
+def qlora_mlp_fwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, ws: Workspace, Y=None, saved=None):
+    return _mlp_fwd("qlora_mlp_fwd", qlora_mlp_workspace_bytes, act, gate, up, down, X, ws, Y, saved)
+
+
+def qlora_mlp16_fwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, ws: Workspace, Y=None,
+                    saved=None):
+    return _mlp_fwd("qlora_mlp16_fwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, ws, Y, saved)
+
+
+def _mlp_bwd(fn, wsq, act, gate, up, down, X, saved, dY, ws, grads):
     M, d = X.shape
-    h = gate.w.n_out
+    h = _dims(gate)[0]
     if grads is None:
         grads = {"dX": torch.empty(M, d, dtype=torch.bfloat16, device=X.device),
                  "dA_g": torch.empty_like(gate.A), "dB_g": torch.empty_like(gate.B),
                  "dA_u": torch.empty_like(up.A), "dB_u": torch.empty_like(up.B),
                  "dA_d": torch.empty_like(down.A), "dB_d": torch.empty_like(down.B)}
-    buf = ws.get(qlora_mlp_workspace_bytes(M, d, h, gate.A.shape[1]))
+    buf = ws.get(wsq(M, d, h, gate.A.shape[1]))
     g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
     outs = [_p(grads[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
-    _check("qlora_mlp_bwd", lib().qlora_mlp_bwd(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn),
-                                                _p(X), ctypes.byref(sv), _p(dY), M, *outs, _p(buf), buf.numel(),
-                                                _stream()))
+    _check(fn, getattr(lib(), fn)(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X),
+                                  ctypes.byref(sv), _p(dY), M, *outs, _p(buf), buf.numel(), _stream()))
     return grads
+
+
+def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, dY, ws: Workspace, grads=None):
+    return _mlp_bwd("qlora_mlp_bwd", qlora_mlp_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
+
+
+def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, saved, dY, ws: Workspace,
+                    grads=None):
+    return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
 
 
 # ------------------------------------------------------------ utilities ----

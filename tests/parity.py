@@ -106,8 +106,24 @@ def run_linear_gpu(p, tiles=4, ws=None):
             "codes": codes, "absmax": absmax, "status": st}
 
 
-def run_linear_oracle(p):
-    codes, absmax, W = oracle_weight(p["W"])
+def run_linear16_gpu(p, ws=None):
+    """The 16-bit entry points: the bf16 weight itself is the frozen base."""
+    lin = ops.LoraLinear16(dev(p["W"]), dev(p["A"]), dev(p["B"]), p["s"])
+    ws = ws or ops.Workspace()
+    X, dY = dev(p["X"]), dev(p["dY"])
+    Y, XA = ops.qlora_linear16_fwd(lin, X, ws)
+    dX, dA, dB = ops.qlora_linear16_bwd(lin, X, XA, dY, ws)
+    torch.cuda.synchronize()
+    st = ops.qlora_last_device_status(ws)
+    return {"Y": gpu_f64(Y), "XA": gpu_f64(XA), "dX": gpu_f64(dX), "dA": gpu_f64(dA), "dB": gpu_f64(dB), "status": st}
+
+
+def run_linear_oracle(p, base="nf4"):
+    """base = "nf4": the oracle's own NF4 quantisation of W; "bf16": W itself."""
+    if base == "nf4":
+        codes, absmax, W = oracle_weight(p["W"])
+    else:
+        codes, absmax, W = None, None, f64(p["W"])
     X, A, B, dY = f64(p["X"]), f64(p["A"]), f64(p["B"]), f64(p["dY"])
     Y, XA = oracle.linear_fwd(X, W, A, B, p["s"])
     dX, dA, dB = oracle.linear_bwd(X, W, A, B, p["s"], dY)
@@ -135,10 +151,30 @@ def run_mlp_gpu(p, act, tiles=4, ws=None):
     return out
 
 
-def run_mlp_oracle(p, act):
+def run_mlp16_gpu(p, act, ws=None, rows=None):
+    """The 16-bit MLP entry points; `rows` selects returned rows of Y, dX and the saved tensors."""
+    lins = {k: ops.LoraLinear16(dev(p["W_" + k]), dev(p["A_" + k]), dev(p["B_" + k]), p["s"]) for k in ("g", "u", "d")}
+    ws = ws or ops.Workspace()
+    X, dY = dev(p["X"]), dev(p["dY"])
+    Y, saved = ops.qlora_mlp16_fwd(act, lins["g"], lins["u"], lins["d"], X, ws)
+    grads = ops.qlora_mlp16_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws)
+    torch.cuda.synchronize()
+    sel = (lambda t: t) if rows is None else (lambda t: t[torch.as_tensor(rows, device=t.device)])
+    out = {"Y": gpu_f64(sel(Y)), "status": ops.qlora_last_device_status(ws)}
+    for k in ("E", "G", "H", "XA_g", "XA_u", "HA_d"):
+        out[k] = gpu_f64(sel(saved[k]))
+    for k, v in grads.items():
+        out[k] = gpu_f64(sel(v) if k == "dX" else v)
+    return out
+
+
+def run_mlp_oracle(p, act, base="nf4"):
     lin, qs = {}, {}
     for k in ("g", "u", "d"):
-        c, a, W = oracle_weight(p["W_" + k])
+        if base == "nf4":
+            c, a, W = oracle_weight(p["W_" + k])
+        else:
+            c, a, W = None, None, f64(p["W_" + k])
         lin[k] = (W, f64(p["A_" + k]), f64(p["B_" + k]), p["s"])
         qs[k] = (c, a)
     X, dY = f64(p["X"]), f64(p["dY"])
