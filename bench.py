@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
+    ap.add_argument("--rank", type=int, default=0, choices=[0, 16, 32, 64],
+                    help="LoRA rank (0 = the workload's, 16); s = alpha / r with alpha = the rank")
     ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
                     help="frozen base format: NF4 (QLoRA, the metric) or bf16 (plain LoRA, for comparison)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -418,6 +420,8 @@ def main():
     wl = dict(MLP_WORKLOADS[args.workload])
     if args.tokens:
         wl["M"] = args.tokens
+    if args.rank:
+        wl["r"], wl["alpha"] = args.rank, float(args.rank)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

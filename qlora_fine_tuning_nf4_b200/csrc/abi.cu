@@ -24,8 +24,8 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, i
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
 int gemm_nf4_b_cols_per_cta(int tiles);
-cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
-                           const ReduceJob& job, int nkc, int* status, cudaStream_t st);
+cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
+                           const CUtensorMap& v1, const ReduceJob& job, int nkc, int* status, cudaStream_t st);
 cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
                            int* status, cudaStream_t st);
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
@@ -162,8 +162,14 @@ bool map_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t
 }
 
 // ---------------------------------------------------------- planning ----
-// Skinny passes run kTargetCtas persistent CTAs (four per SM on B200).
-constexpr int kTargetCtas = 4 * 148;
+// Skinny passes run up to four persistent CTAs per SM; a CTA's ring holds four
+// stages of one 64x64 tile of T plus 128 bytes per factor column (the grid
+// shrinks when wide factor tiles limit residency).
+constexpr int kSMs = 148;
+int skinny_target_ctas(int factor_cols) {
+  const int smem = 4 * (8192 + 128 * factor_cols) + 64 + 1024;
+  return kSMs * std::max(1, std::min(4, 232448 / smem));
+}
 
 // Partition of `groups` output groups of `upg` units each over the CTAs:
 // unit granularity while there are fewer groups than CTAs (every CTA streams
@@ -172,14 +178,14 @@ struct SkPlan {
   SkPart sp;
   int slot_cap;
 };
-SkPlan plan_skinny(int64_t groups, int64_t upg) {
+SkPlan plan_skinny(int64_t groups, int64_t upg, int target) {
   SkPlan p;
   const int64_t units = groups * upg;
-  int64_t align = groups >= kTargetCtas ? upg : 1;
+  int64_t align = groups >= target ? upg : 1;
   while (cdiv(units, align) > (int64_t(1) << 30)) align *= 2;  // keep the unit count in int range
   const int64_t U = cdiv(units, align);
   p.sp.U = static_cast<int>(U);
-  p.sp.P = static_cast<int>(std::min<int64_t>(kTargetCtas, U));
+  p.sp.P = static_cast<int>(std::min<int64_t>(target, U));
   p.sp.align = static_cast<int>(align);
   p.sp.upg = static_cast<int>(upg);
   p.slot_cap = 1;
@@ -187,19 +193,28 @@ SkPlan plan_skinny(int64_t groups, int64_t upg) {
   return p;
 }
 constexpr int kDyCC = 4;  // column chunks of 64 per dypass unit (matches the kernel)
-SkPlan plan_rowproj(int64_t M, int64_t K) { return plan_skinny(cdiv(M, 64), K / 64); }
-SkPlan plan_colproj(int64_t M, int64_t ncols) { return plan_skinny(cdiv(ncols, 64), cdiv(M, 64)); }
-SkPlan plan_dypass(int64_t M, int64_t N) { return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64)); }
+// rowproj: T [M, K] times factors of `fcols` columns in all; reduction over K (padded to 64)
+SkPlan plan_rowproj(int64_t M, int64_t K, int fcols) {
+  return plan_skinny(cdiv(M, 64), cdiv(K, 64), skinny_target_ctas(fcols));
+}
+SkPlan plan_colproj(int64_t M, int64_t ncols, int R) {
+  return plan_skinny(cdiv(ncols, 64), cdiv(M, 64), skinny_target_ctas(R));
+}
+SkPlan plan_dypass(int64_t M, int64_t N) {
+  return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64), skinny_target_ctas(32));
+}
 size_t rowproj_part_bytes(int64_t M, int64_t K, int R) {
-  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K).slot_cap * 64 * R * 4;
+  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K, R).slot_cap * 64 * R * 4;
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
-  return static_cast<size_t>(cdiv(ncols, 64)) * plan_colproj(M, ncols).slot_cap * 64 * R * 4;
+  return static_cast<size_t>(cdiv(ncols, 64)) * plan_colproj(M, ncols, R).slot_cap * 64 * R * 4;
 }
 size_t dypass_gpart_bytes(int64_t M, int64_t N) {
   return align256(static_cast<size_t>(cdiv(M, 64)) * cdiv(cdiv(N, 64), kDyCC) * 64 * 16 * 4);
 }
-size_t dypass_part_bytes(int64_t M, int64_t N) {
+// partials of the dY pass: fused for rank 16, a G pass then a dB pass for larger ranks
+size_t dypass_part_bytes(int64_t M, int64_t N, int r) {
+  if (r != 16) return std::max(rowproj_part_bytes(M, N, r), colproj_part_bytes(M, N, r));
   const int64_t ncb = cdiv(cdiv(N, 64), kDyCC);
   return dypass_gpart_bytes(M, N) + static_cast<size_t>(ncb) * plan_dypass(M, N).slot_cap * kDyCC * 64 * 16 * 4;
 }
@@ -222,33 +237,60 @@ ReduceJob reduce_job(float* part, int64_t groups, int grows, int64_t rows, int R
 // ------------------------------------------------------------ passes ----
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
-// P = T V (V = one or two [K, 16] LoRA A factors) -> out[j] (bf16, optional scaled copy)
-qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, float* part,
+// A rank-side factor [rows, cols] (row stride ld) as the skinny kernels read it:
+// 64-row boxes of min(cols, 64) columns in the swizzle of that row width.
+bool map_factor(CUtensorMap* m, const void* p, int64_t rows, int cols, int64_t ld) {
+  const int subw = cols < 64 ? cols : 64;
+  const CUtensorMapSwizzle swz = subw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                            : (subw == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  return map_bf16(m, p, cols, rows, ld, subw, 64, swz);
+}
+
+// P = T V (V = one or two [K, r] LoRA A factors) -> outs (bf16, optional scaled copies)
+qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, int r, float* part,
                           ReduceOuts outs, int* status, cudaStream_t st) {
   CUtensorMap mt, mv0, mv1;
   const int nv = V1 ? 2 : 1;
   if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_bf16(&mv0, V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
-  if (!map_bf16(&mv1, V1 ? V1 : V0, 16, K, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
-  const SkPlan p = plan_rowproj(M, K);
+  if (!map_factor(&mv0, V0, K, r, r)) return QLORA_ERR_CUDA;
+  if (!map_factor(&mv1, V1 ? V1 : V0, K, r, r)) return QLORA_ERR_CUDA;
+  const SkPlan p = plan_rowproj(M, K, nv * r);
   const int64_t nrc = cdiv(M, 64);
-  const ReduceJob j = reduce_job(part, nrc, 64, M, 16 * nv, p.slot_cap, 0, p.sp, outs);
+  const ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_ROWPROJ, st);
-    const qlora_status s = cuda_status(launch_rowproj(nv, mt, mv0, mv1, j, (int)(K / 64), status, st));
+    const qlora_status s = cuda_status(launch_rowproj(r, nv, false, mt, mv0, mv1, j, (int)cdiv(K, 64), status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
   return cuda_status(launch_reduce(j, nullptr, st));
 }
 
-// Q = T^T U (U [M, R]) -> outs
+// G = T B^T (B = LoRA right factor [r, N]) -> outs
+qlora_status pass_rowproj_bt(const bf16* T, int64_t M, int64_t N, const bf16* B, int r, float* part,
+                             ReduceOuts outs, int* status, cudaStream_t st) {
+  CUtensorMap mt, mb;
+  if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mb, B, N, r, N, 64, r, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  const SkPlan p = plan_rowproj(M, N, r);
+  const int64_t nrc = cdiv(M, 64);
+  const ReduceJob j = reduce_job(part, nrc, 64, M, r, p.slot_cap, 0, p.sp, outs);
+  {
+    KScope k(K_ROWPROJ, st);
+    const qlora_status s = cuda_status(launch_rowproj(r, 1, true, mt, mb, mb, j, (int)cdiv(N, 64), status, st));
+    if (s != QLORA_OK) return s;
+  }
+  KScope k(K_REDUCE, st);
+  return cuda_status(launch_reduce(j, nullptr, st));
+}
+
+// Q = T^T U (U [M, R], contiguous) -> outs
 qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U, int R, float* part,
                           ReduceOuts outs, int* status, cudaStream_t st) {
   CUtensorMap mt, mu;
   if (!map_bf16(&mt, T, ncols, M, ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_bf16(&mu, U, R, M, R, R, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
-  const SkPlan p = plan_colproj(M, ncols);
+  if (!map_factor(&mu, U, M, R, R)) return QLORA_ERR_CUDA;
+  const SkPlan p = plan_colproj(M, ncols, R);
   const int64_t ncc = cdiv(ncols, 64);
   const ReduceJob j = reduce_job(part, ncc, 64, ncols, R, p.slot_cap, 0, p.sp, outs);
   {
@@ -260,12 +302,18 @@ qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U
   return cuda_status(launch_reduce(j, nullptr, st));
 }
 
-// G = T Bl^T ([M,16]) and Q = T^T U ([N,16]) from one read of T [M, N].
-qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, const bf16* Bl, float* part,
+// G = T Bl^T ([M, r]) and Q = T^T U ([N, r]) for T [M, N]: one fused read of T
+// at rank 16, a G pass and a Q pass at larger ranks.
+qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, const bf16* Bl, int r, float* part,
                          ReduceOuts gouts, ReduceOuts qouts, int* status, cudaStream_t st) {
+  if (r != 16) {
+    const qlora_status s = pass_rowproj_bt(T, M, N, Bl, r, part, gouts, status, st);
+    if (s != QLORA_OK) return s;
+    return pass_colproj(T, M, N, U, r, part, qouts, status, st);
+  }
   CUtensorMap mt, mu, mb;
   if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_bf16(&mu, U, 16, M, 16, 16, 64, CU_TENSOR_MAP_SWIZZLE_NONE)) return QLORA_ERR_CUDA;
+  if (!map_factor(&mu, U, M, 16, 16)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mb, Bl, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_dypass(M, N);
   const int64_t nrc = cdiv(M, 64), nch = cdiv(N, 64), ncb = cdiv(nch, kDyCC);
@@ -282,9 +330,13 @@ qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, con
   return cuda_status(launch_reduce(jg, &jq, st));
 }
 
-ReduceOut rout(bf16* p, int col0, int ld, int transpose, float scale) { return {p, col0, ld, transpose, scale}; }
-ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0.f}, ReduceOut c = {nullptr, 0, 0, 0, 0.f},
-                 ReduceOut d = {nullptr, 0, 0, 0, 0.f}) {
+// One reduction output: columns [col0, col0 + width) of the partials, scaled, bf16
+// into p (row stride ld, or transposed).
+ReduceOut rout(bf16* p, int col0, int width, int ld, int transpose, float scale) {
+  return {p, col0, width, ld, transpose, scale};
+}
+ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0, 0.f}, ReduceOut c = {nullptr, 0, 0, 0, 0, 0.f},
+                 ReduceOut d = {nullptr, 0, 0, 0, 0, 0.f}) {
   ReduceOuts o;
   o.o[0] = a;
   o.o[1] = b;
@@ -363,11 +415,32 @@ qlora_status map_weights(GemmMaps& maps, const Wt& w0, const Wt* w1, bool bwd, i
   return QLORA_OK;
 }
 
-qlora_status check_linear(const Lin* lin) {
+// LoRA operand maps of the GEMM.  Left operand [rows, r] with row stride ld (s X A or
+// s G); right factor: forward B [r, n], backward A [n, r].  The staged feed streams
+// both as one 64-wide reduction block through the operand ring (zeros beyond the
+// rank); the in-mainloop feed (rank 16) keeps its dedicated tiles.
+bool map_lora_left(CUtensorMap* m, const void* p, int64_t rows, int r, int64_t ld, int tiles) {
+  if (is_staged(tiles)) return map_bf16(m, p, r, rows, ld, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  return map_bf16(m, p, 16, rows, ld, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B);
+}
+bool map_lora_right(CUtensorMap* m, const void* p, int64_t n, int r, bool bwd, int tiles) {
+  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
+  if (is_staged(tiles)) {
+    if (bwd) return map_bf16(m, p, r, n, r, 64, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_128B);
+    return map_bf16(m, p, n, r, n, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (bwd) return map_bf16(m, p, 16, n, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B);
+  return map_bf16(m, p, n, 16, n, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// LoRA ranks: 16, 32 or 64 with the staged feed (configuration 4 or a bf16 base),
+// 16 with the feeds that dequantise in the mainloop.
+bool rank_ok(int r, int tiles) { return is_staged(tiles) ? (r == 16 || r == 32 || r == 64) : r == 16; }
+
+qlora_status check_linear(const Lin* lin, int tiles) {
   if (!lin || !lin->A || !lin->B) return QLORA_ERR_INVALID_ARG;
   if (lin->w.w16 ? false : (!lin->w.codes || !lin->w.absmax)) return QLORA_ERR_INVALID_ARG;
   if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
-  if (lin->r != 16) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!rank_ok(lin->r, tiles)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in % 256 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in > (1 << 30) || lin->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->w.w16) || misaligned(lin->A) ||
@@ -385,8 +458,8 @@ qlora_status gemm_fwd(const Lin& lin, const bf16* X, int64_t M, const bf16* XAs,
   if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   const qlora_status s = map_weights(maps, lin.w, nullptr, false, tiles, stage, nullptr, st);
   if (s != QLORA_OK) return s;
-  if (!map_bf16(&maps.la[0], XAs, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-  if (!map_bf16(&maps.lb[0], lin.B, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_lora_left(&maps.la[0], XAs, M, lin.r, lin.r, tiles)) return QLORA_ERR_CUDA;
+  if (!map_lora_right(&maps.lb[0], lin.B, N, lin.r, false, tiles)) return QLORA_ERR_CUDA;
   maps.a[1] = maps.a[0];
   maps.codes[1] = maps.codes[0];
   maps.absmax[1] = maps.absmax[0];
@@ -401,6 +474,7 @@ qlora_status gemm_fwd(const Lin& lin, const bf16* X, int64_t M, const bf16* XAs,
   a.nkb0 = (int)(K / 64);
   a.nkb1 = 0;
   a.lora = 1;
+  a.lora_k16 = lin.r / 16;
   a.ldo = (int)N;
   a.D = Y;
   a.status = status;
@@ -466,19 +540,19 @@ qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n
 }
 
 namespace {
-// Linear workspace: [status word | 256 B][M x 16 vector][partials][staged weight, if `stage`]
-size_t linear_ws(int64_t M, int64_t K, int64_t N, bool stage) {
-  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
-  size_t part = rowproj_part_bytes(M, K, 16);
-  part = std::max(part, dypass_part_bytes(M, N));
-  part = std::max(part, colproj_part_bytes(M, K, 16));
+// Linear workspace: [status word | 256 B][M x r vector][partials][staged weight, if `stage`]
+size_t linear_ws(int64_t M, int64_t K, int64_t N, int r, bool stage) {
+  const size_t vec = align256(static_cast<size_t>(M) * r * 2);
+  size_t part = rowproj_part_bytes(M, K, r);
+  part = std::max(part, dypass_part_bytes(M, N, r));
+  part = std::max(part, colproj_part_bytes(M, K, r));
   return 256 + vec + align256(part) + (stage ? stage_bytes(N, K) : 0);
 }
 }  // namespace
 
 size_t qlora_linear_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
-  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
-  return linear_ws(M, K, N, is_staged(g_tiles));
+  if (M <= 0 || K <= 0 || N <= 0 || !rank_ok(r, g_tiles)) return 256;
+  return linear_ws(M, K, N, r, is_staged(g_tiles));
 }
 
 namespace {
@@ -488,20 +562,20 @@ struct LinearWs {
   float* part;
   bf16* stage;
 };
-LinearWs carve_linear(void* ws, int64_t M, int64_t K, int64_t N, bool stage) {
+LinearWs carve_linear(void* ws, int64_t M, int64_t K, int64_t N, int r, bool stage) {
   char* w = static_cast<char*>(ws);
   LinearWs l;
   l.status = reinterpret_cast<int*>(w);
   l.vec = reinterpret_cast<bf16*>(w + 256);
-  l.part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * 32));
-  l.stage = stage ? reinterpret_cast<bf16*>(w + linear_ws(M, K, N, true) - stage_bytes(N, K)) : nullptr;
+  l.part = reinterpret_cast<float*>(w + 256 + align256(static_cast<size_t>(M) * r * 2));
+  l.stage = stage ? reinterpret_cast<bf16*>(w + linear_ws(M, K, N, r, true) - stage_bytes(N, K)) : nullptr;
   return l;
 }
 }  // namespace
 
 static qlora_status linear_fwd(const Lin* lin, int tiles, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                                qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
-  qlora_status s = check_linear(lin);
+  qlora_status s = check_linear(lin, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;
@@ -509,15 +583,16 @@ static qlora_status linear_fwd(const Lin* lin, int tiles, const qlora_bf16* X, i
   if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
+  const int r = lin->r;
   const bool stage = is_staged(tiles) && !lin->w.w16;
-  if (ws_bytes < linear_ws(M, K, N, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < linear_ws(M, K, N, r, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  LinearWs l = carve_linear(ws, M, K, N, stage);
+  LinearWs l = carve_linear(ws, M, K, N, r, stage);
   bf16* xa = reinterpret_cast<bf16*>(XA_saved);
   const bool scaled = lin->scale != 1.0f;
   bf16* XAs = scaled ? l.vec : xa;
-  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, l.part,
-                   routs(rout(xa, 0, 16, 0, 1.f), rout(scaled ? XAs : nullptr, 0, 16, 0, lin->scale)),
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, r, l.part,
+                   routs(rout(xa, 0, r, r, 0, 1.f), rout(scaled ? XAs : nullptr, 0, r, r, 0, lin->scale)),
                    l.status, st);
   if (s != QLORA_OK) return s;
   return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), l.status, tiles,
@@ -527,7 +602,7 @@ static qlora_status linear_fwd(const Lin* lin, int tiles, const qlora_bf16* X, i
 static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, const qlora_bf16* XA_saved,
                         const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA, qlora_bf16* dB, void* ws,
                         size_t ws_bytes, qlora_stream_t stream) {
-  qlora_status s = check_linear(lin);
+  qlora_status s = check_linear(lin, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;  // NOTE: dA, dB are left untouched when there are no rows
@@ -537,11 +612,11 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
     return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
+  const int r = lin->r;
   const bool stage_w = is_staged(tiles) && !lin->w.w16;
-  if (ws_bytes < linear_ws(M, K, N, stage_w)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < linear_ws(M, K, N, r, stage_w)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  LinearWs l = carve_linear(ws, M, K, N, stage_w);
+  LinearWs l = carve_linear(ws, M, K, N, r, stage_w);
   int* status = l.status;
   bf16* sG = l.vec;
   bf16* stage = l.stage;
@@ -549,8 +624,8 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
   const float sc = lin->scale;
   // G = dY B^T (stored scaled: sG), dB = s (XA)^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, N, reinterpret_cast<const bf16*>(XA_saved),
-                  reinterpret_cast<const bf16*>(lin->B), part, routs(rout(sG, 0, 16, 0, sc)),
-                  routs(rout(reinterpret_cast<bf16*>(dB), 0, (int)N, 1, sc)), status, st);
+                  reinterpret_cast<const bf16*>(lin->B), r, part, routs(rout(sG, 0, r, r, 0, sc)),
+                  routs(rout(reinterpret_cast<bf16*>(dB), 0, r, (int)N, 1, sc)), status, st);
   if (s != QLORA_OK) return s;
   // dX = dY W + (s G) A^T
   {
@@ -558,9 +633,8 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, N, M, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if ((s = map_weights(maps, lin->w, nullptr, true, tiles, stage, nullptr, st)) != QLORA_OK) return s;
-    if (!map_bf16(&maps.la[0], sG, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], lin->A, 16, K, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
-      return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[0], sG, M, r, r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[0], lin->A, K, r, true, tiles)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
@@ -573,6 +647,7 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
     a.N = (int)K;
     a.nkb0 = (int)cdiv(N, 64);
     a.lora = 1;
+    a.lora_k16 = r / 16;
     a.ldo = (int)K;
     a.D = reinterpret_cast<bf16*>(dX);
     if (!map_outs(maps, tiles, M, K, K, dX)) return QLORA_ERR_CUDA;
@@ -583,41 +658,41 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
     if (s != QLORA_OK) return s;
   }
   // dA = X^T (s G)
-  return pass_colproj(reinterpret_cast<const bf16*>(X), M, K, sG, 16, part,
-                      routs(rout(reinterpret_cast<bf16*>(dA), 0, 16, 0, 1.f)), status, st);
+  return pass_colproj(reinterpret_cast<const bf16*>(X), M, K, sG, r, part,
+                      routs(rout(reinterpret_cast<bf16*>(dA), 0, r, r, 0, 1.f)), status, st);
 }
 
 namespace {
 // MLP workspace: [status | 256 B][dE][dG][5 rank vectors][partials][two staged weights, if `stage`]
-size_t mlp_ws(int64_t M, int64_t d, int64_t h, bool stage) {
+size_t mlp_ws(int64_t M, int64_t d, int64_t h, int r, bool stage) {
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
-  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
-  size_t part = rowproj_part_bytes(M, d, 32);
-  part = std::max(part, rowproj_part_bytes(M, h, 16));
-  part = std::max(part, dypass_part_bytes(M, d));
-  part = std::max(part, dypass_part_bytes(M, h));
-  part = std::max(part, colproj_part_bytes(M, h, 16));
-  part = std::max(part, colproj_part_bytes(M, d, 32));
+  const size_t vec = align256(static_cast<size_t>(M) * r * 2);
+  size_t part = rowproj_part_bytes(M, d, 2 * r);
+  part = std::max(part, rowproj_part_bytes(M, h, r));
+  part = std::max(part, dypass_part_bytes(M, d, r));
+  part = std::max(part, dypass_part_bytes(M, h, r));
+  part = std::max(part, colproj_part_bytes(M, h, r));
+  part = std::max(part, colproj_part_bytes(M, d, 2 * r));
   return 256 + 2 * big + 5 * vec + align256(part) + (stage ? 2 * stage_bytes(h, d) : 0);
 }
 }  // namespace
 
 size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
-  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
-  return mlp_ws(M, d, h, is_staged(g_tiles));
+  if (M <= 0 || d <= 0 || h <= 0 || !rank_ok(r, g_tiles)) return 256;
+  return mlp_ws(M, d, h, r, is_staged(g_tiles));
 }
 
 namespace {
 struct MlpWs {
   int* status;
-  bf16 *dE, *dG, *v0, *v1, *v2, *gu;  // v*: [M,16] vectors; gu: [M,32]
+  bf16 *dE, *dG, *v0, *v1, *v2, *gu;  // v*: [M, r] vectors; gu: [M, 2r]
   float* part;
   bf16 *stage0, *stage1;  // staged feed: room for two dequantised [h, d] weights (gate, up; or down)
 };
-MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h, bool stage) {
+MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h, int r, bool stage) {
   char* w = static_cast<char*>(ws);
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
-  const size_t vec = align256(static_cast<size_t>(M) * 16 * 2);
+  const size_t vec = align256(static_cast<size_t>(M) * r * 2);
   MlpWs m;
   m.status = reinterpret_cast<int*>(w);
   size_t off = 256;
@@ -628,7 +703,7 @@ MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h, bool stage) {
   m.v2 = reinterpret_cast<bf16*>(w + off); off += vec;
   m.gu = reinterpret_cast<bf16*>(w + off); off += 2 * vec;
   m.part = reinterpret_cast<float*>(w + off);
-  const size_t total = mlp_ws(M, d, h, true);
+  const size_t total = mlp_ws(M, d, h, r, true);
   m.stage0 = m.stage1 = nullptr;
   if (stage) {
     m.stage0 = reinterpret_cast<bf16*>(w + total - 2 * stage_bytes(h, d));
@@ -636,10 +711,12 @@ MlpWs carve_mlp(void* ws, int64_t M, int64_t d, int64_t h, bool stage) {
   }
   return m;
 }
-qlora_status check_mlp(const Lin* g, const Lin* u, const Lin* d) {
+qlora_status check_mlp(const Lin* g, const Lin* u, const Lin* d, int tiles) {
   qlora_status s;
-  if ((s = check_linear(g)) != QLORA_OK || (s = check_linear(u)) != QLORA_OK || (s = check_linear(d)) != QLORA_OK)
+  if ((s = check_linear(g, tiles)) != QLORA_OK || (s = check_linear(u, tiles)) != QLORA_OK ||
+      (s = check_linear(d, tiles)) != QLORA_OK)
     return s;
+  if (g->r != u->r || g->r != d->r) return QLORA_ERR_UNSUPPORTED_SHAPE;  // one rank for the three
   if (g->w.n_out != u->w.n_out || g->w.k_in != u->w.k_in || d->w.k_in != g->w.n_out || d->w.n_out != g->w.k_in)
     return QLORA_ERR_INVALID_ARG;
   if (g->w.n_out % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
@@ -652,7 +729,7 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
                      int64_t M, qlora_bf16* Y, const qlora_mlp_saved* sv, void* ws, size_t ws_bytes,
                      qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
-  qlora_status s = check_mlp(gate, up, down);
+  qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;
@@ -663,10 +740,11 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
     return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
+  const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
-  if (ws_bytes < mlp_ws(M, d, h, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < mlp_ws(M, d, h, r, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  MlpWs w = carve_mlp(ws, M, d, h, stage);
+  MlpWs w = carve_mlp(ws, M, d, h, r, stage);
   const bf16* x = reinterpret_cast<const bf16*>(X);
   bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
   bf16* xau = reinterpret_cast<bf16*>(sv->XA_u);
@@ -675,10 +753,10 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
   bf16* xaus = up->scale != 1.f ? w.v1 : xau;
   bf16* hads = down->scale != 1.f ? w.v2 : had;
   // XA_g, XA_u = X [A_g | A_u] (one pass over X)
-  s = pass_rowproj(x, M, d, reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A), w.part,
-                   routs(rout(xag, 0, 16, 0, 1.f), rout(xau, 16, 16, 0, 1.f),
-                         rout(xags != xag ? xags : nullptr, 0, 16, 0, gate->scale),
-                         rout(xaus != xau ? xaus : nullptr, 16, 16, 0, up->scale)),
+  s = pass_rowproj(x, M, d, reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A), r, w.part,
+                   routs(rout(xag, 0, r, r, 0, 1.f), rout(xau, r, r, r, 0, 1.f),
+                         rout(xags != xag ? xags : nullptr, 0, r, r, 0, gate->scale),
+                         rout(xaus != xau ? xaus : nullptr, r, r, r, 0, up->scale)),
                    w.status, st);
   if (s != QLORA_OK) return s;
   // gate/up GEMM with the gated activation in the epilogue -> E, G, H
@@ -688,16 +766,17 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     if ((s = map_weights(maps, gate->w, &up->w, false, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
-    if (!map_bf16(&maps.la[0], xags, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.la[1], xaus, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], gate->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[1], up->B, h, 16, h, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[0], xags, M, r, r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[1], xaus, M, r, r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[0], gate->B, h, r, false, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[1], up->B, h, r, false, tiles)) return QLORA_ERR_CUDA;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     a.M = (int)M;
     a.N = (int)h;
     a.nkb0 = (int)(d / 64);
     a.lora = 2;
+    a.lora_k16 = r / 16;
     a.act = act == QLORA_ACT_SWIGLU ? ACT_SILU : ACT_GELU_TANH;
     a.ldo = (int)h;
     a.E = reinterpret_cast<bf16*>(sv->E);
@@ -711,8 +790,8 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (s != QLORA_OK) return s;
   }
   // HA_d = H A_d
-  s = pass_rowproj(reinterpret_cast<const bf16*>(sv->H), M, h, reinterpret_cast<const bf16*>(down->A), nullptr,
-                   w.part, routs(rout(had, 0, 16, 0, 1.f), rout(hads != had ? hads : nullptr, 0, 16, 0, down->scale)),
+  s = pass_rowproj(reinterpret_cast<const bf16*>(sv->H), M, h, reinterpret_cast<const bf16*>(down->A), nullptr, r,
+                   w.part, routs(rout(had, 0, r, r, 0, 1.f), rout(hads != had ? hads : nullptr, 0, r, r, 0, down->scale)),
                    w.status, st);
   if (s != QLORA_OK) return s;
   // Y = H W_d^T + (s H A_d) B_d
@@ -725,7 +804,7 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
                      qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
                      void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
-  qlora_status s = check_mlp(gate, up, down);
+  qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;
@@ -738,16 +817,16 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (misaligned(p)) return QLORA_ERR_MISALIGNED;
   if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
+  const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
-  if (ws_bytes < mlp_ws(M, d, h, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < mlp_ws(M, d, h, r, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int bnc = gemm_nf4_b_cols_per_cta(tiles);
-  MlpWs w = carve_mlp(ws, M, d, h, stage);
+  MlpWs w = carve_mlp(ws, M, d, h, r, stage);
   bf16* sGd = w.v0;
   // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, d, reinterpret_cast<const bf16*>(sv->HA_d),
-                  reinterpret_cast<const bf16*>(down->B), w.part, routs(rout(sGd, 0, 16, 0, down->scale)),
-                  routs(rout(reinterpret_cast<bf16*>(dB_d), 0, (int)d, 1, down->scale)), w.status, st);
+                  reinterpret_cast<const bf16*>(down->B), r, w.part, routs(rout(sGd, 0, r, r, 0, down->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_d), 0, r, (int)d, 1, down->scale)), w.status, st);
   if (s != QLORA_OK) return s;
   // 2. dH = dY W_d + sG_d A_d^T, with dE, dG formed in the epilogue
   {
@@ -755,9 +834,8 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], dY, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if ((s = map_weights(maps, down->w, nullptr, true, tiles, w.stage0, nullptr, st)) != QLORA_OK) return s;
-    if (!map_bf16(&maps.la[0], sGd, 16, M, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], down->A, 16, h, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
-      return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[0], sGd, M, r, r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[0], down->A, h, r, true, tiles)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
     maps.codes[1] = maps.codes[0];
     maps.absmax[1] = maps.absmax[0];
@@ -770,6 +848,7 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     a.N = (int)h;
     a.nkb0 = (int)cdiv(d, 64);
     a.lora = 1;
+    a.lora_k16 = r / 16;
     a.act = act == QLORA_ACT_SWIGLU ? ACT_SILU : ACT_GELU_TANH;
     a.ldo = (int)h;
     a.Ein = reinterpret_cast<const bf16*>(sv->E);
@@ -784,17 +863,17 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (s != QLORA_OK) return s;
   }
   // 3. dA_d = H^T (s_d G_d)
-  s = pass_colproj(reinterpret_cast<const bf16*>(sv->H), M, h, sGd, 16, w.part,
-                   routs(rout(reinterpret_cast<bf16*>(dA_d), 0, 16, 0, 1.f)), w.status, st);
+  s = pass_colproj(reinterpret_cast<const bf16*>(sv->H), M, h, sGd, r, w.part,
+                   routs(rout(reinterpret_cast<bf16*>(dA_d), 0, r, r, 0, 1.f)), w.status, st);
   if (s != QLORA_OK) return s;
   // 4. G_g = dE B_g^T, dB_g = s_g XA_g^T dE ; G_u = dG B_u^T, dB_u = s_u XA_u^T dG
-  s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), w.part,
-                  routs(rout(w.gu, 0, 32, 0, gate->scale)),
-                  routs(rout(reinterpret_cast<bf16*>(dB_g), 0, (int)h, 1, gate->scale)), w.status, st);
+  s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), r,
+                  w.part, routs(rout(w.gu, 0, r, 2 * r, 0, gate->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_g), 0, r, (int)h, 1, gate->scale)), w.status, st);
   if (s != QLORA_OK) return s;
-  s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), w.part,
-                  routs(rout(w.gu + 16, 0, 32, 0, up->scale)),
-                  routs(rout(reinterpret_cast<bf16*>(dB_u), 0, (int)h, 1, up->scale)), w.status, st);
+  s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), r,
+                  w.part, routs(rout(w.gu + r, 0, r, 2 * r, 0, up->scale)),
+                  routs(rout(reinterpret_cast<bf16*>(dB_u), 0, r, (int)h, 1, up->scale)), w.status, st);
   if (s != QLORA_OK) return s;
   // 5. dX = [dE | dG] [W_g ; W_u] + [sG_g | sG_u] [A_g^T ; A_u^T]
   {
@@ -803,12 +882,10 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if ((s = map_weights(maps, gate->w, &up->w, true, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
-    if (!map_bf16(&maps.la[0], w.gu, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.la[1], w.gu + 16, 16, M, 32, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[0], gate->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
-      return QLORA_ERR_CUDA;
-    if (!map_bf16(&maps.lb[1], up->A, 16, d, 16, 16, lora_rows_box(bnc), CU_TENSOR_MAP_SWIZZLE_32B))
-      return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[0], w.gu, M, r, 2 * r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_left(&maps.la[1], w.gu + r, M, r, 2 * r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[0], gate->A, d, r, true, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[1], up->A, d, r, true, tiles)) return QLORA_ERR_CUDA;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     a.M = (int)M;
@@ -816,6 +893,7 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     a.nkb0 = (int)cdiv(h, 64);
     a.nkb1 = (int)cdiv(h, 64);
     a.lora = 2;
+    a.lora_k16 = r / 16;
     a.ldo = (int)d;
     a.D = reinterpret_cast<bf16*>(dX);
     if (!map_outs(maps, tiles, M, d, d, dX)) return QLORA_ERR_CUDA;
@@ -826,9 +904,9 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (s != QLORA_OK) return s;
   }
   // 6. [dA_g | dA_u] = X^T [sG_g | sG_u]
-  return pass_colproj(reinterpret_cast<const bf16*>(X), M, d, w.gu, 32, w.part,
-                      routs(rout(reinterpret_cast<bf16*>(dA_g), 0, 16, 0, 1.f),
-                            rout(reinterpret_cast<bf16*>(dA_u), 16, 16, 0, 1.f)),
+  return pass_colproj(reinterpret_cast<const bf16*>(X), M, d, w.gu, 2 * r, w.part,
+                      routs(rout(reinterpret_cast<bf16*>(dA_g), 0, r, r, 0, 1.f),
+                            rout(reinterpret_cast<bf16*>(dA_u), r, r, r, 0, 1.f)),
                       w.status, st);
 }
 
@@ -867,12 +945,12 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
 // 16-bit entry points: bf16 base weights, always the staged-feed pair tile
 // (the weight is already what the GEMM streams; nothing is dequantised).
 size_t qlora_linear16_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
-  if (M <= 0 || K <= 0 || N <= 0 || r != 16) return 256;
-  return linear_ws(M, K, N, false);
+  if (M <= 0 || K <= 0 || N <= 0 || !rank_ok(r, 4)) return 256;
+  return linear_ws(M, K, N, r, false);
 }
 size_t qlora_mlp16_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
-  if (M <= 0 || d <= 0 || h <= 0 || r != 16) return 256;
-  return mlp_ws(M, d, h, false);
+  if (M <= 0 || d <= 0 || h <= 0 || !rank_ok(r, 4)) return 256;
+  return mlp_ws(M, d, h, r, false);
 }
 qlora_status qlora_linear16_fwd(const qlora_lora_linear16* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                                 qlora_bf16* XA_saved, void* ws, size_t ws_bytes, qlora_stream_t stream) {
@@ -989,7 +1067,10 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const ql
   if (!lin_nf4) return QLORA_ERR_INVALID_ARG;
   const Lin lv = lin_of(*lin_nf4);
   const Lin* lin = &lv;
-  qlora_status s = check_linear(lin);
+  // The fixed scratch has no room for a staged weight: the staged configuration
+  // falls back to the pair tile that dequantises in the mainloop (rank 16).
+  const int tiles = is_staged(g_tiles) ? 2 : g_tiles;
+  qlora_status s = check_linear(lin, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
   if (M == 0) return QLORA_OK;
@@ -1010,12 +1091,10 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const ql
   bf16* xa = reinterpret_cast<bf16*>(XA_saved);
   bf16* XAs = lin->scale != 1.0f ? reinterpret_cast<bf16*>(w + 256) : xa;
   float* part = reinterpret_cast<float*>(w + 256 + vec);
-  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, part,
-                   routs(rout(xa, 0, 16, 0, 1.f), rout(XAs != xa ? XAs : nullptr, 0, 16, 0, lin->scale)), status, st);
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, 16, part,
+                   routs(rout(xa, 0, 16, 16, 0, 1.f), rout(XAs != xa ? XAs : nullptr, 0, 16, 16, 0, lin->scale)),
+                   status, st);
   if (s != QLORA_OK) return s;
-  // The fixed scratch has no room for a staged weight: the staged configuration
-  // falls back to the pair tile that dequantises in the mainloop.
-  const int tiles = is_staged(g_tiles) ? 2 : g_tiles;
   return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, tiles, nullptr,
                   st);
 }

@@ -125,8 +125,10 @@ struct GemmCfg {
   static constexpr int RA_BYTES = (MODE == MODE_BWD) ? 64 * 16 : BNC * 16;
   static constexpr int S = ST ? 5 : ((CG == 1) ? 3 : (MH == 1 ? 5 : 4));  // operand stages
   static constexpr int RS = ST ? 0 : ((CG == 1) ? 4 : (MH == 1 ? 6 : 8));  // raw stages
-  static constexpr int LA_BYTES = BM * 16 * 2;   // one LoRA left operand tile (128 rows x 16)
-  static constexpr int LBOP = BNC * 32;          // one LoRA right operand (BNC x 16 bf16)
+  // dedicated LoRA operand tiles (rank 16) of the in-mainloop feed; the staged
+  // feed streams its LoRA operands through the operand ring instead
+  static constexpr int LA_BYTES = ST ? 0 : BM * 16 * 2;  // one LoRA left operand tile (128 rows x 16)
+  static constexpr int LBOP = ST ? 0 : BNC * 32;         // one LoRA right operand (BNC x 16 bf16)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + S * A_BYTES;
   static constexpr int OFF_RC = OFF_B + S * B_BYTES;
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
   // belong to it; the other chunks stay zero, so both LoRA MMAs span all BNT
   // columns and each only adds to its own half.
   auto glu_chunk_is_gate = [&](int c) { return static_cast<int>(rank) * C::BNC + c * 64 < C::BNT / 2; };
-  if (EPI == EPI_GLU_FWD) {
+  if (!ST && EPI == EPI_GLU_FWD) {
     for (int c = 0; c < C::BNC / 64; ++c) {
       const int zero_op = glu_chunk_is_gate(c) ? 1 : 0;
       uint4* z = reinterpret_cast<uint4*>(sgen + C::OFF_LB + zero_op * C::LBOP + c * 2048);
@@ -308,6 +310,38 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           }
         }
         if (!ok || args.lora == 0) continue;
+        if constexpr (ST) {
+          // LoRA operands as extra reduction blocks through the operand ring:
+          // A slot <- s*XA (or s*G) [128 rows x 64], B slot <- the LoRA right factor;
+          // ranks below 64 leave the rest of the boxes to the TMA's zero fill.
+          for (int i = 0; i < args.lora; ++i, ++j) {
+            const int s = j % C::S;
+            ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
+            if (!ok) break;
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), (C::A_BYTES + C::B_BYTES) * CG);
+            load(sbase + C::OFF_A + s * C::A_BYTES, &maps.la[i], full_bar(s), 0, half_row(mb, 0));
+            const uint32_t bdst = sbase + C::OFF_B + s * C::B_BYTES;
+            if (MODE == MODE_BWD) {
+              // A_lora rows (this CTA's output columns) x rank, K-major
+              for (int bx = 0; bx < C::BNC / C::BOXR; ++bx)
+                load(bdst + bx * C::BOXR * 128, &maps.lb[i], full_bar(s), 0, n0 + (int)rank * C::BNC + bx * C::BOXR);
+            } else {
+              // B_lora [rank x columns], MN-major 64-column chunks; in the gated forward a chunk of
+              // the other half is read from past the factor's last row, i.e. as zeros
+              for (int c = 0; c < C::BNC / 64; ++c) {
+                const int p = (int)rank * C::BNC + c * 64;
+                int col = n0 + p, y = 0;
+                if (MODE == MODE_FWD_GLU) {
+                  const int op = p < C::BNT / 2 ? 0 : 1;
+                  col = n0 + (op ? p - C::BNT / 2 : p);
+                  y = op == i ? 0 : 64;
+                }
+                load(bdst + c * 8192, &maps.lb[i], full_bar(s), col, y);
+              }
+            }
+          }
+          continue;
+        }
         // LoRA operands of this tile (single buffer, released by the MMA's commit)
         ok = mbar_wait(lora_empty, (tl & 1) ^ 1, args.status);
         if (!ok) break;
@@ -402,7 +436,24 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           umma_commit<CG>(empty_bar(s));
         }
         if (!ok) break;
-        if (args.lora > 0) {
+        if (ST && args.lora > 0) {
+          for (int i = 0; i < args.lora && ok; ++i, ++j) {
+            const int s = j % C::S;
+            ok = mbar_wait(full_bar(s), (j / C::S) & 1, args.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t a = sbase + C::OFF_A + s * C::A_BYTES;
+            const uint32_t bs = sbase + C::OFF_B + s * C::B_BYTES;
+            for (int kk = 0; kk < args.lora_k16; ++kk) {
+              const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, QL_SWZ_128B);
+              const uint64_t bd = (MODE == MODE_BWD) ? smem_desc(bs + kk * 32, 16, 1024, QL_SWZ_128B)
+                                                     : smem_desc(bs + kk * 2048, 8192, 1024, QL_SWZ_128B);
+              umma_bf16<CG>(acc, ad, bd, idesc_lora, 1);
+            }
+            umma_commit<CG>(empty_bar(s));
+          }
+          if (!ok) break;
+        } else if (args.lora > 0) {
           ok = mbar_wait(lora_full, tl & 1, args.status);
           if (!ok) break;
           tc_fence_after();

@@ -37,7 +37,8 @@ struct GemmArgs {
   int N;        // output columns (MODE_FWD_GLU: h, the width of E/G/H)
   int nkb0;     // 64-wide reduction blocks in segment 0
   int nkb1;     // ... in segment 1 (0 if one segment)
-  int lora;     // number of LoRA MMAs (0, 1 or 2)
+  int lora;     // number of LoRA operands (0, 1 or 2)
+  int lora_k16; // staged feed: 16-wide reduction steps per LoRA operand (rank / 16, 1..4)
   int act;      // Act
   int ldo;      // leading dimension (elements) of all outputs / epilogue inputs
   bf16* D;      // EPI_STORE output [M, N]
@@ -81,11 +82,12 @@ __host__ __device__ inline int sk_slots(const SkPart& p, int g) {
   return sk_owner(p, g * p.upg + p.upg - 1) - sk_first(p, g) + 1;
 }
 
-// Output of the partial-sum reduction: 16 of the R partial columns, scaled,
-// rounded to bf16 and written row-major or transposed.
+// Output of the partial-sum reduction: `width` of the R partial columns,
+// scaled, rounded to bf16 and written row-major or transposed.
 struct ReduceOut {
   bf16* ptr;      // destination (nullptr = unused)
-  int col0;       // first of the 16 partial columns this output takes
+  int col0;       // first of the partial columns this output takes
+  int width;      // number of partial columns it takes (the LoRA rank)
   int ld;         // row stride of the destination (elements)
   int transpose;  // 0: dst[row * ld + c], 1: dst[c * ld + row]
   float scale;

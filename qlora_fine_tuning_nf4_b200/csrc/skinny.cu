@@ -45,6 +45,27 @@ QL_DEV void frag_b_kn(uint32_t tile, int row_bytes, int k0, int n0, int lane, ui
   const int k = k0 + (lane & 15);
   ldsm_x2_t(tile + k * row_bytes + n0 * 2, b[0], b[1]);
 }
+
+// A rank-side factor tile: 64 rows x W bf16 columns, stored as W / SUBW
+// sub-tiles of SUBW = min(W, 64) columns, each in the TMA swizzle of its row
+// width (32, 64 or 128 bytes) so that 8-row ldmatrix phases hit distinct banks.
+template <int W>
+struct FTile {
+  static constexpr int SUBW = W < 64 ? W : 64;
+  static constexpr int ROWB = SUBW * 2;
+  static constexpr int SUB_BYTES = 64 * ROWB;
+  static constexpr int BYTES = (W / SUBW) * SUB_BYTES;
+  // byte offset of the 16-byte chunk holding columns [c, c + 8) of row k
+  QL_DEV static int off(int k, int c) {
+    const int x = ROWB == 128 ? (k & 7) : (ROWB == 64 ? ((k >> 1) & 3) : ((k >> 2) & 1));
+    return (c / SUBW) * SUB_BYTES + k * ROWB + ((((c % SUBW) >> 3) ^ x) << 4);
+  }
+};
+// B-fragment (16x8) of a factor tile used as [k][n]: rows [k0, k0+16), columns [n0, n0+8).
+template <int W>
+QL_DEV void frag_b_kn_f(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[2]) {
+  ldsm_x2_t(tile + FTile<W>::off(k0 + (lane & 15), n0), b[0], b[1]);
+}
 // B-fragment from a 128B-swizzled [n][k] tile (rows = output column n,
 // 128 bytes of k per row): reduction [k0, k0+16), columns [n0, n0+8).
 QL_DEV void frag_b_nk(uint32_t tile, int k0, int n0, int lane, uint32_t (&b)[2]) {
@@ -121,16 +142,20 @@ QL_DEV void store_acc(float* base, int ld, int r0, int lane, float (&acc)[NB][4]
 
 // ------------------------------------------------------------- rowproj ---
 // Units: 64x64 tiles (rc, kc), kc fastest; group = row block rc (nkc units).
-// job.part[rc][slot][64][R]: T V over the CTA's tiles of row block rc.
-template <int NV>
+// job.part[rc][slot][64][NF * RW]: T V over the CTA's tiles of row block rc,
+// V = NF factors of RW columns side by side.  BT: the single factor is given
+// transposed, as the LoRA right factor B [RW, K] (G = T B^T).
+template <int RW, int NF, bool BT>
 __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_v0,
                                                              const __grid_constant__ CUtensorMap tmap_v1,
                                                              const __grid_constant__ ReduceJob job, int nkc,
                                                              int* status) {
-  constexpr int R = 16 * NV;
-  constexpr int V_TILE = 64 * 16 * 2;
-  constexpr int STAGE = T_TILE + NV * V_TILE;
+  using F = FTile<RW>;
+  constexpr int R = NF * RW;
+  constexpr int V_TILE = BT ? RW * 128 : F::BYTES;
+  constexpr int STAGE = T_TILE + NF * V_TILE;
+  static_assert(!BT || NF == 1, "transposed factor: one factor");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bars = sbase + SK_STAGES * STAGE;
@@ -148,8 +173,16 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
         const uint32_t st = sbase + s * STAGE;
         mbar_arrive_expect_tx(fb, STAGE);
         tma_load_2d(st, &tmap_t, fb, kc * 64, rc * 64);
-        tma_load_2d(st + T_TILE, &tmap_v0, fb, 0, kc * 64);
-        if (NV == 2) tma_load_2d(st + T_TILE + V_TILE, &tmap_v1, fb, 0, kc * 64);
+        if (BT) {
+          tma_load_2d(st + T_TILE, &tmap_v0, fb, kc * 64, 0);
+        } else {
+#pragma unroll
+          for (int f = 0; f < NF; ++f)
+#pragma unroll
+            for (int sub = 0; sub < RW / F::SUBW; ++sub)
+              tma_load_2d(st + T_TILE + f * V_TILE + sub * F::SUB_BYTES, f ? &tmap_v1 : &tmap_v0, fb,
+                          sub * F::SUBW, kc * 64);
+        }
       });
     return;
   }
@@ -167,7 +200,10 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
 #pragma unroll
         for (int nb = 0; nb < R / 8; ++nb) {
           uint32_t b[2];
-          frag_b_kn(tb + T_TILE + (nb >> 1) * V_TILE, 32, kk * 16, (nb & 1) * 8, lane, b);
+          if (BT)
+            frag_b_nk(tb + T_TILE, kk * 16, nb * 8, lane, b);
+          else
+            frag_b_kn_f<RW>(tb + T_TILE + (nb / (RW / 8)) * V_TILE, kk * 16, (nb % (RW / 8)) * 8, lane, b);
           mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
         }
       }
@@ -188,8 +224,8 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
                                                              const __grid_constant__ CUtensorMap tmap_u,
                                                              const __grid_constant__ ReduceJob job, int nmc,
                                                              int* status) {
-  constexpr int U_TILE = 64 * R * 2;
-  constexpr int STAGE = T_TILE + U_TILE;
+  using F = FTile<R>;
+  constexpr int STAGE = T_TILE + F::BYTES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bars = sbase + SK_STAGES * STAGE;
@@ -207,7 +243,9 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
         const uint32_t st = sbase + s * STAGE;
         mbar_arrive_expect_tx(fb, STAGE);
         tma_load_2d(st, &tmap_t, fb, cc * 64, mc * 64);
-        tma_load_2d(st + T_TILE, &tmap_u, fb, 0, mc * 64);
+#pragma unroll
+        for (int sub = 0; sub < R / F::SUBW; ++sub)
+          tma_load_2d(st + T_TILE + sub * F::SUB_BYTES, &tmap_u, fb, sub * F::SUBW, mc * 64);
       });
     return;
   }
@@ -225,7 +263,7 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
 #pragma unroll
         for (int nb = 0; nb < R / 8; ++nb) {
           uint32_t b[2];
-          frag_b_kn(tb + T_TILE, R * 2, kk * 16, nb * 8, lane, b);
+          frag_b_kn_f<R>(tb + T_TILE, kk * 16, nb * 8, lane, b);
           mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
         }
       }
@@ -316,7 +354,7 @@ __global__ void __launch_bounds__(SK_THREADS) dypass_kernel(const __grid_constan
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
             uint32_t b[2];
-            frag_b_kn(tb + T_TILE, 32, kk * 16, nb * 8, lane, b);
+            frag_b_kn_f<16>(tb + T_TILE, kk * 16, nb * 8, lane, b);
             mma_bf16_16816(qacc[cc][nb], a[0], a[1], a[2], a[3], b[0], b[1]);
           }
         }
@@ -371,7 +409,7 @@ __global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ Red
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const ReduceOut& o = j.outs.o[q];
-    if (o.ptr == nullptr || c < o.col0 || c >= o.col0 + 16) continue;
+    if (o.ptr == nullptr || c < o.col0 || c >= o.col0 + o.width) continue;
     const int cc = c - o.col0;
     const bf16 b0 = __float2bfloat16_rn(o.scale * acc.x), b1 = __float2bfloat16_rn(o.scale * acc.y);
     const bf16 b2 = __float2bfloat16_rn(o.scale * acc.z), b3 = __float2bfloat16_rn(o.scale * acc.w);
@@ -401,34 +439,52 @@ static cudaError_t set_smem(const void* f, int bytes) {
 }
 static int sk_smem(int stage) { return SK_STAGES * stage + 2 * SK_STAGES * 8 + 1024; }
 
-cudaError_t launch_rowproj(int nv, const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
-                           const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
-  const int smem = sk_smem(T_TILE + nv * 2048);
-  if (nv == 1) {
-    cudaError_t e = set_smem((const void*)rowproj_kernel<1>, smem);
-    if (e != cudaSuccess) return e;
-    rowproj_kernel<1><<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
-  } else {
-    cudaError_t e = set_smem((const void*)rowproj_kernel<2>, smem);
-    if (e != cudaSuccess) return e;
-    rowproj_kernel<2><<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
-  }
+template <int RW, int NF, bool BT>
+static cudaError_t launch_rowproj_t(const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
+                                    const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
+  const int vt = BT ? RW * 128 : FTile<RW>::BYTES;
+  const int smem = sk_smem(T_TILE + NF * vt);
+  auto k = rowproj_kernel<RW, NF, BT>;
+  cudaError_t e = set_smem((const void*)k, smem);
+  if (e != cudaSuccess) return e;
+  k<<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
   return cudaGetLastError();
 }
 
+// rank rw in {16, 32, 64}; nf factors (1 or 2), or bt: one factor given as B [rw, K]
+cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
+                           const CUtensorMap& v1, const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
+#define QL_ROW(RW_)                                                                              \
+  if (rw == RW_) {                                                                               \
+    if (bt) return launch_rowproj_t<RW_, 1, true>(t, v0, v1, job, nkc, status, st);              \
+    if (nf == 1) return launch_rowproj_t<RW_, 1, false>(t, v0, v1, job, nkc, status, st);        \
+    return launch_rowproj_t<RW_, 2, false>(t, v0, v1, job, nkc, status, st);                     \
+  }
+  QL_ROW(16)
+  QL_ROW(32)
+  QL_ROW(64)
+#undef QL_ROW
+  return cudaErrorInvalidValue;
+}
+
+template <int R>
+static cudaError_t launch_colproj_t(const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+                                    int* status, cudaStream_t st) {
+  const int smem = sk_smem(T_TILE + FTile<R>::BYTES);
+  cudaError_t e = set_smem((const void*)colproj_kernel<R>, smem);
+  if (e != cudaSuccess) return e;
+  colproj_kernel<R><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
+  return cudaGetLastError();
+}
+
+// R in {16, 32, 64, 128}
 cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
                            int* status, cudaStream_t st) {
-  const int smem = sk_smem(T_TILE + 64 * R * 2);
-  if (R == 16) {
-    cudaError_t e = set_smem((const void*)colproj_kernel<16>, smem);
-    if (e != cudaSuccess) return e;
-    colproj_kernel<16><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
-  } else {
-    cudaError_t e = set_smem((const void*)colproj_kernel<32>, smem);
-    if (e != cudaSuccess) return e;
-    colproj_kernel<32><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
-  }
-  return cudaGetLastError();
+  if (R == 16) return launch_colproj_t<16>(t, u, job, nmc, status, st);
+  if (R == 32) return launch_colproj_t<32>(t, u, job, nmc, status, st);
+  if (R == 64) return launch_colproj_t<64>(t, u, job, nmc, status, st);
+  if (R == 128) return launch_colproj_t<128>(t, u, job, nmc, status, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,

@@ -83,6 +83,22 @@ def test_host_side_rejections(lib):
     assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, 8, 16, ctypes.byref(sv), 16, 10, None) == 4
 
 
+def test_rank_support_follows_the_tile_configuration(lib):
+    prev = ops.qlora_set_tile_config(4)
+    try:
+        for r in (16, 32, 64):  # staged feed: ranks 16, 32, 64
+            assert ops.qlora_linear_workspace_bytes(256, 512, 1024, r) > 256
+            assert ops.qlora_mlp16_workspace_bytes(256, 512, 1024, r) > 256
+        assert ops.qlora_linear_workspace_bytes(256, 512, 1024, 48) == 256
+        f = lib.qlora_linear_fwd
+        assert f(ctypes.byref(_lin(r=48)), 16, 8, 16, 16, 16, 1 << 30, None) == 2
+        ops.qlora_set_tile_config(2)  # dequantised in the mainloop: rank 16 only
+        assert ops.qlora_linear_workspace_bytes(256, 512, 1024, 32) == 256
+        assert f(ctypes.byref(_lin(r=32)), 16, 8, 16, 16, 16, 1 << 30, None) == 2
+    finally:
+        ops.qlora_set_tile_config(prev)
+
+
 def test_tile_config_setting(lib):
     prev = ops.qlora_set_tile_config(1)
     assert ops.qlora_set_tile_config(prev) == 1
