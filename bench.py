@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
+    ap.add_argument("--op", default="mlp", choices=["mlp", "qkv"],
+                    help="the timed step: the gated MLP (the metric) or the fused Q/K/V projection (GQA widths)")
     ap.add_argument("--rank", type=int, default=0, choices=[0, 16, 32, 64],
                     help="LoRA rank (0 = the workload's, 16); s = alpha / r with alpha = the rank")
     ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
@@ -232,24 +234,13 @@ def run_reference(args, wl):
 
 # -------------------------------------------------------------- GPU arm ----
 
-def run_ours(args, wl):
+def setup_mlp(args, wl, M, d, h, r, act, rank, world, dev):
+    """Tensors and step of the gated MLP fwd + bwd (the metric's workload)."""
     import torch
     import torch.distributed as dist
 
     from qlora_fine_tuning_nf4_b200 import ops
     from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_mlp_problem
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    ops.lib()
-    ops.qlora_set_tile_config(args.tiles)
-    M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
 
     # Inputs: same seeded recipe as the tests; each rank draws its own batch.
     p = make_mlp_problem(M, d, h, r, wl["alpha"], wl["seed"] + 1000 * rank)
@@ -283,6 +274,80 @@ def run_ours(args, wl):
         mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads)
         if world > 1:
             dist.all_reduce(flat)
+
+    kflops = {k: kernel_flops(k, M, d, h, r) for k in ("gemm_nf4_gateup_glu_fwd", "gemm_nf4_fwd",
+                                                         "gemm_nf4_down_bwd_glu", "gemm_nf4_bwd_dx")}
+    dq = 2 * (2 * h * d + h * d) * (0.5 + 4 / 64 + 2)  # gate, up, down in the forward and in the backward
+    return X, dY, Y, grads, flat, step, mlp_flops(M, d, h, r), kflops, dq, ws, {"h": h, "act": act}
+
+
+def setup_qkv(args, wl, M, d, r, rank, world, dev):
+    """Tensors and step of the fused Q/K/V projection fwd + bwd at the workload's attention widths."""
+    import torch
+    import torch.distributed as dist
+
+    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_qkv_problem
+    from qlora_fine_tuning_nf4_b200.workloads import linear_flops
+
+    nq, nkv = wl["nq"], wl["nkv"]
+    p = make_qkv_problem(M, d, nq, nkv, nkv, r, wl["alpha"], wl["seed"] + 1000 * rank)
+    lins = {}
+    for n in "qkv":
+        lins[n] = ops.LoraLinear(ops.nf4_quantize(bits_to_torch(p["W_" + n], dev)), bits_to_torch(p["A_" + n], dev),
+                                 bits_to_torch(p["B_" + n], dev), p["s"])
+    X = bits_to_torch(p["X"], dev)
+    dY = bits_to_torch(p["dY"], dev)
+    del p
+    ws = ops.Workspace(dev)
+    nt = nq + 2 * nkv
+    Y = torch.empty(M, nt, dtype=torch.bfloat16, device=dev)
+    XA = torch.empty(M, 3 * r, dtype=torch.bfloat16, device=dev)
+    sizes = [(f"d{m}_{n}", (d, r) if m == "A" else (r, wn)) for n, wn in (("q", nq), ("k", nkv), ("v", nkv))
+             for m in "AB"]
+    flat = torch.empty(sum(a * b for _, (a, b) in sizes), dtype=torch.bfloat16, device=dev)
+    grads, off = {}, 0
+    for name, (a, b) in sizes:
+        grads[name] = flat[off:off + a * b].view(a, b)
+        off += a * b
+    grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        ops.qlora_qkv_fwd(lins["q"], lins["k"], lins["v"], X, ws, Y=Y, XA=XA)
+        ops.qlora_qkv_bwd(lins["q"], lins["k"], lins["v"], X, XA, dY, ws, grads=grads)
+        if world > 1:
+            dist.all_reduce(flat)
+
+    flop = sum(linear_flops(M, d, n, r) for n in (nq, nkv, nkv))
+    kflops = {"gemm_nf4_fwd": 2 * M * d * nt + 2 * M * r * nt, "gemm_nf4_bwd_dx": 2 * M * nt * d + 2 * M * 3 * r * d}
+    dq = 2 * nt * d * (0.5 + 4 / 64 + 2)
+    return X, dY, Y, grads, flat, step, flop, kflops, dq, ws, {"nq": nq, "nk": nkv, "nv": nkv}
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_mlp_problem
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ops.lib()
+    ops.qlora_set_tile_config(args.tiles)
+    M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
+    if args.op == "qkv":
+        (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
+            setup_qkv(args, wl, M, d, r, rank, world, dev)
+    else:
+        (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
+            setup_mlp(args, wl, M, d, h, r, act, rank, world, dev)
 
     stream = torch.cuda.current_stream()
     clk = ClockSampler(smi_device_id(local))
@@ -320,18 +385,17 @@ def run_ours(args, wl):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
-    flop_step = mlp_flops(M, d, h, r)
     value = flop_step * args.steps * world / (ms / 1e3) / 1e12
     tokens = M * args.steps * world / (ms / 1e3)
     pk = peaks()
 
     # ---- end-to-end through the public API with host buffers ----
-    hX = torch.empty(M, d, dtype=torch.bfloat16, pin_memory=True)
-    hdY = torch.empty(M, d, dtype=torch.bfloat16, pin_memory=True)
+    hX = torch.empty(X.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdY = torch.empty(dY.shape, dtype=torch.bfloat16, pin_memory=True)
     hX.copy_(X.cpu())
     hdY.copy_(dY.cpu())
-    hY = torch.empty_like(hX, pin_memory=True)
-    hdX = torch.empty_like(hX, pin_memory=True)
+    hY = torch.empty(Y.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdX = torch.empty(grads["dX"].shape, dtype=torch.bfloat16, pin_memory=True)
     hflat = torch.empty(flat.numel(), dtype=torch.bfloat16, pin_memory=True)
     e2e_steps = max(3, min(args.steps, 20))
 
@@ -356,17 +420,17 @@ def run_ours(args, wl):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ems = float(t.item())
     e2e_value = flop_step * e2e_steps * world / (ems / 1e3) / 1e12
-    h2d = 2 * M * d * 2
-    d2h = 2 * M * d * 2 + flat.numel() * 2
+    h2d = (X.numel() + dY.numel()) * 2
+    d2h = (Y.numel() + grads["dX"].numel() + flat.numel()) * 2
 
     # ---- roofline of the dominant kernel (live CUDA-event times) ----
     roof = None
-    tc = {k: v for k, v in trace.items() if kernel_flops(k, M, d, h, r)}
+    tc = {k: v for k, v in trace.items() if kflops.get(k)}
     if tc:
         top = max(tc, key=lambda k: tc[k][1])
         n_l, tot = tc[top]
         avg_s = tot / n_l / 1e3
-        ach = kernel_flops(top, M, d, h, r) / avg_s / 1e12
+        ach = kflops[top] / avg_s / 1e12
         peak = pk["bf16_sustained"]
         roof = {"bound": "tensor", "kernel": top, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "peak_kind": f"bf16 dense, sustained, {pk['src']}",
@@ -378,13 +442,12 @@ def run_ours(args, wl):
     dq = None
     if "nf4_dequantize" in trace:
         n_l, tot = trace["nf4_dequantize"]
-        dq_bytes = args.steps * 2 * (2 * h * d + h * d) * (0.5 + 4 / 64 + 2)  # gate, up, down in fwd and in bwd
-        gbs = dq_bytes / (tot / 1e3) / 1e9
+        gbs = args.steps * dq_step_bytes / (tot / 1e3) / 1e9
         dq = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
               "launches": n_l, "ms_per_step": tot / args.steps}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "mlp":
         rows = 512
         dt, fl, cores = oracle_sample(wl, rows)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -400,7 +463,7 @@ def run_ours(args, wl):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "tokens_per_s": tokens, "frac_of_bf16_peak": value / world / pk["bf16"],
         "frac_of_bf16_peak_sustained": value / world / pk["bf16_sustained"],
-        "config": {"workload": args.workload, "M_per_gpu": M, "d": d, "h": h, "r": r, "act": act,
+        "config": {"workload": args.workload, "op": args.op, "M_per_gpu": M, "d": d, **cfg_extra, "r": r,
                    "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
                    "gemm_tiles": ops.TILE_CONFIGS[4 if args.weights == "bf16" else args.tiles],
                    "base_weights": args.weights, "l2": L2_NOTE},

@@ -57,7 +57,7 @@ typedef uint16_t qlora_bf16;                /* bf16 bit pattern */
 typedef enum {
   QLORA_OK = 0,
   QLORA_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum */
-  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* k_in % 256 != 0 for the GEMM paths, n_out % 8 != 0, r != 16 ... */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* k_in % 256 != 0 for the GEMM paths, n_out % 8 != 0, unsupported rank ... */
   QLORA_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
   QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
   QLORA_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
@@ -82,8 +82,8 @@ typedef struct {
   qlora_nf4 w;
   const qlora_bf16* A;
   const qlora_bf16* B;
-  int32_t r;   /* must be 16 */
-  float scale; /* s = alpha / r */
+  int32_t r;   /* 16, 32 or 64 (tile configuration 4); 16 (configurations 1-3) */
+  float scale; /* s = alpha / r (or any scale, e.g. alpha / sqrt(r)) */
 } qlora_lora_linear;
 
 /* One projection with a frozen bf16 base W [n_out, k_in] (row-major) instead
@@ -96,8 +96,8 @@ typedef struct {
   int64_t k_in;
   const qlora_bf16* A;
   const qlora_bf16* B;
-  int32_t r;   /* must be 16 */
-  float scale; /* s = alpha / r */
+  int32_t r;   /* 16, 32 or 64 */
+  float scale; /* s = alpha / r (or any scale) */
 } qlora_lora_linear16;
 
 /* Tensors the MLP forward saves for its backward (caller-allocated):
@@ -208,6 +208,31 @@ QLORA_API qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16*
                                        int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
                                        qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
                                        void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Fused Q/K/V projection (the pages' manual-autograd QKV, with grouped-query
+ * K/V widths, e.g. Mistral's 4096 / 1024 / 1024): three NF4 projections q, k,
+ * v of one input X [M, k_in] with the same k_in and rank, computed as one GEMM
+ * over the three dequantised weights stacked by rows.
+ *   XA = X [A_q | A_k | A_v]                        -> XA_saved [M, 3r]
+ *   Y  = [Y_q | Y_k | Y_v], Y_p = X dequant(W_p)^T + s_p XA_p B_p
+ *                                                   -> Y [M, nq + nk + nv]
+ * Backward from dY = [dY_q | dY_k | dY_v] (same layout as Y):
+ *   dX = sum_p dY_p dequant(W_p) + s_p (dY_p B_p^T) A_p^T   (one GEMM over the
+ *   concatenated reduction, three LoRA steps), dA_p, dB_p as qlora_linear_bwd.
+ * Requires nq % 256 == 0 and nk % 256 == 0 (an output tile never spans two
+ * projections), k_in % 256 == 0, r in {16, 32, 64}.  Always runs the staged
+ * feed (tile configuration 4); the workspace also holds the stacked bf16
+ * weight ((nq + nk + nv) * k_in * 2 bytes). */
+QLORA_API size_t qlora_qkv_workspace_bytes(int64_t M, int64_t k_in, int64_t nq, int64_t nk, int64_t nv, int32_t r);
+QLORA_API qlora_status qlora_qkv_fwd(const qlora_lora_linear* q, const qlora_lora_linear* k,
+                                     const qlora_lora_linear* v, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
+                                     qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes,
+                                     qlora_stream_t stream);
+QLORA_API qlora_status qlora_qkv_bwd(const qlora_lora_linear* q, const qlora_lora_linear* k,
+                                     const qlora_lora_linear* v, const qlora_bf16* X, const qlora_bf16* XA_saved,
+                                     const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_q,
+                                     qlora_bf16* dB_q, qlora_bf16* dA_k, qlora_bf16* dB_k, qlora_bf16* dA_v,
+                                     qlora_bf16* dB_v, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* Reads the device status word in `workspace` (synchronising `stream`),
  * clears it, and maps it to a status: QLORA_OK, QLORA_ERR_TIMEOUT or

@@ -25,7 +25,8 @@ cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, 
                             cudaStream_t stream);
 int gemm_nf4_b_cols_per_cta(int tiles);
 cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
-                           const CUtensorMap& v1, const ReduceJob& job, int nkc, int* status, cudaStream_t st);
+                           const CUtensorMap& v1, const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
+                           cudaStream_t st);
 cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
                            int* status, cudaStream_t st);
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
@@ -207,6 +208,7 @@ size_t rowproj_part_bytes(int64_t M, int64_t K, int R) {
   return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K, R).slot_cap * 64 * R * 4;
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
+  R = R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 128));  // the kernel's tile width
   return static_cast<size_t>(cdiv(ncols, 64)) * plan_colproj(M, ncols, R).slot_cap * 64 * R * 4;
 }
 size_t dypass_gpart_bytes(int64_t M, int64_t N) {
@@ -237,29 +239,33 @@ ReduceJob reduce_job(float* part, int64_t groups, int grows, int64_t rows, int R
 // ------------------------------------------------------------ passes ----
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
-// A rank-side factor [rows, cols] (row stride ld) as the skinny kernels read it:
-// 64-row boxes of min(cols, 64) columns in the swizzle of that row width.
-bool map_factor(CUtensorMap* m, const void* p, int64_t rows, int cols, int64_t ld) {
-  const int subw = cols < 64 ? cols : 64;
+// A rank-side factor [rows, cols] (row stride ld) as the skinny kernels read it
+// in tiles `tcols` wide (>= cols; the TMA zero-fills the difference): 64-row
+// boxes of min(tcols, 64) columns in the swizzle of that row width.
+bool map_factor(CUtensorMap* m, const void* p, int64_t rows, int cols, int64_t ld, int tcols = 0) {
+  const int tc = tcols ? tcols : cols;
+  const int subw = tc < 64 ? tc : 64;
   const CUtensorMapSwizzle swz = subw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                             : (subw == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
   return map_bf16(m, p, cols, rows, ld, subw, 64, swz);
 }
 
-// P = T V (V = one or two [K, r] LoRA A factors) -> outs (bf16, optional scaled copies)
+// P = T V (V = up to three [K, r] LoRA A factors side by side) -> outs (bf16, optional scaled copies)
 qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, int r, float* part,
-                          ReduceOuts outs, int* status, cudaStream_t st) {
-  CUtensorMap mt, mv0, mv1;
-  const int nv = V1 ? 2 : 1;
+                          ReduceOuts outs, int* status, cudaStream_t st, const bf16* V2 = nullptr) {
+  CUtensorMap mt, mv0, mv1, mv2;
+  const int nv = V2 ? 3 : (V1 ? 2 : 1);
   if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_factor(&mv0, V0, K, r, r)) return QLORA_ERR_CUDA;
   if (!map_factor(&mv1, V1 ? V1 : V0, K, r, r)) return QLORA_ERR_CUDA;
+  if (!map_factor(&mv2, V2 ? V2 : V0, K, r, r)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_rowproj(M, K, nv * r);
   const int64_t nrc = cdiv(M, 64);
   const ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_ROWPROJ, st);
-    const qlora_status s = cuda_status(launch_rowproj(r, nv, false, mt, mv0, mv1, j, (int)cdiv(K, 64), status, st));
+    const qlora_status s =
+        cuda_status(launch_rowproj(r, nv, false, mt, mv0, mv1, mv2, j, (int)cdiv(K, 64), status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
@@ -268,28 +274,32 @@ qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, c
 
 // G = T B^T (B = LoRA right factor [r, N]) -> outs
 qlora_status pass_rowproj_bt(const bf16* T, int64_t M, int64_t N, const bf16* B, int r, float* part,
-                             ReduceOuts outs, int* status, cudaStream_t st) {
+                             ReduceOuts outs, int* status, cudaStream_t st, int64_t ldt = 0) {
   CUtensorMap mt, mb;
-  if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mt, T, N, M, ldt ? ldt : N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mb, B, N, r, N, 64, r, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_rowproj(M, N, r);
   const int64_t nrc = cdiv(M, 64);
   const ReduceJob j = reduce_job(part, nrc, 64, M, r, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_ROWPROJ, st);
-    const qlora_status s = cuda_status(launch_rowproj(r, 1, true, mt, mb, mb, j, (int)cdiv(N, 64), status, st));
+    const qlora_status s = cuda_status(launch_rowproj(r, 1, true, mt, mb, mb, mb, j, (int)cdiv(N, 64), status, st));
     if (s != QLORA_OK) return s;
   }
   KScope k(K_REDUCE, st);
   return cuda_status(launch_reduce(j, nullptr, st));
 }
 
-// Q = T^T U (U [M, R], contiguous) -> outs
+// Supported factor-tile widths of the colproj kernel: R rounded up to 16, 32, 64 or 128.
+int colproj_width(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 128)); }
+
+// Q = T^T U (U [M, R] with row stride ldu, R <= 128) -> outs
 qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U, int R, float* part,
-                          ReduceOuts outs, int* status, cudaStream_t st) {
+                          ReduceOuts outs, int* status, cudaStream_t st, int64_t ldt = 0, int64_t ldu = 0) {
   CUtensorMap mt, mu;
-  if (!map_bf16(&mt, T, ncols, M, ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_factor(&mu, U, M, R, R)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mt, T, ncols, M, ldt ? ldt : ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_factor(&mu, U, M, R, ldu ? ldu : R, colproj_width(R))) return QLORA_ERR_CUDA;
+  R = colproj_width(R);
   const SkPlan p = plan_colproj(M, ncols, R);
   const int64_t ncc = cdiv(ncols, 64);
   const ReduceJob j = reduce_job(part, ncc, 64, ncols, R, p.slot_cap, 0, p.sp, outs);
@@ -305,15 +315,16 @@ qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U
 // G = T Bl^T ([M, r]) and Q = T^T U ([N, r]) for T [M, N]: one fused read of T
 // at rank 16, a G pass and a Q pass at larger ranks.
 qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, const bf16* Bl, int r, float* part,
-                         ReduceOuts gouts, ReduceOuts qouts, int* status, cudaStream_t st) {
+                         ReduceOuts gouts, ReduceOuts qouts, int* status, cudaStream_t st, int64_t ldt = 0,
+                         int64_t ldu = 0) {
   if (r != 16) {
-    const qlora_status s = pass_rowproj_bt(T, M, N, Bl, r, part, gouts, status, st);
+    const qlora_status s = pass_rowproj_bt(T, M, N, Bl, r, part, gouts, status, st, ldt);
     if (s != QLORA_OK) return s;
-    return pass_colproj(T, M, N, U, r, part, qouts, status, st);
+    return pass_colproj(T, M, N, U, r, part, qouts, status, st, ldt, ldu);
   }
   CUtensorMap mt, mu, mb;
-  if (!map_bf16(&mt, T, N, M, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-  if (!map_factor(&mu, U, M, 16, 16)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mt, T, N, M, ldt ? ldt : N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_factor(&mu, U, M, 16, ldu ? ldu : 16)) return QLORA_ERR_CUDA;
   if (!map_bf16(&mb, Bl, N, 16, N, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_dypass(M, N);
   const int64_t nrc = cdiv(M, 64), nch = cdiv(N, 64), ncb = cdiv(nch, kDyCC);
@@ -908,6 +919,192 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
                       routs(rout(reinterpret_cast<bf16*>(dA_g), 0, r, r, 0, 1.f),
                             rout(reinterpret_cast<bf16*>(dA_u), r, r, r, 0, 1.f)),
                       w.status, st);
+}
+
+// ------------------------------------------------------------ fused QKV --
+namespace {
+// QKV workspace: [status | 256 B][s XA, M x 3r][s G, M x 3r][partials][staged [nq+nk+nv, K] weight]
+size_t qkv_ws(int64_t M, int64_t K, int64_t nq, int64_t nk, int64_t nv, int r) {
+  const size_t vec = align256(static_cast<size_t>(M) * 3 * r * 2);
+  size_t part = rowproj_part_bytes(M, K, 3 * r);
+  for (int64_t n : {nq, nk, nv}) part = std::max(part, dypass_part_bytes(M, n, r));
+  part = std::max(part, 3 * r <= 128 ? colproj_part_bytes(M, K, 3 * r) : colproj_part_bytes(M, K, r));
+  return 256 + 2 * vec + align256(part) + stage_bytes(nq + nk + nv, K);
+}
+qlora_status check_qkv(const Lin* q, const Lin* k, const Lin* v) {
+  qlora_status s;
+  for (const Lin* l : {q, k, v})
+    if ((s = check_linear(l, 4)) != QLORA_OK) return s;
+  if (q->w.k_in != k->w.k_in || q->w.k_in != v->w.k_in) return QLORA_ERR_INVALID_ARG;
+  if (q->r != k->r || q->r != v->r) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (q->w.n_out % 256 || k->w.n_out % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;  // tiles never straddle
+  if (q->w.w16 || k->w.w16 || v->w.w16) return QLORA_ERR_INVALID_ARG;
+  if (q->w.n_out + k->w.n_out + v->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+// the three weights dequantised into consecutive rows of one [nq + nk + nv, K] buffer
+qlora_status stage_qkv(const Lin* q, const Lin* k, const Lin* v, bf16* stage, cudaStream_t st) {
+  const int64_t K = q->w.k_in;
+  qlora_status s = stage_weights(q->w, stage, &k->w, stage + q->w.n_out * K, st);
+  if (s != QLORA_OK) return s;
+  return stage_weights(v->w, stage + (q->w.n_out + k->w.n_out) * K, nullptr, nullptr, st);
+}
+}  // namespace
+
+size_t qlora_qkv_workspace_bytes(int64_t M, int64_t k_in, int64_t nq, int64_t nk, int64_t nv, int32_t r) {
+  if (M <= 0 || k_in <= 0 || nq <= 0 || nk <= 0 || nv <= 0 || !rank_ok(r, 4)) return 256;
+  return qkv_ws(M, k_in, nq, nk, nv, r);
+}
+
+qlora_status qlora_qkv_fwd(const qlora_lora_linear* q_, const qlora_lora_linear* k_, const qlora_lora_linear* v_,
+                           const qlora_bf16* X, int64_t M, qlora_bf16* Y, qlora_bf16* XA_saved, void* ws,
+                           size_t ws_bytes, qlora_stream_t stream) {
+  if (!q_ || !k_ || !v_) return QLORA_ERR_INVALID_ARG;
+  const Lin lq = lin_of(*q_), lk = lin_of(*k_), lv = lin_of(*v_);
+  const Lin* L[3] = {&lq, &lk, &lv};
+  qlora_status s = check_qkv(&lq, &lk, &lv);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  if (!X || !Y || !XA_saved || !ws) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int r = lq.r;
+  const int64_t K = lq.w.k_in, nq = lq.w.n_out, nk = lk.w.n_out, nv = lv.w.n_out, Nt = nq + nk + nv;
+  if (ws_bytes < qkv_ws(M, K, nq, nk, nv, r)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const size_t vec = align256(static_cast<size_t>(M) * 3 * r * 2);
+  int* status = reinterpret_cast<int*>(w);
+  bf16* sxa = reinterpret_cast<bf16*>(w + 256);
+  float* part = reinterpret_cast<float*>(w + 256 + 2 * vec);
+  bf16* stage = reinterpret_cast<bf16*>(w + qkv_ws(M, K, nq, nk, nv, r) - stage_bytes(Nt, K));
+  bf16* xa = reinterpret_cast<bf16*>(XA_saved);
+  // [XA_q | XA_k | XA_v] = X [A_q | A_k | A_v] in one pass over X, plus the s-scaled copies
+  s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lq.A),
+                   reinterpret_cast<const bf16*>(lk.A), r, part,
+                   routs(rout(xa, 0, 3 * r, 3 * r, 0, 1.f), rout(sxa, 0, r, 3 * r, 0, lq.scale),
+                         rout(sxa + r, r, r, 3 * r, 0, lk.scale), rout(sxa + 2 * r, 2 * r, r, 3 * r, 0, lv.scale)),
+                   status, st, reinterpret_cast<const bf16*>(lv.A));
+  if (s != QLORA_OK) return s;
+  if ((s = stage_qkv(&lq, &lk, &lv, stage, st)) != QLORA_OK) return s;
+  // Y = X [W_q ; W_k ; W_v]^T + per column block s_p (X A_p) B_p
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const Wt wall = {nullptr, nullptr, nullptr, Nt, K};
+  const int tiles = 4;
+  if (!map_bf16(&maps.a[0], X, K, M, K, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  if (!map_staged(&maps.b[0], stage, wall, false, gemm_nf4_b_cols_per_cta(tiles))) return QLORA_ERR_CUDA;
+  for (int p = 0; p < 3; ++p) {
+    if (!map_lora_left(&maps.la[p], sxa + p * r, M, r, 3 * r, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[p], L[p]->B, L[p]->w.n_out, r, false, tiles)) return QLORA_ERR_CUDA;
+  }
+  maps.a[1] = maps.a[0];
+  maps.b[1] = maps.b[0];
+  if (!map_outs(maps, tiles, M, Nt, Nt, Y)) return QLORA_ERR_CUDA;
+  GemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.M = (int)M;
+  a.N = (int)Nt;
+  a.nkb0 = (int)(K / 64);
+  a.lora = 1;
+  a.lora_k16 = r / 16;
+  a.ncut[0] = (int)nq;
+  a.ncut[1] = (int)(nq + nk);
+  a.ldo = (int)Nt;
+  a.D = reinterpret_cast<bf16*>(Y);
+  a.status = status;
+  a.group_m = kGroupM;
+  KScope kk(K_GEMM_FWD, st);
+  return cuda_status(launch_gemm_nf4(MODE_FWD, EPI_STORE, tiles, maps, a, st));
+}
+
+qlora_status qlora_qkv_bwd(const qlora_lora_linear* q_, const qlora_lora_linear* k_, const qlora_lora_linear* v_,
+                           const qlora_bf16* X, const qlora_bf16* XA_saved, const qlora_bf16* dY, int64_t M,
+                           qlora_bf16* dX, qlora_bf16* dA_q, qlora_bf16* dB_q, qlora_bf16* dA_k, qlora_bf16* dB_k,
+                           qlora_bf16* dA_v, qlora_bf16* dB_v, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!q_ || !k_ || !v_) return QLORA_ERR_INVALID_ARG;
+  const Lin lq = lin_of(*q_), lk = lin_of(*k_), lv = lin_of(*v_);
+  const Lin* L[3] = {&lq, &lk, &lv};
+  qlora_status s = check_qkv(&lq, &lk, &lv);
+  if (s != QLORA_OK) return s;
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (M == 0) return QLORA_OK;
+  qlora_bf16* dA[3] = {dA_q, dA_k, dA_v};
+  qlora_bf16* dB[3] = {dB_q, dB_k, dB_v};
+  if (!X || !XA_saved || !dY || !dX || !ws) return QLORA_ERR_INVALID_ARG;
+  for (int p = 0; p < 3; ++p)
+    if (!dA[p] || !dB[p]) return QLORA_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, XA_saved, dY, dX, dA_q, dB_q, dA_k, dB_k, dA_v, dB_v, ws};
+  for (const void* p : ptrs)
+    if (misaligned(p)) return QLORA_ERR_MISALIGNED;
+  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int r = lq.r;
+  const int64_t K = lq.w.k_in, nq = lq.w.n_out, nk = lk.w.n_out, nv = lv.w.n_out, Nt = nq + nk + nv;
+  const int64_t off[3] = {0, nq, nq + nk};
+  if (ws_bytes < qkv_ws(M, K, nq, nk, nv, r)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const size_t vec = align256(static_cast<size_t>(M) * 3 * r * 2);
+  int* status = reinterpret_cast<int*>(w);
+  bf16* sg = reinterpret_cast<bf16*>(w + 256 + vec);
+  float* part = reinterpret_cast<float*>(w + 256 + 2 * vec);
+  bf16* stage = reinterpret_cast<bf16*>(w + qkv_ws(M, K, nq, nk, nv, r) - stage_bytes(Nt, K));
+  const bf16* dy = reinterpret_cast<const bf16*>(dY);
+  const bf16* xa = reinterpret_cast<const bf16*>(XA_saved);
+  // per projection: G_p = dY_p B_p^T (stored s_p-scaled into [sG_q | sG_k | sG_v]), dB_p = s_p XA_p^T dY_p
+  for (int p = 0; p < 3; ++p) {
+    s = pass_dypass(dy + off[p], M, L[p]->w.n_out, xa + p * r, reinterpret_cast<const bf16*>(L[p]->B), r, part,
+                    routs(rout(sg + p * r, 0, r, 3 * r, 0, L[p]->scale)),
+                    routs(rout(reinterpret_cast<bf16*>(dB[p]), 0, r, (int)L[p]->w.n_out, 1, L[p]->scale)), status,
+                    st, Nt, 3 * r);
+    if (s != QLORA_OK) return s;
+  }
+  if ((s = stage_qkv(&lq, &lk, &lv, stage, st)) != QLORA_OK) return s;
+  // dX = dY [W_q ; W_k ; W_v] + sum_p (s_p G_p) A_p^T: one concatenated reduction and three LoRA blocks
+  {
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    const Wt wall = {nullptr, nullptr, nullptr, Nt, K};
+    const int tiles = 4;
+    if (!map_bf16(&maps.a[0], dY, Nt, M, Nt, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (!map_staged(&maps.b[0], stage, wall, true, gemm_nf4_b_cols_per_cta(tiles))) return QLORA_ERR_CUDA;
+    for (int p = 0; p < 3; ++p) {
+      if (!map_lora_left(&maps.la[p], sg + p * r, M, r, 3 * r, tiles)) return QLORA_ERR_CUDA;
+      if (!map_lora_right(&maps.lb[p], L[p]->A, K, r, true, tiles)) return QLORA_ERR_CUDA;
+    }
+    maps.a[1] = maps.a[0];
+    maps.b[1] = maps.b[0];
+    if (!map_outs(maps, tiles, M, K, K, dX)) return QLORA_ERR_CUDA;
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.M = (int)M;
+    a.N = (int)K;
+    a.nkb0 = (int)cdiv(Nt, 64);
+    a.lora = 3;
+    a.lora_k16 = r / 16;
+    a.ldo = (int)K;
+    a.D = reinterpret_cast<bf16*>(dX);
+    a.status = status;
+    a.group_m = kGroupM;
+    KScope kk(K_GEMM_BWD, st);
+    s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
+    if (s != QLORA_OK) return s;
+  }
+  // dA_p = X^T (s_p G_p): one pass over X while 3r fits a factor tile
+  const bf16* x = reinterpret_cast<const bf16*>(X);
+  if (3 * r <= 128)
+    return pass_colproj(x, M, K, sg, 3 * r, part,
+                        routs(rout(reinterpret_cast<bf16*>(dA_q), 0, r, r, 0, 1.f),
+                              rout(reinterpret_cast<bf16*>(dA_k), r, r, r, 0, 1.f),
+                              rout(reinterpret_cast<bf16*>(dA_v), 2 * r, r, r, 0, 1.f)),
+                        status, st);
+  for (int p = 0; p < 3; ++p) {
+    s = pass_colproj(x, M, K, sg + p * r, r, part, routs(rout(reinterpret_cast<bf16*>(dA[p]), 0, r, r, 0, 1.f)),
+                     status, st, 0, 3 * r);
+    if (s != QLORA_OK) return s;
+  }
+  return QLORA_OK;
 }
 
 // NF4 entry points: the current tile configuration.

@@ -260,6 +260,8 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
       bool ok = true;
       for (int i = 0; i < 2; ++i) {
         tma_prefetch_desc(&maps.a[i]);
+        tma_prefetch_desc(&maps.la[i]);
+        tma_prefetch_desc(&maps.lb[i]);
         if constexpr (ST) {
           tma_prefetch_desc(&maps.b[i]);
         } else {
@@ -314,29 +316,33 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           // LoRA operands as extra reduction blocks through the operand ring:
           // A slot <- s*XA (or s*G) [128 rows x 64], B slot <- the LoRA right factor;
           // ranks below 64 leave the rest of the boxes to the TMA's zero fill.
+          // plain forward of fused projections: the tile's columns belong to one of them
+          const int fop = (args.ncut[1] > 0 && n0 >= args.ncut[1]) ? 2 : ((args.ncut[0] > 0 && n0 >= args.ncut[0]) ? 1 : 0);
+          const int fcol0 = fop == 0 ? 0 : args.ncut[fop - 1];
           for (int i = 0; i < args.lora; ++i, ++j) {
             const int s = j % C::S;
+            const int op = MODE == MODE_FWD ? fop : i;
             ok = mbar_wait(empty_bar(s), ((j / C::S) & 1) ^ 1, args.status);
             if (!ok) break;
             if (rank == 0) mbar_arrive_expect_tx(full_bar(s), (C::A_BYTES + C::B_BYTES) * CG);
-            load(sbase + C::OFF_A + s * C::A_BYTES, &maps.la[i], full_bar(s), 0, half_row(mb, 0));
+            load(sbase + C::OFF_A + s * C::A_BYTES, &maps.la[op], full_bar(s), 0, half_row(mb, 0));
             const uint32_t bdst = sbase + C::OFF_B + s * C::B_BYTES;
             if (MODE == MODE_BWD) {
               // A_lora rows (this CTA's output columns) x rank, K-major
               for (int bx = 0; bx < C::BNC / C::BOXR; ++bx)
-                load(bdst + bx * C::BOXR * 128, &maps.lb[i], full_bar(s), 0, n0 + (int)rank * C::BNC + bx * C::BOXR);
+                load(bdst + bx * C::BOXR * 128, &maps.lb[op], full_bar(s), 0, n0 + (int)rank * C::BNC + bx * C::BOXR);
             } else {
               // B_lora [rank x columns], MN-major 64-column chunks; in the gated forward a chunk of
               // the other half is read from past the factor's last row, i.e. as zeros
               for (int c = 0; c < C::BNC / 64; ++c) {
                 const int p = (int)rank * C::BNC + c * 64;
-                int col = n0 + p, y = 0;
+                int col = n0 + p - fcol0, y = 0;
                 if (MODE == MODE_FWD_GLU) {
-                  const int op = p < C::BNT / 2 ? 0 : 1;
-                  col = n0 + (op ? p - C::BNT / 2 : p);
-                  y = op == i ? 0 : 64;
+                  const int half = p < C::BNT / 2 ? 0 : 1;
+                  col = n0 + (half ? p - C::BNT / 2 : p);
+                  y = half == i ? 0 : 64;
                 }
-                load(bdst + c * 8192, &maps.lb[i], full_bar(s), col, y);
+                load(bdst + c * 8192, &maps.lb[op], full_bar(s), col, y);
               }
             }
           }

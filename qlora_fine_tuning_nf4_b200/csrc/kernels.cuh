@@ -26,8 +26,8 @@ struct GemmMaps {
   CUtensorMap a[2];       // A operand per segment: bf16 [M, Kseg], box {64,128}, 128B swizzle
   CUtensorMap codes[2];   // NF4 codes (per segment, or gate/up half for MODE_FWD_GLU)
   CUtensorMap absmax[2];  // fp32 absmax, matching codes[]
-  CUtensorMap la[2];      // LoRA left operand(s): bf16 [M, 16], box {16,128}, 32B swizzle
-  CUtensorMap lb[2];      // LoRA right operand(s)
+  CUtensorMap la[3];      // LoRA left operand(s): s*XA or s*G [M, r]
+  CUtensorMap lb[3];      // LoRA right operand(s): B [r, N] (forward) or A [N, r] (backward)
   CUtensorMap b[2];       // staged feed only: the dequantised bf16 weight, matching codes[]
   CUtensorMap out[3];     // staged feed only: outputs (D | E, G, H | dE, dG), box {32,32}, 64B swizzle
 };
@@ -37,8 +37,10 @@ struct GemmArgs {
   int N;        // output columns (MODE_FWD_GLU: h, the width of E/G/H)
   int nkb0;     // 64-wide reduction blocks in segment 0
   int nkb1;     // ... in segment 1 (0 if one segment)
-  int lora;     // number of LoRA operands (0, 1 or 2)
+  int lora;     // number of LoRA operands (0..3; MODE_FWD: 1, chosen per tile by ncut)
   int lora_k16; // staged feed: 16-wide reduction steps per LoRA operand (rank / 16, 1..4)
+  int ncut[2];  // MODE_FWD, staged feed: output columns [0, ncut0) take LoRA operand 0,
+                // [ncut0, ncut1) operand 1, the rest operand 2 (fused projections); 0 = no cut
   int act;      // Act
   int ldo;      // leading dimension (elements) of all outputs / epilogue inputs
   bf16* D;      // EPI_STORE output [M, N]

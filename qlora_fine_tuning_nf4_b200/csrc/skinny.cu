@@ -149,6 +149,7 @@ template <int RW, int NF, bool BT>
 __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_v0,
                                                              const __grid_constant__ CUtensorMap tmap_v1,
+                                                             const __grid_constant__ CUtensorMap tmap_v2,
                                                              const __grid_constant__ ReduceJob job, int nkc,
                                                              int* status) {
   using F = FTile<RW>;
@@ -180,8 +181,8 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
           for (int f = 0; f < NF; ++f)
 #pragma unroll
             for (int sub = 0; sub < RW / F::SUBW; ++sub)
-              tma_load_2d(st + T_TILE + f * V_TILE + sub * F::SUB_BYTES, f ? &tmap_v1 : &tmap_v0, fb,
-                          sub * F::SUBW, kc * 64);
+              tma_load_2d(st + T_TILE + f * V_TILE + sub * F::SUB_BYTES,
+                          f == 0 ? &tmap_v0 : (f == 1 ? &tmap_v1 : &tmap_v2), fb, sub * F::SUBW, kc * 64);
         }
       });
     return;
@@ -441,24 +442,27 @@ static int sk_smem(int stage) { return SK_STAGES * stage + 2 * SK_STAGES * 8 + 1
 
 template <int RW, int NF, bool BT>
 static cudaError_t launch_rowproj_t(const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
-                                    const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
+                                    const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
+                                    cudaStream_t st) {
   const int vt = BT ? RW * 128 : FTile<RW>::BYTES;
   const int smem = sk_smem(T_TILE + NF * vt);
   auto k = rowproj_kernel<RW, NF, BT>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
-  k<<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, job, nkc, status);
+  k<<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, v2, job, nkc, status);
   return cudaGetLastError();
 }
 
-// rank rw in {16, 32, 64}; nf factors (1 or 2), or bt: one factor given as B [rw, K]
+// rank rw in {16, 32, 64}; nf factors (1 to 3), or bt: one factor given as B [rw, K]
 cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
-                           const CUtensorMap& v1, const ReduceJob& job, int nkc, int* status, cudaStream_t st) {
+                           const CUtensorMap& v1, const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
+                           cudaStream_t st) {
 #define QL_ROW(RW_)                                                                              \
   if (rw == RW_) {                                                                               \
-    if (bt) return launch_rowproj_t<RW_, 1, true>(t, v0, v1, job, nkc, status, st);              \
-    if (nf == 1) return launch_rowproj_t<RW_, 1, false>(t, v0, v1, job, nkc, status, st);        \
-    return launch_rowproj_t<RW_, 2, false>(t, v0, v1, job, nkc, status, st);                     \
+    if (bt) return launch_rowproj_t<RW_, 1, true>(t, v0, v1, v2, job, nkc, status, st);          \
+    if (nf == 1) return launch_rowproj_t<RW_, 1, false>(t, v0, v1, v2, job, nkc, status, st);    \
+    if (nf == 2) return launch_rowproj_t<RW_, 2, false>(t, v0, v1, v2, job, nkc, status, st);    \
+    return launch_rowproj_t<RW_, 3, false>(t, v0, v1, v2, job, nkc, status, st);                 \
   }
   QL_ROW(16)
   QL_ROW(32)

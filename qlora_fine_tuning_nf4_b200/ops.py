@@ -87,6 +87,13 @@ _SIGS = {
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_qkv_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 5 + [ctypes.c_int32]),
+    "qlora_qkv_fwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear)] * 3 + [ctypes.c_void_p, ctypes.c_int64,
+                                                                             ctypes.c_void_p, ctypes.c_void_p,
+                                                                             ctypes.c_void_p, ctypes.c_size_t,
+                                                                             ctypes.c_void_p]),
+    "qlora_qkv_bwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear)] * 3 + [ctypes.c_void_p] * 3 +
+                      [ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_linear16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                                          ctypes.c_int32]),
     "qlora_mlp16_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
@@ -364,6 +371,42 @@ def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, sa
 def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, saved, dY, ws: Workspace,
                     grads=None):
     return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
+
+
+def qlora_qkv_workspace_bytes(M, K, nq, nk, nv, r=16):
+    return int(lib().qlora_qkv_workspace_bytes(M, K, nq, nk, nv, r))
+
+
+def qlora_qkv_fwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, ws: Workspace, Y=None, XA=None):
+    """Fused Q/K/V projection: Y = [Y_q | Y_k | Y_v] [M, nq + nk + nv], XA = [XA_q | XA_k | XA_v] [M, 3r]."""
+    M, K = X.shape
+    r = q.A.shape[1]
+    nt = q.w.n_out + k.w.n_out + v.w.n_out
+    if Y is None:
+        Y = torch.empty(M, nt, dtype=torch.bfloat16, device=X.device)
+    if XA is None:
+        XA = torch.empty(M, 3 * r, dtype=torch.bfloat16, device=X.device)
+    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
+    cq, ck, cv = q.c(), k.c(), v.c()
+    _check("qlora_qkv_fwd", lib().qlora_qkv_fwd(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv), _p(X), M,
+                                                _p(Y), _p(XA), _p(buf), buf.numel(), _stream()))
+    return Y, XA
+
+
+def qlora_qkv_bwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, XA, dY, ws: Workspace, grads=None):
+    M, K = X.shape
+    r = q.A.shape[1]
+    if grads is None:
+        grads = {"dX": torch.empty(M, K, dtype=torch.bfloat16, device=X.device)}
+        for n, l in (("q", q), ("k", k), ("v", v)):
+            grads["dA_" + n] = torch.empty_like(l.A)
+            grads["dB_" + n] = torch.empty_like(l.B)
+    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
+    cq, ck, cv = q.c(), k.c(), v.c()
+    outs = [_p(grads[n]) for n in ("dX", "dA_q", "dB_q", "dA_k", "dB_k", "dA_v", "dB_v")]
+    _check("qlora_qkv_bwd", lib().qlora_qkv_bwd(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv), _p(X), _p(XA),
+                                                _p(dY), M, *outs, _p(buf), buf.numel(), _stream()))
+    return grads
 
 
 # ------------------------------------------------------------ utilities ----

@@ -85,3 +85,21 @@ def make_mlp_problem(M, d, h, r=16, alpha=16.0, seed=0):
         "s": float(alpha) / float(r),
         "M": M, "d": d, "h": h, "r": r,
     }
+
+
+def make_qkv_problem(M, K, nq, nk, nv, r=16, alpha=16.0, seed=0):
+    """Fused Q/K/V projections of one input: X [M,K]; W_p [n_p,K], A_p [K,r],
+    B_p [r,n_p] for p in q, k, v; dY [M, nq+nk+nv] (bf16 bits).
+
+    Child order: X, W_q, W_k, W_v, A_q, A_k, A_v, B_q, B_k, B_v, dY.
+    """
+    ch = [np.random.default_rng(c) for c in np.random.SeedSequence(seed).spawn(11)]
+    n = {"q": nq, "k": nk, "v": nv}
+    out = {"X": _normal(ch[0], (M, K))}
+    for i, p in enumerate("qkv"):
+        out["W_" + p] = _normal(ch[1 + i], (n[p], K), 0.02)
+        out["A_" + p] = _uniform(ch[4 + i], (K, r), 1.0 / np.sqrt(K))
+        out["B_" + p] = _normal(ch[7 + i], (r, n[p]), 0.02)
+    out["dY"] = _normal(ch[10], (M, nq + nk + nv))
+    out.update({"s": float(alpha) / float(r), "M": M, "K": K, "nq": nq, "nk": nk, "nv": nv, "r": r})
+    return out

@@ -16,10 +16,14 @@ LINEAR_WORKLOADS = {
     "gemma7b_q_proj": dict(M=16384, K=3072, N=4096, r=16, alpha=16.0, seed=1),
 }
 
+# nq / nkv: the same models' attention projection widths (q, and each of k and v;
+# Mistral's grouped-query k/v are 1024 wide), for the fused Q/K/V projection.
 MLP_WORKLOADS = {
-    "llama7b_swiglu_mlp": dict(M=8192, d=4096, h=11008, r=16, alpha=16.0, act="swiglu", seed=0),
-    "mistral7b_swiglu_mlp": dict(M=8192, d=4096, h=14336, r=16, alpha=16.0, act="swiglu", seed=0),
-    "gemma7b_geglu_mlp": dict(M=16384, d=3072, h=24576, r=16, alpha=16.0, act="geglu_tanh", seed=0),
+    "llama7b_swiglu_mlp": dict(M=8192, d=4096, h=11008, r=16, alpha=16.0, act="swiglu", seed=0, nq=4096, nkv=4096),
+    "mistral7b_swiglu_mlp": dict(M=8192, d=4096, h=14336, r=16, alpha=16.0, act="swiglu", seed=0, nq=4096,
+                                 nkv=1024),
+    "gemma7b_geglu_mlp": dict(M=16384, d=3072, h=24576, r=16, alpha=16.0, act="geglu_tanh", seed=0, nq=4096,
+                              nkv=4096),
 }
 
 
