@@ -21,7 +21,8 @@ Sources (web pages on Unsloth's QLoRA kernels; cited by title and section):
   approximation); the thread links the QLoRA paper (arXiv 2305.14314) for the
   NormalFloat format.
 * [Reddit talk]  "探索让 LLM 训练加速的神奇技巧" (r/LocalLLaMA talk summary):
-  kernel list items 链式矩阵乘法, 融合LoRA, SwiGLU.
+  kernel list items 链式矩阵乘法, 融合LoRA, SwiGLU, RMS Layernorm.
+* [Gemma blog] "+1 to RMS LayerNorm" (the (1 + w) gain of Gemma).
 
 The pages do not print the NF4 codebook, the block size or the absmax type;
 the oracle takes the QLoRA NormalFloat construction (block 64, fp32 absmax,
@@ -42,11 +43,12 @@ from .nf4 import (NF4_BLOCK, nf4_codebook, nf4_dequantize, nf4_midpoints,
 from .lora import (ACTIVATIONS, act_fwd, act_grad, linear_bwd, linear_fwd,
                    mlp_bwd, mlp_fwd)
 from .cost import bracket_costs, bracket_speedup_limit
+from .norm import rmsnorm_bwd, rmsnorm_fwd
 
 __all__ = [
     "bf16_bits_to_f64", "f32_to_bf16_bits", "f64_to_f32",
     "NF4_BLOCK", "nf4_codebook", "nf4_midpoints", "nf4_quantize",
     "nf4_quantize_bruteforce", "nf4_dequantize",
     "ACTIVATIONS", "act_fwd", "act_grad", "linear_fwd", "linear_bwd",
-    "mlp_fwd", "mlp_bwd", "bracket_costs", "bracket_speedup_limit",
+    "mlp_fwd", "mlp_bwd", "bracket_costs", "bracket_speedup_limit", "rmsnorm_fwd", "rmsnorm_bwd",
 ]
