@@ -44,8 +44,9 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
-    ap.add_argument("--op", default="mlp", choices=["mlp", "qkv"],
-                    help="the timed step: the gated MLP (the metric) or the fused Q/K/V projection (GQA widths)")
+    ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "qkv"],
+                    help="the timed step: the gated MLP (the metric), the MLP behind its RMS layer norm (norm "
+                         "forward and backward added), or the fused Q/K/V projection (GQA widths)")
     ap.add_argument("--rank", type=int, default=0, choices=[0, 16, 32, 64],
                     help="LoRA rank (0 = the workload's, 16); s = alpha / r with alpha = the rank")
     ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
@@ -281,6 +282,34 @@ def setup_mlp(args, wl, M, d, h, r, act, rank, world, dev):
     return X, dY, Y, grads, flat, step, mlp_flops(M, d, h, r), kflops, dq, ws, {"h": h, "act": act}
 
 
+def setup_norm_mlp(args, wl, M, d, h, r, act, rank, world, dev):
+    """The MLP behind its RMS layer norm: X -> norm -> MLP fwd + bwd -> norm backward (frozen gain)."""
+    import torch
+
+    from qlora_fine_tuning_nf4_b200 import ops
+
+    Xn, dY, Y, grads, flat, mlp_step, flop, kflops, dq, ws, extra = setup_mlp(args, wl, M, d, h, r, act, rank,
+                                                                              world, dev)
+    gemma = act == "geglu_tanh"
+    g = torch.Generator(device="cpu").manual_seed(wl["seed"] + 77)
+    w = (torch.randn(d, generator=g) * 0.1 + (0.0 if gemma else 1.0)).to(torch.bfloat16).to(dev)
+    X = Xn.clone()  # the norm's input (the MLP's own input buffer receives the normalised rows)
+    rstd = torch.empty(M, dtype=torch.float32, device=dev)
+    dXn = grads["dX"]
+    dX = torch.empty_like(X)
+    eps = 1e-6 if gemma else 1e-5
+    out = dict(grads)
+    out["dX"] = dX
+
+    def step():
+        ops.qlora_rmsnorm_fwd(X, w, eps, plus_one=gemma, Y=Xn, rstd=rstd)
+        mlp_step()
+        ops.qlora_rmsnorm_bwd(X, w, rstd, dXn, plus_one=gemma, dX=dX)
+
+    extra = dict(extra, norm="rms, gain 1 + w" if gemma else "rms, gain w")
+    return X, dY, Y, out, flat, step, flop, kflops, dq, ws, extra
+
+
 def setup_qkv(args, wl, M, d, r, rank, world, dev):
     """Tensors and step of the fused Q/K/V projection fwd + bwd at the workload's attention widths."""
     import torch
@@ -342,9 +371,14 @@ def run_ours(args, wl):
     ops.lib()
     ops.qlora_set_tile_config(args.tiles)
     M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
+    norm_step_bytes = 0
     if args.op == "qkv":
         (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
             setup_qkv(args, wl, M, d, r, rank, world, dev)
+    elif args.op == "norm_mlp":
+        (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
+            setup_norm_mlp(args, wl, M, d, h, r, act, rank, world, dev)
+        norm_step_bytes = 10 * M * d  # forward reads X, writes Xn; backward reads X and dXn, writes dX
     else:
         (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
             setup_mlp(args, wl, M, d, h, r, act, rank, world, dev)
@@ -446,6 +480,13 @@ def run_ours(args, wl):
         dq = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
               "launches": n_l, "ms_per_step": tot / args.steps}
 
+    nrm = None
+    if norm_step_bytes and "rmsnorm_fwd" in trace:
+        tot = trace["rmsnorm_fwd"][1] + trace["rmsnorm_bwd"][1]
+        gbs = args.steps * norm_step_bytes / (tot / 1e3) / 1e9
+        nrm = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+               "ms_per_step": tot / args.steps}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "mlp":
         rows = 512
@@ -472,6 +513,7 @@ def run_ours(args, wl):
         "gpu_launches": launches,
         "roofline": roof,
         "dequant": dq,
+        "norm": nrm,
         "kernels": kernels,
         "cpu_baseline": cpu,
         "clocks": clocks,

@@ -234,6 +234,20 @@ QLORA_API qlora_status qlora_qkv_bwd(const qlora_lora_linear* q, const qlora_lor
                                      qlora_bf16* dB_q, qlora_bf16* dA_k, qlora_bf16* dB_k, qlora_bf16* dA_v,
                                      qlora_bf16* dB_v, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* RMS layer norm of X [M, d] (the step before the MLP; Mistral blog item
+ * "8. 快速 RMS Layernorm", Gemma blog "+1 to RMS LayerNorm"):
+ *   rstd = 1 / sqrt(mean_j x_j^2 + eps),  Y = X * rstd * g,
+ *   g = w (plus_one = 0: Llama, Mistral) or 1 + w (plus_one = 1: Gemma).
+ * Y [M, d] bf16; rstd [M] fp32 is kept for the backward.  Statistics in fp32.
+ * Requires d % 8 == 0 and 16-byte aligned pointers. */
+QLORA_API qlora_status qlora_rmsnorm_fwd(const qlora_bf16* X, const qlora_bf16* w, int64_t M, int64_t d, float eps,
+                                         int32_t plus_one, qlora_bf16* Y, float* rstd, qlora_stream_t stream);
+/* Its backward with the norm weight frozen: from dY [M, d] (the gradient of Y),
+ *   dX = rstd * (g * dY - n * mean_j(n_j g_j dY_j)),  n = X * rstd. */
+QLORA_API qlora_status qlora_rmsnorm_bwd(const qlora_bf16* X, const qlora_bf16* w, const float* rstd,
+                                         const qlora_bf16* dY, int64_t M, int64_t d, int32_t plus_one,
+                                         qlora_bf16* dX, qlora_stream_t stream);
+
 /* Reads the device status word in `workspace` (synchronising `stream`),
  * clears it, and maps it to a status: QLORA_OK, QLORA_ERR_TIMEOUT or
  * QLORA_ERR_DEVICE. */

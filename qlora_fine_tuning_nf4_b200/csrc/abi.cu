@@ -32,6 +32,10 @@ cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, co
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
 cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st);
+cudaError_t launch_rmsnorm_fwd(const bf16* X, const bf16* w, int M, int d, float eps, int plus_one, bf16* Y,
+                               float* rstd, cudaStream_t st);
+cudaError_t launch_rmsnorm_bwd(const bf16* X, const bf16* w, const float* rstd, const bf16* dY, int M, int d,
+                               int plus_one, bf16* dX, cudaStream_t st);
 extern const uint32_t h_nf4_bits[16];
 }  // namespace ql
 
@@ -42,11 +46,11 @@ namespace {
 // ------------------------------------------------------------- tracing ---
 enum KernelId : int {
   K_QUANT = 0, K_DEQUANT, K_GEMM_FWD, K_GEMM_GLU_FWD, K_GEMM_BWD, K_GEMM_GLU_BWD, K_ROWPROJ, K_COLPROJ, K_DYPASS,
-  K_REDUCE, K_COUNT
+  K_REDUCE, K_NORM_FWD, K_NORM_BWD, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "nf4_quantize", "nf4_dequantize", "gemm_nf4_fwd", "gemm_nf4_gateup_glu_fwd", "gemm_nf4_bwd_dx",
-    "gemm_nf4_down_bwd_glu", "skinny_rowproj", "skinny_colproj", "skinny_dypass", "skinny_reduce"};
+    "gemm_nf4_down_bwd_glu", "skinny_rowproj", "skinny_colproj", "skinny_dypass", "skinny_reduce", "rmsnorm_fwd", "rmsnorm_bwd"};
 
 std::atomic<uint64_t> g_launches{0};
 bool g_trace = false;
@@ -1105,6 +1109,35 @@ qlora_status qlora_qkv_bwd(const qlora_lora_linear* q_, const qlora_lora_linear*
     if (s != QLORA_OK) return s;
   }
   return QLORA_OK;
+}
+
+// ---------------------------------------------------------------- norm ----
+qlora_status qlora_rmsnorm_fwd(const qlora_bf16* X, const qlora_bf16* w, int64_t M, int64_t d, float eps,
+                               int32_t plus_one, qlora_bf16* Y, float* rstd, qlora_stream_t stream) {
+  if (M < 0 || d <= 0 || !(eps >= 0.f)) return QLORA_ERR_INVALID_ARG;
+  if (d % 8 || d > (1 << 30) || M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return QLORA_OK;
+  if (!X || !w || !Y || !rstd) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(w) || misaligned(Y) || misaligned(rstd)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  KScope k(K_NORM_FWD, st);
+  return cuda_status(launch_rmsnorm_fwd(reinterpret_cast<const bf16*>(X), reinterpret_cast<const bf16*>(w), (int)M,
+                                        (int)d, eps, plus_one ? 1 : 0, reinterpret_cast<bf16*>(Y), rstd, st));
+}
+
+qlora_status qlora_rmsnorm_bwd(const qlora_bf16* X, const qlora_bf16* w, const float* rstd, const qlora_bf16* dY,
+                               int64_t M, int64_t d, int32_t plus_one, qlora_bf16* dX, qlora_stream_t stream) {
+  if (M < 0 || d <= 0) return QLORA_ERR_INVALID_ARG;
+  if (d % 8 || d > (1 << 30) || M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return QLORA_OK;
+  if (!X || !w || !rstd || !dY || !dX) return QLORA_ERR_INVALID_ARG;
+  if (misaligned(X) || misaligned(w) || misaligned(rstd) || misaligned(dY) || misaligned(dX))
+    return QLORA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  KScope k(K_NORM_BWD, st);
+  return cuda_status(launch_rmsnorm_bwd(reinterpret_cast<const bf16*>(X), reinterpret_cast<const bf16*>(w), rstd,
+                                        reinterpret_cast<const bf16*>(dY), (int)M, (int)d, plus_one ? 1 : 0,
+                                        reinterpret_cast<bf16*>(dX), st));
 }
 
 // NF4 entry points: the current tile configuration.

@@ -87,6 +87,11 @@ _SIGS = {
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_rmsnorm_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_float, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p]),
+    "qlora_rmsnorm_bwd": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                                                 ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_qkv_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64] * 5 + [ctypes.c_int32]),
     "qlora_qkv_fwd": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear)] * 3 + [ctypes.c_void_p, ctypes.c_int64,
                                                                              ctypes.c_void_p, ctypes.c_void_p,
@@ -371,6 +376,27 @@ def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, sa
 def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, saved, dY, ws: Workspace,
                     grads=None):
     return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
+
+
+def qlora_rmsnorm_fwd(X, w, eps, plus_one=False, Y=None, rstd=None):
+    """RMS layer norm of X [M, d] with gain w (or 1 + w): returns (Y, rstd)."""
+    M, d = X.shape
+    if Y is None:
+        Y = torch.empty_like(X)
+    if rstd is None:
+        rstd = torch.empty(M, dtype=torch.float32, device=X.device)
+    _check("qlora_rmsnorm_fwd", lib().qlora_rmsnorm_fwd(_p(X), _p(w), M, d, float(eps), int(bool(plus_one)), _p(Y),
+                                                        _p(rstd), _stream()))
+    return Y, rstd
+
+
+def qlora_rmsnorm_bwd(X, w, rstd, dY, plus_one=False, dX=None):
+    M, d = X.shape
+    if dX is None:
+        dX = torch.empty_like(X)
+    _check("qlora_rmsnorm_bwd", lib().qlora_rmsnorm_bwd(_p(X), _p(w), _p(rstd), _p(dY), M, d, int(bool(plus_one)),
+                                                        _p(dX), _stream()))
+    return dX
 
 
 def qlora_qkv_workspace_bytes(M, K, nq, nk, nv, r=16):
