@@ -237,6 +237,8 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
   if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_holder);
+  grid_dep_wait();  // the previous kernel's outputs (this kernel's inputs) are complete
+  grid_dep_launch();
 
   // shared::cluster address of a barrier in the pair's leader CTA
   auto leader = [&](uint32_t bar) { return (CG == 2) ? mapa_shared(bar, 0) : bar; };
@@ -795,13 +797,15 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaSt
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!resident[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);

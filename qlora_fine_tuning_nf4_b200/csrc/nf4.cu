@@ -27,6 +27,8 @@ const uint32_t h_nf4_bits[16] = {0xbf800000u, 0xbf3239b1u, 0xbf066b2eu, 0xbeca32
 // v, so a value on a midpoint takes the lower level; absmax 0 -> level 7.
 __global__ void nf4_quantize_kernel(const bf16* __restrict__ w, int64_t nblocks, uint8_t* __restrict__ codes,
                                     float* __restrict__ absmax) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (blk >= nblocks) return;
@@ -69,6 +71,8 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, con
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = __uint_as_float(c_nf4_bits[threadIdx.x]);
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t total = j0.runs + j1.runs;
@@ -100,8 +104,8 @@ cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, fl
   const int64_t nblocks = numel / 64;
   const int64_t threads = nblocks * 32;
   const int64_t grid = (threads + 255) / 256;
-  nf4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(w, nblocks, codes, absmax);
-  return cudaGetLastError();
+  return launch_pdl(nf4_quantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, w, nblocks, codes,
+                    absmax);
 }
 
 // Dequantises one tensor, or two (codes1 != nullptr) in the same launch.
@@ -114,8 +118,7 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, i
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 CTAs of 256 threads per SM
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  nf4_dequantize_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(j0, j1);
-  return cudaGetLastError();
+  return launch_pdl(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, j0, j1);
 }
 
 }  // namespace ql

@@ -43,6 +43,14 @@ QL_DEV void cluster_sync() {
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------ dependent launches ---
+// Every kernel of the library is launched with programmatic stream
+// serialisation: it may start while the previous kernel in the stream is still
+// draining, so it waits here for that kernel's completion (and memory) before
+// touching global data, and lets the next kernel start launching right away.
+QL_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QL_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------- mbarrier ---
 QL_DEV void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

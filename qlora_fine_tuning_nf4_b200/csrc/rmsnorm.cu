@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(32 * NORM_WARPS) rmsnorm_fwd_kernel(const bf16
                                                                       const bf16* __restrict__ w, int M, int d,
                                                                       float eps, int plus_one, bf16* __restrict__ Y,
                                                                       float* __restrict__ rstd_out) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * NORM_WARPS + (threadIdx.x >> 5);
   if (row >= M) return;
@@ -74,6 +76,8 @@ __global__ void __launch_bounds__(32 * NORM_WARPS) rmsnorm_bwd_kernel(const bf16
                                                                       const float* __restrict__ rstd_in,
                                                                       const bf16* __restrict__ dY, int M, int d,
                                                                       int plus_one, bf16* __restrict__ dX) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * NORM_WARPS + (threadIdx.x >> 5);
   if (row >= M) return;
@@ -127,6 +131,8 @@ __global__ void __launch_bounds__(NR_THREADS) rmsnorm_fwd_row_kernel(const bf16*
                                                                      const bf16* __restrict__ w, int d, float eps,
                                                                      int plus_one, bf16* __restrict__ Y,
                                                                      float* __restrict__ rstd_out) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float red[4];
   const int row = blockIdx.x;
   const bf16* x = X + static_cast<size_t>(row) * d;
@@ -169,6 +175,8 @@ __global__ void __launch_bounds__(NR_THREADS) rmsnorm_bwd_row_kernel(const bf16*
                                                                      const float* __restrict__ rstd_in,
                                                                      const bf16* __restrict__ dY, int d, int plus_one,
                                                                      bf16* __restrict__ dX) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ float red[4];
   const int row = blockIdx.x;
   const size_t off = static_cast<size_t>(row) * d;
@@ -217,23 +225,19 @@ __global__ void __launch_bounds__(NR_THREADS) rmsnorm_bwd_row_kernel(const bf16*
 cudaError_t launch_rmsnorm_fwd(const bf16* X, const bf16* w, int M, int d, float eps, int plus_one, bf16* Y,
                                float* rstd, cudaStream_t st) {
   if (d <= NR_THREADS * NR_MAXCH * 8) {
-    rmsnorm_fwd_row_kernel<<<M, NR_THREADS, 0, st>>>(X, w, d, eps, plus_one, Y, rstd);
-    return cudaGetLastError();
+    return launch_pdl(rmsnorm_fwd_row_kernel, dim3(M), dim3(NR_THREADS), 0, st, X, w, d, eps, plus_one, Y, rstd);
   }
-  rmsnorm_fwd_kernel<<<(M + NORM_WARPS - 1) / NORM_WARPS, 32 * NORM_WARPS, 0, st>>>(X, w, M, d, eps, plus_one, Y,
-                                                                                    rstd);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_fwd_kernel, dim3((M + NORM_WARPS - 1) / NORM_WARPS), dim3(32 * NORM_WARPS), 0, st, X, w,
+                    M, d, eps, plus_one, Y, rstd);
 }
 
 cudaError_t launch_rmsnorm_bwd(const bf16* X, const bf16* w, const float* rstd, const bf16* dY, int M, int d,
                                int plus_one, bf16* dX, cudaStream_t st) {
   if (d <= NR_THREADS * NR_MAXCH * 8) {
-    rmsnorm_bwd_row_kernel<<<M, NR_THREADS, 0, st>>>(X, w, rstd, dY, d, plus_one, dX);
-    return cudaGetLastError();
+    return launch_pdl(rmsnorm_bwd_row_kernel, dim3(M), dim3(NR_THREADS), 0, st, X, w, rstd, dY, d, plus_one, dX);
   }
-  rmsnorm_bwd_kernel<<<(M + NORM_WARPS - 1) / NORM_WARPS, 32 * NORM_WARPS, 0, st>>>(X, w, rstd, dY, M, d, plus_one,
-                                                                                    dX);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_bwd_kernel, dim3((M + NORM_WARPS - 1) / NORM_WARPS), dim3(32 * NORM_WARPS), 0, st, X, w,
+                    rstd, dY, M, d, plus_one, dX);
 }
 
 }  // namespace ql

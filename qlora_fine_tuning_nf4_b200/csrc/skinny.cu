@@ -91,6 +91,8 @@ QL_DEV void sk_init(uint32_t bars) {
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dep_wait();
+  grid_dep_launch();
 }
 
 // Producer (one thread): issue(i, s, full_bar) loads tile i of the CTA's range
@@ -381,6 +383,8 @@ struct ReduceJobs {
   int n0, n1;  // float4 elements (rows * R / 4) of each job
 };
 __global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ ReduceJobs js) {
+  grid_dep_wait();
+  grid_dep_launch();
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
   const int k = idx < js.n0 ? 0 : 1;
   if (k == 1) idx -= js.n0;
@@ -395,15 +399,15 @@ __global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ Red
   for (int s = 0; s < ns; s += 16) {
     float4 v[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      if (s + q < ns) v[q] = __ldg(reinterpret_cast<const float4*>(p + (s + q) * slot_stride));
+    for (int t = 0; t < 16; ++t)
+      if (s + t < ns) v[t] = __ldg(reinterpret_cast<const float4*>(p + (s + t) * slot_stride));
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      if (s + q < ns) {
-        acc.x += v[q].x;
-        acc.y += v[q].y;
-        acc.z += v[q].z;
-        acc.w += v[q].w;
+    for (int t = 0; t < 16; ++t) {
+      if (s + t < ns) {
+        acc.x += v[t].x;
+        acc.y += v[t].y;
+        acc.z += v[t].z;
+        acc.w += v[t].w;
       }
     }
   }
@@ -449,8 +453,7 @@ static cudaError_t launch_rowproj_t(const CUtensorMap& t, const CUtensorMap& v0,
   auto k = rowproj_kernel<RW, NF, BT>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
-  k<<<job.sp.P, SK_THREADS, smem, st>>>(t, v0, v1, v2, job, nkc, status);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, v0, v1, v2, job, nkc, status);
 }
 
 // rank rw in {16, 32, 64}; nf factors (1 to 3), or bt: one factor given as B [rw, K]
@@ -477,8 +480,7 @@ static cudaError_t launch_colproj_t(const CUtensorMap& t, const CUtensorMap& u, 
   const int smem = sk_smem(T_TILE + FTile<R>::BYTES);
   cudaError_t e = set_smem((const void*)colproj_kernel<R>, smem);
   if (e != cudaSuccess) return e;
-  colproj_kernel<R><<<job.sp.P, SK_THREADS, smem, st>>>(t, u, job, nmc, status);
-  return cudaGetLastError();
+  return launch_pdl(colproj_kernel<R>, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, u, job, nmc, status);
 }
 
 // R in {16, 32, 64, 128}
@@ -496,8 +498,7 @@ cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUte
   const int smem = sk_smem(T_TILE + 2048 + 2048);
   cudaError_t e = set_smem((const void*)dypass_kernel, smem);
   if (e != cudaSuccess) return e;
-  dypass_kernel<<<qjob.sp.P, SK_THREADS, smem, st>>>(t, u, b, gjob, qjob, nch, status);
-  return cudaGetLastError();
+  return launch_pdl(dypass_kernel, dim3(qjob.sp.P), dim3(SK_THREADS), smem, st, t, u, b, gjob, qjob, nch, status);
 }
 
 cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st) {
@@ -510,8 +511,7 @@ cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t
     js.n1 = j1->rows * j1->R / 4;
   }
   const int n = js.n0 + js.n1;
-  reduce_kernel<<<(n + 255) / 256, 256, 0, st>>>(js);
-  return cudaGetLastError();
+  return launch_pdl(reduce_kernel, dim3((n + 255) / 256), dim3(256), 0, st, js);
 }
 
 }  // namespace ql
