@@ -488,6 +488,27 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
     const int lg = warp & 3;            // TMEM lane quadrant this warp may access
     const int half = ew >> 2;           // which half of the tile's column chunks
     const int row = lg * 32 + lane;
+    // Staged gated backward: the saved e, g of this warp's next 32 x 32 chunk
+    // are requested one chunk ahead (across tile boundaries too), so their
+    // latency hides behind the current chunk and the wait for the next
+    // accumulator.
+    uint4 ec[4], gc[4];
+    auto fetch_eg = [&](int t_, int it_) {
+      int mb_, n0_;
+      tile_coords(t_, mb_, n0_);
+      constexpr int CPH = C::BNT / 32;
+      const int grow_ = half_row(mb_, it_ / CPH) + row;
+      const bool row_ok = grow_ < args.M;
+      const size_t rbase = static_cast<size_t>(row_ok ? grow_ : 0) * args.ldo;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = n0_ + (it_ % CPH) * 32 + q * 8;
+        const bool in = row_ok && col < args.N;
+        ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
+        gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    if (ST && EPI == EPI_GLU_BWD && cluster < total_tiles) fetch_eg(cluster, half * 4);
     int tl = 0;
     for (int t = cluster; t < total_tiles; t += clusters, ++tl) {
       int mb, n0;
@@ -514,19 +535,13 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           for (int it = half * 4; it < half * 4 + 4; ++it) {
             const int h = it / CPH, c = it % CPH;
             const int grow0 = half_row(mb, h) + lg * 32;
-            const int grow = grow0 + lane;
             const int col0 = n0 + c * 32;
-            uint4 ec[4], gc[4];
+            uint4 ecur[4], gcur[4];
             if (EPI == EPI_GLU_BWD) {
-              const bool row_ok = grow < args.M;
-              const size_t rbase = static_cast<size_t>(row_ok ? grow : 0) * args.ldo;
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int col = col0 + q * 8;
-                const bool in = row_ok && col < args.N;
-                ec[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Ein + rbase + col)) : make_uint4(0, 0, 0, 0);
-                gc[q] = in ? __ldg(reinterpret_cast<const uint4*>(args.Gin + rbase + col)) : make_uint4(0, 0, 0, 0);
-              }
+              for (int q = 0; q < 4; ++q) ecur[q] = ec[q], gcur[q] = gc[q];
+              if (it + 1 < half * 4 + 4) fetch_eg(t, it + 1);
+              else if (t + clusters < total_tiles) fetch_eg(t + clusters, half * 4);
             }
             float v[32];
             tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, v);
@@ -542,8 +557,8 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
                 o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
                 put(0, q, o);
               } else {
-                const uint32_t ewv[4] = {ec[q].x, ec[q].y, ec[q].z, ec[q].w};
-                const uint32_t gwv[4] = {gc[q].x, gc[q].y, gc[q].z, gc[q].w};
+                const uint32_t ewv[4] = {ecur[q].x, ecur[q].y, ecur[q].z, ecur[q].w};
+                const uint32_t gwv[4] = {gcur[q].x, gcur[q].y, gcur[q].z, gcur[q].w};
                 uint32_t de[4], dg[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
