@@ -28,11 +28,21 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from qlora_fine_tuning_nf4_b200.workloads import MLP_WORKLOADS, mlp_flops  # noqa: E402
+from qlora_fine_tuning_nf4_b200.workloads import LINEAR_WORKLOADS, MLP_WORKLOADS, mlp_flops  # noqa: E402
 
 METRIC = "QLoRA MLP fwd+bwd TFLOP/s & tokens/s (Llama-7B shape), % of bf16 peak"
 UNIT = "TFLOP/s"
-L2_NOTE = "inputs larger than L2 (saved E/G/H and dE/dG are 5 x 172 MiB per step)"
+
+
+def l2_note(op, M, d, h, extra):
+    """How the timed steps avoid running out of a warm L2 (126 MB): every step streams more than that."""
+    mib = lambda n: f"{n * 2 / 2 ** 20:.0f} MiB"
+    if op == "linear":
+        return f"inputs larger than L2 (X and dX {mib(M * d)} each, dY and Y {mib(M * extra['N'])} each per step)"
+    if op == "qkv":
+        nt = extra["nq"] + extra["nk"] + extra["nv"]
+        return f"inputs larger than L2 (X and dX {mib(M * d)} each, dY and Y {mib(M * nt)} each per step)"
+    return f"inputs larger than L2 (saved E/G/H and dE/dG are 5 x {mib(M * h)} per step)"
 
 
 def parse():
@@ -41,12 +51,14 @@ def parse():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS))
+    ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS) + sorted(LINEAR_WORKLOADS),
+                    help="an MLP workload (ops mlp, norm_mlp, qkv) or a single-projection one (op linear)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
-    ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "qkv"],
+    ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "qkv", "linear"],
                     help="the timed step: the gated MLP (the metric), the MLP behind its RMS layer norm (norm "
-                         "forward and backward added), or the fused Q/K/V projection (GQA widths)")
+                         "forward and backward added), the fused Q/K/V projection (GQA widths), or one QLoRA "
+                         "projection (qlora_linear_fwd + qlora_linear_bwd)")
     ap.add_argument("--rank", type=int, default=0, choices=[0, 16, 32, 64],
                     help="LoRA rank (0 = the workload's, 16); s = alpha / r with alpha = the rank")
     ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
@@ -353,6 +365,45 @@ def setup_qkv(args, wl, M, d, r, rank, world, dev):
     return X, dY, Y, grads, flat, step, flop, kflops, dq, ws, {"nq": nq, "nk": nkv, "nv": nkv}
 
 
+def setup_linear(args, wl, rank, world, dev):
+    """Tensors and step of one QLoRA projection fwd + bwd (qlora_linear_fwd / qlora_linear_bwd)."""
+    import torch
+    import torch.distributed as dist
+
+    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_linear_problem
+    from qlora_fine_tuning_nf4_b200.workloads import linear_flops
+
+    M, K, N, r = wl["M"], wl["K"], wl["N"], wl["r"]
+    p = make_linear_problem(M, K, N, r, wl["alpha"], wl["seed"] + 1000 * rank)
+    A, B = bits_to_torch(p["A"], dev), bits_to_torch(p["B"], dev)
+    if args.weights == "nf4":
+        lin = ops.LoraLinear(ops.nf4_quantize(bits_to_torch(p["W"], dev)), A, B, p["s"])
+        fwd, bwd = ops.qlora_linear_fwd, ops.qlora_linear_bwd
+    else:
+        lin = ops.LoraLinear16(bits_to_torch(p["W"], dev), A, B, p["s"])
+        fwd, bwd = ops.qlora_linear16_fwd, ops.qlora_linear16_bwd
+    X = bits_to_torch(p["X"], dev)
+    dY = bits_to_torch(p["dY"], dev)
+    del p
+    ws = ops.Workspace(dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    XA = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    flat = torch.empty(K * r + r * N, dtype=torch.bfloat16, device=dev)
+    grads = {"dA": flat[:K * r].view(K, r), "dB": flat[K * r:].view(r, N),
+             "dX": torch.empty(M, K, dtype=torch.bfloat16, device=dev)}
+
+    def step():
+        fwd(lin, X, ws, Y=Y, XA=XA)
+        bwd(lin, X, XA, dY, ws, dX=grads["dX"], dA=grads["dA"], dB=grads["dB"])
+        if world > 1:
+            dist.all_reduce(flat)
+
+    kflops = {"gemm_nf4_fwd": 2 * M * K * N + 2 * M * r * N, "gemm_nf4_bwd_dx": 2 * M * N * K + 2 * M * r * K}
+    dq = 2 * N * K * (0.5 + 4 / 64 + 2) if args.weights == "nf4" else 0  # the forward's and the backward's
+    return X, dY, Y, grads, flat, step, linear_flops(M, K, N, r), kflops, dq, ws, {"N": N}
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -370,9 +421,13 @@ def run_ours(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     ops.lib()
     ops.qlora_set_tile_config(args.tiles)
-    M, d, h, r, act = wl["M"], wl["d"], wl["h"], wl["r"], wl["act"]
+    M, r = wl["M"], wl["r"]
+    d, h, act = wl.get("d", wl.get("K")), wl.get("h"), wl.get("act")
     norm_step_bytes = 0
-    if args.op == "qkv":
+    if args.op == "linear":
+        (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
+            setup_linear(args, wl, rank, world, dev)
+    elif args.op == "qkv":
         (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
             setup_qkv(args, wl, M, d, r, rank, world, dev)
     elif args.op == "norm_mlp":
@@ -519,7 +574,7 @@ def run_ours(args, wl):
         "config": {"workload": args.workload, "op": args.op, "M_per_gpu": M, "d": d, **cfg_extra, "r": r,
                    "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
                    "gemm_tiles": ops.TILE_CONFIGS[4 if args.weights == "bf16" else args.tiles],
-                   "base_weights": args.weights, "l2": L2_NOTE},
+                   "base_weights": args.weights, "l2": l2_note(args.op, M, d, h, cfg_extra)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": launches,
@@ -534,7 +589,11 @@ def run_ours(args, wl):
 
 def main():
     args = parse()
-    wl = dict(MLP_WORKLOADS[args.workload])
+    if (args.op == "linear") != (args.workload in LINEAR_WORKLOADS):
+        sys.exit(f"--op {args.op} needs {'a single-projection' if args.op == 'linear' else 'an MLP'} workload")
+    if args.op == "linear" and args.impl == "reference":
+        sys.exit("--impl reference times the MLP workloads only")
+    wl = dict(LINEAR_WORKLOADS[args.workload] if args.op == "linear" else MLP_WORKLOADS[args.workload])
     if args.tokens:
         wl["M"] = args.tokens
     if args.rank:
