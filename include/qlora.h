@@ -253,6 +253,17 @@ QLORA_API qlora_status qlora_rmsnorm_bwd(const qlora_bf16* X, const qlora_bf16* 
  * QLORA_ERR_DEVICE. */
 QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t stream);
 
+/* Test hook for the timeout path (synchronous; not needed in normal use).
+ * Arms a one-shot fault: the first CTA of the next skinny pass (the rank-side
+ * products X A, dY B^T, ...) leaves one of its tiles unloaded, so that CTA's
+ * consumers reach their bounded wait (about 4 s), record QLORA_ERR_TIMEOUT in
+ * the status word and return; the kernels after it in the same call see the
+ * status and return early too.  Nothing traps or hangs: every wait is bounded
+ * and every copy already issued lands before its CTA exits.  The call's
+ * results are then meaningless; qlora_last_device_status reports and clears
+ * the timeout, and the next call computes normally. */
+QLORA_API qlora_status qlora_test_inject_timeout(void);
+
 /* Human-readable name of a status code (static string). */
 QLORA_API const char* qlora_status_string(qlora_status status);
 

@@ -31,6 +31,7 @@ cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, co
                            int* status, cudaStream_t st);
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
+cudaError_t arm_inject_timeout();
 cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st);
 cudaError_t launch_rmsnorm_fwd(const bf16* X, const bf16* w, int M, int d, float eps, int plus_one, bf16* Y,
                                float* rstd, cudaStream_t st);
@@ -1212,6 +1213,10 @@ qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16* gate, con
   if (!gate || !up || !down || !gate->w || !up->w || !down->w) return QLORA_ERR_INVALID_ARG;
   const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
   return mlp_bwd(act, &g, &u, &d, 4, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes, stream);
+}
+
+qlora_status qlora_test_inject_timeout(void) {
+  return cuda_status(arm_inject_timeout());
 }
 
 qlora_status qlora_last_device_status(void* ws, qlora_stream_t stream) {

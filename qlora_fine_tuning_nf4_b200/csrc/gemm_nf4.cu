@@ -374,6 +374,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
                    n0 + (int)rank * C::BNC + bx * C::BOXR);
         }
       }
+      if (!ok) settle_inflight();  // loads already issued land before the CTA can exit
     }
   } else if (warp == 2) {
     // ------------------------------------------------ raw-code producer --
@@ -410,6 +411,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           }
         }
       }
+      if (!ok) settle_inflight();
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA -----
@@ -478,9 +480,9 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
         }
         umma_commit<CG>(acc_full0 + 8u * b);
       }
-      // let every issued MMA finish before TMEM can be released
+      // let every issued MMA finish before TMEM can be released (after an error too)
       umma_commit<CG>(drain_bar);
-      mbar_wait(drain_bar, 0, args.status);
+      mbar_drain(drain_bar, 0);
     }
   } else if (warp < C::DQ_WARP0) {
     // ------------------------------------------------------ epilogue -----

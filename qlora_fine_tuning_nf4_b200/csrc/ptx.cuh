@@ -99,6 +99,23 @@ QL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
   }
 }
 
+// Waits used on the way out after an error, for this thread's own operations
+// still in flight.  Unlike mbar_wait they do not give up when the status word
+// already holds a timeout (that is why they run), but they are bounded too.
+QL_DEV void mbar_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 <= QL_WAIT_LIMIT_NS) {
+  }
+}
+// Bounded pause for TMA loads already issued whose completion this thread
+// cannot observe (they complete on a barrier another CTA or role owns).
+constexpr unsigned long long QL_SETTLE_NS = 200000ull;  // 200 us
+QL_DEV void settle_inflight() {
+  const unsigned long long t0 = globaltimer();
+  while (globaltimer() - t0 <= QL_SETTLE_NS) {
+  }
+}
+
 // ------------------------------------------------------------------ TMA ---
 QL_DEV void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -95,19 +95,27 @@ QL_DEV void sk_init(uint32_t bars) {
   grid_dep_launch();
 }
 
+// Test-only fault injection (qlora_test_inject_timeout): when set, the first
+// CTA of the next skinny launch leaves its tile 1 unloaded, so that CTA's
+// consumers run into their bounded wait; the launch clears it (one shot).
+__device__ int g_inject_timeout = 0;
+
 // Producer (one thread): issue(i, s, full_bar) loads tile i of the CTA's range
-// into slot s once the consumers released it; afterwards waits (bounded) until
-// every load it issued has landed, so no copy is in flight when the CTA exits.
+// into slot s once the consumers released it; afterwards waits (bounded, and
+// after an error too) until every load it issued has landed, so no copy is in
+// flight when the CTA exits.
 template <typename Issue>
 QL_DEV void sk_produce(int ntiles, uint32_t bars, int* status, Issue issue) {
+  int skip = -1;
+  if (blockIdx.x == 0 && ntiles > 1 && atomicExch(&g_inject_timeout, 0) != 0) skip = 1;
   int i = 0;
   for (; i < ntiles; ++i) {
     const int s = i % SK_STAGES;
     if (!mbar_wait(sk_empty(bars, s), ((i / SK_STAGES) & 1) ^ 1, status)) break;
-    issue(i, s, sk_full(bars, s));
+    if (i != skip) issue(i, s, sk_full(bars, s));
   }
   for (int j = i > SK_STAGES ? i - SK_STAGES : 0; j < i; ++j)
-    mbar_wait(sk_full(bars, j % SK_STAGES), (j / SK_STAGES) & 1, status);
+    if (j != skip) mbar_drain(sk_full(bars, j % SK_STAGES), (j / SK_STAGES) & 1);
 }
 
 // Consumer side of tile i: wait until it has landed (uniform over the warp).
@@ -499,6 +507,11 @@ cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUte
   cudaError_t e = set_smem((const void*)dypass_kernel, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(dypass_kernel, dim3(qjob.sp.P), dim3(SK_THREADS), smem, st, t, u, b, gjob, qjob, nch, status);
+}
+
+cudaError_t arm_inject_timeout() {
+  const int one = 1;
+  return cudaMemcpyToSymbol(g_inject_timeout, &one, sizeof(one));
 }
 
 cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st) {

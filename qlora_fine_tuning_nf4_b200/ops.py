@@ -80,6 +80,7 @@ _SIGS = {
                                      ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
                                      ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_last_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_test_inject_timeout": (ctypes.c_int, []),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_tile_config": (ctypes.c_int32, [ctypes.c_int32]),
     "qlora_trace_begin": (ctypes.c_int, []),
@@ -436,6 +437,11 @@ def qlora_qkv_bwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, XA, dY, ws: Wo
 
 
 # ------------------------------------------------------------ utilities ----
+
+def qlora_test_inject_timeout():
+    """Arms the library's one-shot timeout injection (test hook; see include/qlora.h)."""
+    _check("qlora_test_inject_timeout", lib().qlora_test_inject_timeout())
+
 
 def qlora_last_device_status(ws: Workspace):
     return int(lib().qlora_last_device_status(_p(ws.buf), _stream()))
