@@ -205,6 +205,29 @@ def oracle_sample(wl, rows, seed_rows=0):
     return dt, mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0))
 
 
+def c_loop_oracle_sample():
+    """Time the plain C loop oracle's projection fwd+bwd on the tiny configuration
+    (256 tokens, 512 -> 1024, rank 16; one thread).  Returns a summary dict."""
+    from oracle import c_oracle
+    from qlora_fine_tuning_nf4_b200.synth import make_linear_problem
+    from qlora_fine_tuning_nf4_b200.workloads import linear_flops
+
+    cfg = LINEAR_WORKLOADS["tiny_linear"]
+    p = make_linear_problem(cfg["M"], cfg["K"], cfg["N"], cfg["r"], cfg["alpha"], cfg["seed"])
+    n, k = p["W"].shape
+    codes, absmax = c_oracle.nf4_quantize(p["W"], n, k)
+    W = c_oracle.nf4_dequantize_f64(codes, absmax, n, k)
+    wide = lambda b: (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+    X, A, B, dY = (wide(p[t]) for t in ("X", "A", "B", "dY"))
+    t0 = time.perf_counter()
+    c_oracle.linear_fwd(X, W, A, B, p["s"])
+    c_oracle.linear_bwd(X, W, A, B, p["s"], dY)
+    dt = time.perf_counter() - t0
+    fl = linear_flops(cfg["M"], cfg["K"], cfg["N"], cfg["r"])
+    return {"workload": "tiny_linear (256 tokens, 512 -> 1024, r 16)", "value": fl / dt / 1e12, "unit": UNIT,
+            "ms": dt * 1e3, "threads": 1, "kind": "C loop oracle, binary64"}
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -616,7 +639,8 @@ def run_ours(args, wl):
         rows = 512
         dt, fl, cores = oracle_sample(wl, rows)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"{rows} of {M} token rows, one fwd+bwd (fp64 numpy, {dt:.1f} s)"}
+               "sample": f"{rows} of {M} token rows, one fwd+bwd (fp64 numpy, {dt:.1f} s)",
+               "c_loop_oracle": c_loop_oracle_sample()}
 
     if world > 1:
         dist.destroy_process_group()

@@ -1,6 +1,7 @@
 """Plain, slow, fp64 CPU oracle for the QLoRA NF4 projection and gated MLP.
 
-TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the ``libqlora``
+TEST INFRASTRUCTURE ONLY.  (``oracle/c/`` restates the tiny configuration in
+plain C loops; ``oracle/c_oracle.py`` binds it.)  Nothing in the product path (the ``libqlora``
 shared library and its Python binding) may import, call or link this package.
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
 legs of ``bench.py`` use it.  It shares no code with the CUDA path: its bf16
