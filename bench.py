@@ -56,10 +56,10 @@ def parse():
                     help="an MLP workload (ops mlp, norm_mlp, qkv) or a single-projection one (op linear)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
-    ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "norm_mlp_fused", "qkv", "linear"],
+    ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "qkv", "linear"],
                     help="the timed step: the gated MLP (the metric), the MLP behind its RMS layer norm (norm "
-                         "forward and backward as their own kernels, or fused into the MLP), the fused Q/K/V "
-                         "projection (GQA widths), or one QLoRA projection (qlora_linear_fwd + qlora_linear_bwd)")
+                         "forward and backward added), the fused Q/K/V projection (GQA widths), or one QLoRA "
+                         "projection (qlora_linear_fwd + qlora_linear_bwd)")
     ap.add_argument("--rank", type=int, default=0, choices=[0, 16, 32, 64],
                     help="LoRA rank (0 = the workload's, 16); s = alpha / r with alpha = the rank")
     ap.add_argument("--weights", default="nf4", choices=["nf4", "bf16"],
@@ -356,49 +356,6 @@ def setup_norm_mlp(args, wl, M, d, h, r, act, rank, world, dev):
     return X, dY, Y, out, flat, step, flop, kflops, dq, ws, extra
 
 
-def setup_norm_mlp_fused(args, wl, M, d, h, r, act, rank, world, dev):
-    """The MLP behind its RMS layer norm, the norm fused into it (qlora_norm_mlp_fwd / _bwd)."""
-    import torch
-    import torch.distributed as dist
-
-    from qlora_fine_tuning_nf4_b200 import ops
-    from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_norm_mlp_problem
-
-    gemma = act == "geglu_tanh"
-    p = make_norm_mlp_problem(M, d, h, r, wl["alpha"], wl["seed"] + 1000 * rank, plus_one=gemma)
-    lins = {k: ops.LoraLinear(ops.nf4_quantize(bits_to_torch(p["W_" + k], dev)), bits_to_torch(p["A_" + k], dev),
-                              bits_to_torch(p["B_" + k], dev), p["s"]) for k in ("g", "u", "d")}
-    X, dY, w = bits_to_torch(p["X"], dev), bits_to_torch(p["dY"], dev), bits_to_torch(p["w"], dev)
-    del p
-    ws = ops.Workspace(dev)
-    saved = ops.make_mlp_saved(M, h, r, dev)
-    Y = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-    rstd = torch.empty(M, dtype=torch.float32, device=dev)
-    sizes = [("dA_g", (d, r)), ("dB_g", (r, h)), ("dA_u", (d, r)), ("dB_u", (r, h)), ("dA_d", (h, r)),
-             ("dB_d", (r, d))]
-    flat = torch.empty(sum(a * b for _, (a, b) in sizes), dtype=torch.bfloat16, device=dev)
-    grads, off = {}, 0
-    for name, (a, b) in sizes:
-        grads[name] = flat[off:off + a * b].view(a, b)
-        off += a * b
-    grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-    eps = 1e-6 if gemma else 1e-5
-
-    def step():
-        ops.qlora_norm_mlp_fwd(act, w, eps, lins["g"], lins["u"], lins["d"], X, ws, plus_one=gemma, Y=Y,
-                               saved=saved, rstd=rstd)
-        ops.qlora_norm_mlp_bwd(act, w, lins["g"], lins["u"], lins["d"], X, saved, rstd, dY, ws, plus_one=gemma,
-                               grads=grads)
-        if world > 1:
-            dist.all_reduce(flat)
-
-    kflops = {k: kernel_flops(k, M, d, h, r) for k in ("gemm_nf4_gateup_glu_fwd", "gemm_nf4_fwd",
-                                                         "gemm_nf4_down_bwd_glu", "gemm_nf4_bwd_dx")}
-    dq = 2 * (2 * h * d + h * d) * (0.5 + 4 / 64 + 2)
-    extra = {"h": h, "act": act, "norm": ("rms, gain 1 + w" if gemma else "rms, gain w") + ", fused into the MLP"}
-    return X, dY, Y, grads, flat, step, mlp_flops(M, d, h, r), kflops, dq, ws, extra
-
-
 def setup_qkv(args, wl, M, d, r, rank, world, dev):
     """Tensors and step of the fused Q/K/V projection fwd + bwd at the workload's attention widths."""
     import torch
@@ -507,9 +464,6 @@ def run_ours(args, wl):
     elif args.op == "qkv":
         (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
             setup_qkv(args, wl, M, d, r, rank, world, dev)
-    elif args.op == "norm_mlp_fused":
-        (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
-            setup_norm_mlp_fused(args, wl, M, d, h, r, act, rank, world, dev)
     elif args.op == "norm_mlp":
         (X, dY, Y, grads, flat, step, flop_step, kflops, dq_step_bytes, ws, cfg_extra) = \
             setup_norm_mlp(args, wl, M, d, h, r, act, rank, world, dev)

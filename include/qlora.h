@@ -253,38 +253,6 @@ QLORA_API qlora_status qlora_rmsnorm_bwd(const qlora_bf16* X, const qlora_bf16* 
  * QLORA_ERR_DEVICE. */
 QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t stream);
 
-/* RMS layer norm fused into the gated MLP behind it (Mistral blog "8. 快速 RMS
- * Layernorm"; Gemma blog "+1 to RMS LayerNorm"): the MLP of qlora_mlp_fwd
- * applied to Xn = rmsnorm(X), rstd = 1 / sqrt(mean_j X_j^2 + eps), gain
- * g = w (plus_one = 0) or 1 + w (plus_one = 1), the norm weight frozen.
- * Xn is never written: g is folded into the staged gate/up weights and A
- * factors (W diag(g), diag(g) A, one bf16 rounding of the binary32 product),
- * the X A pass also gathers the rows' sums of squares, and the gate/up GEMM's
- * epilogue scales each row by rstd.  saved->XA_g / XA_u hold Xn A as in
- * qlora_mlp_fwd on Xn; rstd [M] (fp32) is written for the backward.  Needs
- * NF4 weights under tile configuration 4 (QLORA_ERR_UNSUPPORTED_SHAPE
- * otherwise); norm_w [d] bf16, 16-byte aligned.  Results match the unfused
- * norm + MLP up to where the roundings fall (the gain is rounded into the
- * weights instead of into Xn). */
-QLORA_API size_t qlora_norm_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r);
-QLORA_API qlora_status qlora_norm_mlp_fwd(qlora_act act, const qlora_bf16* norm_w, float eps, int32_t plus_one,
-                                          const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                                          const qlora_lora_linear* down, const qlora_bf16* X, int64_t M,
-                                          qlora_bf16* Y, const qlora_mlp_saved* saved, float* rstd,
-                                          void* workspace, size_t workspace_bytes, qlora_stream_t stream);
-/* Its backward: the gradients of qlora_mlp_bwd, with dX the gradient with
- * respect to X (the norm's input).  The dX GEMM runs on the gained weights
- * and factors, so it yields g * dXn, and the norm's backward then needs no
- * gain: dX = rstd * (g dXn - n * mean_j(n_j g_j dXn_j)), n = X * rstd;
- * dA_g = diag(g) X^T (rstd s_g G_g) (likewise for up). */
-QLORA_API qlora_status qlora_norm_mlp_bwd(qlora_act act, const qlora_bf16* norm_w, int32_t plus_one,
-                                          const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                                          const qlora_lora_linear* down, const qlora_bf16* X,
-                                          const qlora_mlp_saved* saved, const float* rstd, const qlora_bf16* dY,
-                                          int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
-                                          qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
-                                          void* workspace, size_t workspace_bytes, qlora_stream_t stream);
-
 /* Test hook for the timeout path (synchronous; not needed in normal use).
  * Arms a one-shot fault: the first CTA of the next skinny pass (the rank-side
  * products X A, dY B^T, ...) leaves one of its tiles unloaded, so that CTA's

@@ -20,7 +20,7 @@ namespace ql {
 cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st);
 cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
                                   const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
-                                  cudaStream_t st, int num_sms, const bf16* colgain, int plus_one, int k_in);
+                                  cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
 int gemm_nf4_b_cols_per_cta(int tiles);
@@ -32,8 +32,6 @@ cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, co
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
 cudaError_t arm_inject_timeout();
-cudaError_t launch_gain_rows(const bf16* A0, const bf16* A1, const bf16* w, int plus_one, int rows, int r, bf16* out0,
-                             bf16* out1, cudaStream_t st);
 cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st);
 cudaError_t launch_rmsnorm_fwd(const bf16* X, const bf16* w, int M, int d, float eps, int plus_one, bf16* Y,
                                float* rstd, cudaStream_t st);
@@ -49,12 +47,11 @@ namespace {
 // ------------------------------------------------------------- tracing ---
 enum KernelId : int {
   K_QUANT = 0, K_DEQUANT, K_GEMM_FWD, K_GEMM_GLU_FWD, K_GEMM_BWD, K_GEMM_GLU_BWD, K_ROWPROJ, K_COLPROJ, K_DYPASS,
-  K_REDUCE, K_NORM_FWD, K_NORM_BWD, K_NORM_GAIN, K_COUNT
+  K_REDUCE, K_NORM_FWD, K_NORM_BWD, K_COUNT
 };
 const char* const kKernelNames[K_COUNT] = {
     "nf4_quantize", "nf4_dequantize", "gemm_nf4_fwd", "gemm_nf4_gateup_glu_fwd", "gemm_nf4_bwd_dx",
-    "gemm_nf4_down_bwd_glu", "skinny_rowproj", "skinny_colproj", "skinny_dypass", "skinny_reduce", "rmsnorm_fwd", "rmsnorm_bwd",
-    "norm_gain_factor"};
+    "gemm_nf4_down_bwd_glu", "skinny_rowproj", "skinny_colproj", "skinny_dypass", "skinny_reduce", "rmsnorm_fwd", "rmsnorm_bwd"};
 
 std::atomic<uint64_t> g_launches{0};
 bool g_trace = false;
@@ -259,16 +256,8 @@ bool map_factor(CUtensorMap* m, const void* p, int64_t rows, int cols, int64_t l
 }
 
 // P = T V (V = up to three [K, r] LoRA A factors side by side) -> outs (bf16, optional scaled copies)
-// Fused RMS norm over the rows of T (rowproj with two factors): partial sums of
-// squares, the statistic's width and epsilon, and where rstd goes.
-struct NormStat {
-  float* ss_part;
-  float d, eps;
-  float* rstd_out;
-};
 qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, int r, float* part,
-                          ReduceOuts outs, int* status, cudaStream_t st, const bf16* V2 = nullptr,
-                          const NormStat* ns = nullptr) {
+                          ReduceOuts outs, int* status, cudaStream_t st, const bf16* V2 = nullptr) {
   CUtensorMap mt, mv0, mv1, mv2;
   const int nv = V2 ? 3 : (V1 ? 2 : 1);
   if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -277,13 +266,7 @@ qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, c
   if (!map_factor(&mv2, V2 ? V2 : V0, K, r, r)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_rowproj(M, K, nv * r);
   const int64_t nrc = cdiv(M, 64);
-  ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, p.slot_cap, 0, p.sp, outs);
-  if (ns) {
-    j.ss_part = ns->ss_part;
-    j.ss_d = ns->d;
-    j.ss_eps = ns->eps;
-    j.rstd_out = ns->rstd_out;
-  }
+  const ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, p.slot_cap, 0, p.sp, outs);
   {
     KScope k(K_ROWPROJ, st);
     const qlora_status s =
@@ -366,21 +349,7 @@ qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, con
 // One reduction output: columns [col0, col0 + width) of the partials, scaled, bf16
 // into p (row stride ld, or transposed).
 ReduceOut rout(bf16* p, int col0, int width, int ld, int transpose, float scale) {
-  return {p, col0, width, ld, transpose, scale, 0, nullptr, nullptr, 0};
-}
-// ... times the job's rstd / a per-row binary32 factor / a per-row gain (w or 1 + w)
-ReduceOut by_rstd(ReduceOut o) {
-  o.by_rstd = 1;
-  return o;
-}
-ReduceOut row_scaled(ReduceOut o, const float* f) {
-  o.rscale = f;
-  return o;
-}
-ReduceOut row_gained(ReduceOut o, const bf16* w, int plus_one) {
-  o.gain = w;
-  o.gain_plus_one = plus_one;
-  return o;
+  return {p, col0, width, ld, transpose, scale};
 }
 ReduceOuts routs(ReduceOut a, ReduceOut b = {nullptr, 0, 0, 0, 0, 0.f}, ReduceOut c = {nullptr, 0, 0, 0, 0, 0.f},
                  ReduceOut d = {nullptr, 0, 0, 0, 0, 0.f}) {
@@ -422,14 +391,12 @@ bool map_staged(CUtensorMap* m, const void* wq, const Wt& w, bool bwd, int bnc) 
   if (!bwd) return map_bf16(m, wq, K, N, K, 64, bnc < 128 ? bnc : 128, CU_TENSOR_MAP_SWIZZLE_128B);
   return map_bf16(m, wq, K, N, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// Dequantises one weight (w1 == nullptr) or two in one launch into their staging buffers,
-// optionally with a gain per input feature folded in (both weights then share k_in).
-qlora_status stage_weights(const Wt& w0, bf16* dst0, const Wt* w1, bf16* dst1, cudaStream_t st,
-                           const bf16* colgain = nullptr, int plus_one = 0) {
+// Dequantises one weight (w1 == nullptr) or two in one launch into their staging buffers.
+qlora_status stage_weights(const Wt& w0, bf16* dst0, const Wt* w1, bf16* dst1, cudaStream_t st) {
   KScope k(K_DEQUANT, st);
   return cuda_status(launch_nf4_dequantize(w0.codes, w0.absmax, w0.n_out * w0.k_in, dst0, w1 ? w1->codes : nullptr,
                                            w1 ? w1->absmax : nullptr, w1 ? w1->n_out * w1->k_in : 0, dst1, st,
-                                           num_sms(), colgain, plus_one, (int)w0.k_in));
+                                           num_sms()));
 }
 // Output maps of the staged configuration's TMA-store epilogue: bf16 [rows, cols]
 // with row stride ld, written in 32 x 32 boxes (64B swizzle).  No-ops otherwise.
@@ -445,7 +412,7 @@ bool map_outs(GemmMaps& maps, int tiles, int64_t rows, int64_t cols, int64_t ld,
 // either feed; under the staged feed NF4 weights are first dequantised into stage0 / stage1, and
 // bf16 weights are read where they are (they always use the staged feed).
 qlora_status map_weights(GemmMaps& maps, const Wt& w0, const Wt* w1, bool bwd, int tiles, bf16* stage0,
-                         bf16* stage1, cudaStream_t st, bool staged = false) {
+                         bf16* stage1, cudaStream_t st) {
   const int bnc = gemm_nf4_b_cols_per_cta(tiles);
   if (w0.w16) {
     if (!is_staged(tiles) || !map_staged(&maps.b[0], w0.w16, w0, bwd, bnc)) return QLORA_ERR_CUDA;
@@ -453,7 +420,7 @@ qlora_status map_weights(GemmMaps& maps, const Wt& w0, const Wt* w1, bool bwd, i
     return QLORA_OK;
   }
   if (is_staged(tiles)) {
-    const qlora_status s = staged ? QLORA_OK : stage_weights(w0, stage0, w1, stage1, st);
+    const qlora_status s = stage_weights(w0, stage0, w1, stage1, st);
     if (s != QLORA_OK) return s;
     if (!map_staged(&maps.b[0], stage0, w0, bwd, bnc)) return QLORA_ERR_CUDA;
     if (w1 && !map_staged(&maps.b[1], stage1, *w1, bwd, bnc)) return QLORA_ERR_CUDA;
@@ -585,7 +552,7 @@ qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   KScope k(K_DEQUANT, st);
   return cuda_status(launch_nf4_dequantize(codes, absmax, n_out * k_in, reinterpret_cast<bf16*>(out), nullptr, nullptr,
-                                           0, nullptr, st, num_sms(), nullptr, 0, (int)k_in));
+                                           0, nullptr, st, num_sms()));
 }
 
 namespace {
@@ -726,54 +693,6 @@ size_t mlp_ws(int64_t M, int64_t d, int64_t h, int r, bool stage) {
 }
 }  // namespace
 
-namespace {
-// The norm + MLP adds, after the staged MLP's workspace: the norm-gained gate and up A
-// factors [d, r] each, the partial sums of squares of the X pass, rstd-scaled copies of
-// s G_g | s G_u [M, 2r], and the gradient g * dXn before the norm's backward [M, d].
-size_t norm_ss_bytes(int64_t M, int64_t d, int r) {
-  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, d, 2 * r).slot_cap * 64 * 4;
-}
-size_t norm_mlp_ws(int64_t M, int64_t d, int64_t h, int r) {
-  return mlp_ws(M, d, h, r, true) + 2 * align256(static_cast<size_t>(d) * r * 2) + align256(norm_ss_bytes(M, d, r)) +
-         align256(static_cast<size_t>(M) * 2 * r * 2) + align256(static_cast<size_t>(M) * d * 2);
-}
-}  // namespace
-
-size_t qlora_norm_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
-  if (M <= 0 || d <= 0 || h <= 0 || !rank_ok(r, 4)) return 256;
-  return norm_mlp_ws(M, d, h, r);
-}
-
-namespace {
-// The RMS norm in front of the gated MLP, fused into it: the norm's weight and form,
-// rstd (written by the forward, read by the backward) and the extra workspace.
-struct NormCtx {
-  const bf16* w;
-  float eps;
-  int plus_one;
-  float* rstd;
-  bf16 *Ag, *Au;  // diag(gain) A_g, diag(gain) A_u
-  float* ss;      // partial sums of squares
-  bf16* gr;       // rstd * [s G_g | s G_u]
-  bf16* dxg;      // gain * dXn
-};
-void carve_norm(NormCtx& n, void* ws, int64_t M, int64_t d, int64_t h, int r) {
-  char* w = static_cast<char*>(ws) + mlp_ws(M, d, h, r, true);
-  const size_t fa = align256(static_cast<size_t>(d) * r * 2);
-  n.Ag = reinterpret_cast<bf16*>(w);
-  n.Au = reinterpret_cast<bf16*>(w + fa);
-  n.ss = reinterpret_cast<float*>(w + 2 * fa);
-  n.gr = reinterpret_cast<bf16*>(w + 2 * fa + align256(norm_ss_bytes(M, d, r)));
-  n.dxg = reinterpret_cast<bf16*>(w + 2 * fa + align256(norm_ss_bytes(M, d, r)) +
-                                  align256(static_cast<size_t>(M) * 2 * r * 2));
-}
-qlora_status gain_factors(const NormCtx& n, const Lin* gate, const Lin* up, int64_t d, int r, cudaStream_t st) {
-  KScope k(K_NORM_GAIN, st);
-  return cuda_status(launch_gain_rows(reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A),
-                                      n.w, n.plus_one, (int)d, r, n.Ag, n.Au, st));
-}
-}  // namespace
-
 size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int32_t r) {
   if (M <= 0 || d <= 0 || h <= 0 || !rank_ok(r, g_tiles)) return 256;
   return mlp_ws(M, d, h, r, is_staged(g_tiles));
@@ -822,10 +741,9 @@ qlora_status check_mlp(const Lin* g, const Lin* u, const Lin* d, int tiles) {
 }
 }  // namespace
 
-// nc != nullptr: the input first goes through the RMS norm described by nc (staged NF4 feed only).
 static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const Lin* down, int tiles, const qlora_bf16* X,
                      int64_t M, qlora_bf16* Y, const qlora_mlp_saved* sv, void* ws, size_t ws_bytes,
-                     qlora_stream_t stream, NormCtx* nc = nullptr) {
+                     qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
   qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
@@ -840,39 +758,22 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
-  if (nc && !stage) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (ws_bytes < (nc ? norm_mlp_ws(M, d, h, r) : mlp_ws(M, d, h, r, stage))) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < mlp_ws(M, d, h, r, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   MlpWs w = carve_mlp(ws, M, d, h, r, stage);
-  if (nc) carve_norm(*nc, ws, M, d, h, r);
   const bf16* x = reinterpret_cast<const bf16*>(X);
   bf16* xag = reinterpret_cast<bf16*>(sv->XA_g);
   bf16* xau = reinterpret_cast<bf16*>(sv->XA_u);
   bf16* had = reinterpret_cast<bf16*>(sv->HA_d);
-  bf16* xags = gate->scale != 1.f || nc ? w.v0 : xag;
-  bf16* xaus = up->scale != 1.f || nc ? w.v1 : xau;
+  bf16* xags = gate->scale != 1.f ? w.v0 : xag;
+  bf16* xaus = up->scale != 1.f ? w.v1 : xau;
   bf16* hads = down->scale != 1.f ? w.v2 : had;
-  if (!nc) {
-    // XA_g, XA_u = X [A_g | A_u] (one pass over X)
-    s = pass_rowproj(x, M, d, reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A), r,
-                     w.part,
-                     routs(rout(xag, 0, r, r, 0, 1.f), rout(xau, r, r, r, 0, 1.f),
-                           rout(xags != xag ? xags : nullptr, 0, r, r, 0, gate->scale),
-                           rout(xaus != xau ? xaus : nullptr, r, r, r, 0, up->scale)),
-                     w.status, st);
-  } else {
-    // Norm folded in: Xn = diag(rstd) X diag(gain).  One pass over X gives rstd and
-    // P = X [gain A_g | gain A_u]; XA = rstd P is saved (= Xn A), s P feeds the GEMM,
-    // whose epilogue applies rstd to the whole accumulator.
-    if ((s = gain_factors(*nc, gate, up, d, r, st)) != QLORA_OK) return s;
-    const NormStat ns = {nc->ss, static_cast<float>(d), nc->eps, nc->rstd};
-    s = pass_rowproj(x, M, d, nc->Ag, nc->Au, r, w.part,
-                     routs(by_rstd(rout(xag, 0, r, r, 0, 1.f)), by_rstd(rout(xau, r, r, r, 0, 1.f)),
-                           rout(xags, 0, r, r, 0, gate->scale), rout(xaus, r, r, r, 0, up->scale)),
-                     w.status, st, nullptr, &ns);
-    if (s == QLORA_OK)
-      s = stage_weights(gate->w, w.stage0, &up->w, w.stage1, st, nc->w, nc->plus_one);
-  }
+  // XA_g, XA_u = X [A_g | A_u] (one pass over X)
+  s = pass_rowproj(x, M, d, reinterpret_cast<const bf16*>(gate->A), reinterpret_cast<const bf16*>(up->A), r, w.part,
+                   routs(rout(xag, 0, r, r, 0, 1.f), rout(xau, r, r, r, 0, 1.f),
+                         rout(xags != xag ? xags : nullptr, 0, r, r, 0, gate->scale),
+                         rout(xaus != xau ? xaus : nullptr, r, r, r, 0, up->scale)),
+                   w.status, st);
   if (s != QLORA_OK) return s;
   // gate/up GEMM with the gated activation in the epilogue -> E, G, H
   {
@@ -880,8 +781,7 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], x, d, M, d, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     maps.a[1] = maps.a[0];
-    if ((s = map_weights(maps, gate->w, &up->w, false, tiles, w.stage0, w.stage1, st, nc != nullptr)) != QLORA_OK)
-      return s;
+    if ((s = map_weights(maps, gate->w, &up->w, false, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
     if (!map_lora_left(&maps.la[0], xags, M, r, r, tiles)) return QLORA_ERR_CUDA;
     if (!map_lora_left(&maps.la[1], xaus, M, r, r, tiles)) return QLORA_ERR_CUDA;
     if (!map_lora_right(&maps.lb[0], gate->B, h, r, false, tiles)) return QLORA_ERR_CUDA;
@@ -901,7 +801,6 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (!map_outs(maps, tiles, M, h, h, sv->E, sv->G, sv->H)) return QLORA_ERR_CUDA;
     a.status = w.status;
     a.group_m = kGroupM;
-    a.rstd = nc ? nc->rstd : nullptr;
     KScope k(K_GEMM_GLU_FWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_FWD_GLU, EPI_GLU_FWD, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
@@ -916,12 +815,10 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
                   w.stage0, st);
 }
 
-// nc != nullptr: the forward ran the input through the RMS norm described by nc (rstd
-// from that forward); dX is then the gradient with respect to the norm's input.
 static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const Lin* down, int tiles, const qlora_bf16* X,
                      const qlora_mlp_saved* sv, const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g,
                      qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
-                     void* ws, size_t ws_bytes, qlora_stream_t stream, NormCtx* nc = nullptr) {
+                     void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
   qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
@@ -938,11 +835,9 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
-  if (nc && !stage) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (ws_bytes < (nc ? norm_mlp_ws(M, d, h, r) : mlp_ws(M, d, h, r, stage))) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < mlp_ws(M, d, h, r, stage)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   MlpWs w = carve_mlp(ws, M, d, h, r, stage);
-  if (nc) carve_norm(*nc, ws, M, d, h, r);
   bf16* sGd = w.v0;
   // 1. G_d = dY B_d^T (scaled), dB_d = s_d HA_d^T dY
   s = pass_dypass(reinterpret_cast<const bf16*>(dY), M, d, reinterpret_cast<const bf16*>(sv->HA_d),
@@ -988,39 +883,25 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
                    routs(rout(reinterpret_cast<bf16*>(dA_d), 0, r, r, 0, 1.f)), w.status, st);
   if (s != QLORA_OK) return s;
   // 4. G_g = dE B_g^T, dB_g = s_g XA_g^T dE ; G_u = dG B_u^T, dB_u = s_u XA_u^T dG
-  //    (norm folded in: also rstd * s G for the dA pass over the raw input)
-  const ReduceOut gr_g = nc ? row_scaled(rout(nc->gr, 0, r, 2 * r, 0, gate->scale), nc->rstd)
-                            : rout(nullptr, 0, 0, 0, 0, 0.f);
-  const ReduceOut gr_u = nc ? row_scaled(rout(nc->gr + r, 0, r, 2 * r, 0, up->scale), nc->rstd)
-                            : rout(nullptr, 0, 0, 0, 0, 0.f);
   s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), r,
-                  w.part, routs(rout(w.gu, 0, r, 2 * r, 0, gate->scale), gr_g),
+                  w.part, routs(rout(w.gu, 0, r, 2 * r, 0, gate->scale)),
                   routs(rout(reinterpret_cast<bf16*>(dB_g), 0, r, (int)h, 1, gate->scale)), w.status, st);
   if (s != QLORA_OK) return s;
   s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), r,
-                  w.part, routs(rout(w.gu + r, 0, r, 2 * r, 0, up->scale), gr_u),
+                  w.part, routs(rout(w.gu + r, 0, r, 2 * r, 0, up->scale)),
                   routs(rout(reinterpret_cast<bf16*>(dB_u), 0, r, (int)h, 1, up->scale)), w.status, st);
   if (s != QLORA_OK) return s;
-  // Norm folded in: the dX GEMM runs on the gained weights and A factors, so it yields
-  // gain * dXn, which is what the norm's backward takes (with unit gain).
-  if (nc) {
-    if ((s = gain_factors(*nc, gate, up, d, r, st)) != QLORA_OK) return s;
-    if ((s = stage_weights(gate->w, w.stage0, &up->w, w.stage1, st, nc->w, nc->plus_one)) != QLORA_OK) return s;
-  }
   // 5. dX = [dE | dG] [W_g ; W_u] + [sG_g | sG_u] [A_g^T ; A_u^T]
   {
     GemmMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_bf16(&maps.a[0], w.dE, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
     if (!map_bf16(&maps.a[1], w.dG, h, M, h, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
-    if ((s = map_weights(maps, gate->w, &up->w, true, tiles, w.stage0, w.stage1, st, nc != nullptr)) != QLORA_OK)
-      return s;
+    if ((s = map_weights(maps, gate->w, &up->w, true, tiles, w.stage0, w.stage1, st)) != QLORA_OK) return s;
     if (!map_lora_left(&maps.la[0], w.gu, M, r, 2 * r, tiles)) return QLORA_ERR_CUDA;
     if (!map_lora_left(&maps.la[1], w.gu + r, M, r, 2 * r, tiles)) return QLORA_ERR_CUDA;
-    if (!map_lora_right(&maps.lb[0], nc ? static_cast<const void*>(nc->Ag) : gate->A, d, r, true, tiles))
-      return QLORA_ERR_CUDA;
-    if (!map_lora_right(&maps.lb[1], nc ? static_cast<const void*>(nc->Au) : up->A, d, r, true, tiles))
-      return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[0], gate->A, d, r, true, tiles)) return QLORA_ERR_CUDA;
+    if (!map_lora_right(&maps.lb[1], up->A, d, r, true, tiles)) return QLORA_ERR_CUDA;
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     a.M = (int)M;
@@ -1030,31 +911,19 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     a.lora = 2;
     a.lora_k16 = r / 16;
     a.ldo = (int)d;
-    bf16* dxo = nc ? nc->dxg : reinterpret_cast<bf16*>(dX);
-    a.D = dxo;
-    if (!map_outs(maps, tiles, M, d, d, dxo)) return QLORA_ERR_CUDA;
+    a.D = reinterpret_cast<bf16*>(dX);
+    if (!map_outs(maps, tiles, M, d, d, dX)) return QLORA_ERR_CUDA;
     a.status = w.status;
     a.group_m = kGroupM;
     KScope k(K_GEMM_BWD, st);
     s = cuda_status(launch_gemm_nf4(MODE_BWD, EPI_STORE, tiles, maps, a, st));
     if (s != QLORA_OK) return s;
   }
-  // 6. [dA_g | dA_u] = X^T [sG_g | sG_u]; norm folded in: Xn^T = diag(gain) X^T diag(rstd),
-  //    so diag(gain) X^T (rstd [sG_g | sG_u])
-  if (!nc)
-    return pass_colproj(reinterpret_cast<const bf16*>(X), M, d, w.gu, 2 * r, w.part,
-                        routs(rout(reinterpret_cast<bf16*>(dA_g), 0, r, r, 0, 1.f),
-                              rout(reinterpret_cast<bf16*>(dA_u), r, r, r, 0, 1.f)),
-                        w.status, st);
-  s = pass_colproj(reinterpret_cast<const bf16*>(X), M, d, nc->gr, 2 * r, w.part,
-                   routs(row_gained(rout(reinterpret_cast<bf16*>(dA_g), 0, r, r, 0, 1.f), nc->w, nc->plus_one),
-                         row_gained(rout(reinterpret_cast<bf16*>(dA_u), r, r, r, 0, 1.f), nc->w, nc->plus_one)),
-                   w.status, st);
-  if (s != QLORA_OK) return s;
-  // 7. the norm's backward with unit gain on gain * dXn
-  KScope k(K_NORM_BWD, st);
-  return cuda_status(launch_rmsnorm_bwd(reinterpret_cast<const bf16*>(X), nullptr, nc->rstd, nc->dxg, (int)M, (int)d,
-                                        0, reinterpret_cast<bf16*>(dX), st));
+  // 6. [dA_g | dA_u] = X^T [sG_g | sG_u]
+  return pass_colproj(reinterpret_cast<const bf16*>(X), M, d, w.gu, 2 * r, w.part,
+                      routs(rout(reinterpret_cast<bf16*>(dA_g), 0, r, r, 0, 1.f),
+                            rout(reinterpret_cast<bf16*>(dA_u), r, r, r, 0, 1.f)),
+                      w.status, st);
 }
 
 // ------------------------------------------------------------ fused QKV --
@@ -1302,44 +1171,6 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
   const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
   return mlp_bwd(act, &g, &u, &d, g_tiles, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes,
                  stream);
-}
-
-// RMS norm + gated MLP, the norm fused into the MLP (staged NF4 feed).
-qlora_status qlora_norm_mlp_fwd(qlora_act act, const qlora_bf16* norm_w, float eps, int32_t plus_one,
-                                const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                                const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
-                                const qlora_mlp_saved* sv, float* rstd, void* ws, size_t ws_bytes,
-                                qlora_stream_t stream) {
-  if (!gate || !up || !down || !norm_w || !(eps >= 0.f)) return QLORA_ERR_INVALID_ARG;
-  if (M > 0 && !rstd) return QLORA_ERR_INVALID_ARG;
-  if (misaligned(norm_w) || misaligned(rstd)) return QLORA_ERR_MISALIGNED;
-  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
-  if (g.w.w16 || !is_staged(g_tiles)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  NormCtx nc = {};
-  nc.w = reinterpret_cast<const bf16*>(norm_w);
-  nc.eps = eps;
-  nc.plus_one = plus_one ? 1 : 0;
-  nc.rstd = rstd;
-  return mlp_fwd(act, &g, &u, &d, g_tiles, X, M, Y, sv, ws, ws_bytes, stream, &nc);
-}
-qlora_status qlora_norm_mlp_bwd(qlora_act act, const qlora_bf16* norm_w, int32_t plus_one,
-                                const qlora_lora_linear* gate, const qlora_lora_linear* up,
-                                const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
-                                const float* rstd, const qlora_bf16* dY, int64_t M, qlora_bf16* dX,
-                                qlora_bf16* dA_g, qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u,
-                                qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws, size_t ws_bytes,
-                                qlora_stream_t stream) {
-  if (!gate || !up || !down || !norm_w) return QLORA_ERR_INVALID_ARG;
-  if (M > 0 && !rstd) return QLORA_ERR_INVALID_ARG;
-  if (misaligned(norm_w) || misaligned(rstd)) return QLORA_ERR_MISALIGNED;
-  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
-  if (g.w.w16 || !is_staged(g_tiles)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  NormCtx nc = {};
-  nc.w = reinterpret_cast<const bf16*>(norm_w);
-  nc.plus_one = plus_one ? 1 : 0;
-  nc.rstd = const_cast<float*>(rstd);  // read only in the backward
-  return mlp_bwd(act, &g, &u, &d, g_tiles, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes,
-                 stream, &nc);
 }
 
 // 16-bit entry points: bf16 base weights, always the staged-feed pair tile

@@ -595,15 +595,6 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
             float e[32], g[32];
             tmem_ld_32x32b_x32(tacc + h * C::BNT + c * 32, e);
             tmem_ld_32x32b_x32(tacc + h * C::BNT + C::BNT / 2 + c * 32, g);
-            if (args.rstd != nullptr) {  // fused RMS norm: the A operand was the raw input row
-              const int grow = grow0 + lane;
-              const float rs = grow < args.M ? __ldg(args.rstd + grow) : 0.f;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                e[i] *= rs;
-                g[i] *= rs;
-              }
-            }
             if (lane == 0) bulk_wait_group_read<0>();
             __syncwarp();
 #pragma unroll

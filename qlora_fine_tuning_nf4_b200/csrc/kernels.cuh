@@ -53,7 +53,6 @@ struct GemmArgs {
   bf16* dG;
   int* status;  // device status word (timeouts)
   int group_m;  // tile order: groups of group_m output-row tiles, rows fastest inside a group (>= 1)
-  const float* rstd;  // EPI_GLU_FWD, staged feed: per-row factor of the accumulator (fused RMS norm), or nullptr
 };
 
 // --------------------------------------------------------------- skinny ---
@@ -94,13 +93,6 @@ struct ReduceOut {
   int ld;         // row stride of the destination (elements)
   int transpose;  // 0: dst[row * ld + c], 1: dst[c * ld + row]
   float scale;
-  // Optional per-row factors (row = the partials' row index), applied in binary32
-  // before the one bf16 rounding: the job's rstd (by_rstd), rscale[row], and
-  // gain[row] (+ 1 if gain_plus_one).
-  int by_rstd;
-  const float* rscale;
-  const bf16* gain;
-  int gain_plus_one;
 };
 struct ReduceOuts {
   ReduceOut o[4];
@@ -115,13 +107,6 @@ struct ReduceJob {
   int groups, grows, rows, R, slot_cap, nslots;
   SkPart sp;
   ReduceOuts outs;
-  // Fused RMS norm (rowproj over the norm's input): ss_part[g][slot][row in group]
-  // holds partial row sums of squares; the reduction forms
-  // rstd = 1 / sqrt(sum / ss_d + ss_eps), stores it to rstd_out and offers it to
-  // the outputs (by_rstd).  ss_part == nullptr: no norm.
-  float* ss_part;
-  float ss_d, ss_eps;
-  float* rstd_out;
 };
 
 // Launch with programmatic stream serialisation (the kernel calls

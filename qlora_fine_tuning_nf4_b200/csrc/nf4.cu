@@ -66,11 +66,6 @@ struct DqJob {
   bf16* out;
   int64_t runs;  // numel / 1024, rounded up
   int64_t numel;
-  // Optional gain per input feature (column), folded in before the one bf16
-  // rounding: out[n, k] = bf16(level * absmax * gain[k]), gain = g or 1 + g.
-  const bf16* colgain;
-  int plus_one;
-  int k_in;
 };
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, const DqJob j1) {
   __shared__ float lut[16];
@@ -88,42 +83,19 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, con
     const float* absmax = second ? j1.absmax : j0.absmax;
     bf16* out = second ? j1.out : j0.out;
     const int64_t numel = second ? j1.numel : j0.numel;
-    const DqJob& jb = second ? j1 : j0;
-    if (jb.colgain == nullptr) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t e = base + i * 256 + lane * 8;
-        if (e >= numel) break;
-        const uint32_t c = __ldg(reinterpret_cast<const uint32_t*>(codes + (e >> 1)));
-        const float a = __ldg(absmax + (e >> 6));
-        uint32_t o[4];
+    for (int i = 0; i < 4; ++i) {
+      const int64_t e = base + i * 256 + lane * 8;
+      if (e >= numel) break;
+      const uint32_t c = __ldg(reinterpret_cast<const uint32_t*>(codes + (e >> 1)));
+      const float a = __ldg(absmax + (e >> 6));
+      uint32_t o[4];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t byte = (c >> (8 * b)) & 0xFFu;
-          o[b] = pack_bf16x2(lut[byte >> 4] * a, lut[byte & 0xF] * a);
-        }
-        *reinterpret_cast<uint4*>(out + e) = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t byte = (c >> (8 * b)) & 0xFFu;
+        o[b] = pack_bf16x2(lut[byte >> 4] * a, lut[byte & 0xF] * a);
       }
-    } else {
-      for (int i = 0; i < 4; ++i) {
-        const int64_t e = base + i * 256 + lane * 8;
-        if (e >= numel) break;
-        const uint32_t c = __ldg(reinterpret_cast<const uint32_t*>(codes + (e >> 1)));
-        const float a = __ldg(absmax + (e >> 6));
-        // the 8 elements share a row (k_in % 64 == 0): gains k .. k + 7
-        const uint4 gw = __ldg(reinterpret_cast<const uint4*>(jb.colgain + e % jb.k_in));
-        const uint32_t gv[4] = {gw.x, gw.y, gw.z, gw.w};
-        const float one = jb.plus_one ? 1.0f : 0.0f;
-        uint32_t o[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t byte = (c >> (8 * b)) & 0xFFu;
-          // element 2b is the high nibble (even index), 2b + 1 the low one
-          o[b] = pack_bf16x2((lut[byte >> 4] * a) * (bf16_lo(gv[b]) + one),
-                             (lut[byte & 0xF] * a) * (bf16_hi(gv[b]) + one));
-        }
-        *reinterpret_cast<uint4*>(out + e) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+      *reinterpret_cast<uint4*>(out + e) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
@@ -139,10 +111,9 @@ cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, fl
 // Dequantises one tensor, or two (codes1 != nullptr) in the same launch.
 cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
                                   const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
-                                  cudaStream_t st, int num_sms, const bf16* colgain, int plus_one, int k_in) {
-  DqJob j0 = {codes0, absmax0, out0, (numel0 + 1023) / 1024, numel0, colgain, plus_one, k_in};
-  DqJob j1 = {codes1, absmax1, out1, codes1 ? (numel1 + 1023) / 1024 : 0, codes1 ? numel1 : 0, colgain, plus_one,
-              k_in};
+                                  cudaStream_t st, int num_sms) {
+  DqJob j0 = {codes0, absmax0, out0, (numel0 + 1023) / 1024, numel0};
+  DqJob j1 = {codes1, absmax1, out1, codes1 ? (numel1 + 1023) / 1024 : 0, codes1 ? numel1 : 0};
   int64_t grid = (j0.runs + j1.runs + 7) / 8;             // one run per warp, 8 warps per CTA
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 CTAs of 256 threads per SM
   if (grid > cap) grid = cap;

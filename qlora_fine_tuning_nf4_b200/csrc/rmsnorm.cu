@@ -27,14 +27,7 @@ QL_DEV void unpack8(const uint4& u, float (&f)[8]) {
     f[2 * i + 1] = bf16_hi(w[i]);
   }
 }
-// Gains of columns c .. c + 7: w or 1 + w; w == nullptr means unit gain (the
-// fused norm + MLP backward, whose incoming gradient already carries the gain).
 QL_DEV void gain8(const bf16* w, int c, int plus_one, float (&g)[8]) {
-  if (w == nullptr) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] = 1.0f;
-    return;
-  }
   unpack8(__ldg(reinterpret_cast<const uint4*>(w + c)), g);
   if (plus_one) {
 #pragma unroll
@@ -245,38 +238,6 @@ cudaError_t launch_rmsnorm_bwd(const bf16* X, const bf16* w, const float* rstd, 
   }
   return launch_pdl(rmsnorm_bwd_kernel, dim3((M + NORM_WARPS - 1) / NORM_WARPS), dim3(32 * NORM_WARPS), 0, st, X, w,
                     rstd, dY, M, d, plus_one, dX);
-}
-
-// out[k, :] = gain_k * A[k, :] for a rank-side factor A [rows, r] (bf16, one
-// rounding of the binary32 product), gain = w or 1 + w: the LoRA factor seen
-// through the norm's gain, diag(g) A, for the fused norm + MLP.
-__global__ void __launch_bounds__(256) gain_rows_kernel(const bf16* __restrict__ A0, const bf16* __restrict__ A1,
-                                                         const bf16* __restrict__ w, int plus_one, int rows, int r,
-                                                         bf16* __restrict__ out0, bf16* __restrict__ out1) {
-  grid_dep_wait();
-  grid_dep_launch();
-  const int per = rows * r / 8;  // 8 elements per thread; r % 8 == 0
-  int i = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool second = i >= per;
-  if (second) i -= per;
-  if (i >= per || (second && A1 == nullptr)) return;
-  const int row = (i * 8) / r;
-  const float g = __bfloat162float(w[row]) + (plus_one ? 1.0f : 0.0f);
-  float f[8];
-  unpack8(__ldg(reinterpret_cast<const uint4*>((second ? A1 : A0) + static_cast<size_t>(i) * 8)), f);
-  uint4 o;
-  o.x = pack_bf16x2(f[0] * g, f[1] * g);
-  o.y = pack_bf16x2(f[2] * g, f[3] * g);
-  o.z = pack_bf16x2(f[4] * g, f[5] * g);
-  o.w = pack_bf16x2(f[6] * g, f[7] * g);
-  *reinterpret_cast<uint4*>((second ? out1 : out0) + static_cast<size_t>(i) * 8) = o;
-}
-
-cudaError_t launch_gain_rows(const bf16* A0, const bf16* A1, const bf16* w, int plus_one, int rows, int r, bf16* out0,
-                             bf16* out1, cudaStream_t st) {
-  const int n = (A1 ? 2 : 1) * rows * r / 8;
-  return launch_pdl(gain_rows_kernel, dim3((n + 255) / 256), dim3(256), 0, st, A0, A1, w, plus_one, rows, r, out0,
-                    out1);
 }
 
 }  // namespace ql

@@ -154,11 +154,8 @@ QL_DEV void store_acc(float* base, int ld, int r0, int lane, float (&acc)[NB][4]
 // Units: 64x64 tiles (rc, kc), kc fastest; group = row block rc (nkc units).
 // job.part[rc][slot][64][NF * RW]: T V over the CTA's tiles of row block rc,
 // V = NF factors of RW columns side by side.  BT: the single factor is given
-// transposed, as the LoRA right factor B [RW, K] (G = T B^T).  SS: also the
-// rows' sums of squares (the fused RMS norm's statistic), as the diagonal of
-// T T^T from one more pair of MMAs per 16-wide step on the tile already in
-// shared memory, into job.ss_part[rc][slot][64].
-template <int RW, int NF, bool BT, bool SS>
+// transposed, as the LoRA right factor B [RW, K] (G = T B^T).
+template <int RW, int NF, bool BT>
 __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_v0,
                                                              const __grid_constant__ CUtensorMap tmap_v1,
@@ -201,7 +198,6 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
     return;
   }
   float acc[R / 8][4] = {};
-  float ss[2][4] = {};  // SS: T_w T_w^T for the warp's 16 rows, column blocks of 8
   bool ok = true;
   for (int i = 0; i < nt; ++i) {
     const int t = t0 + i, rc = t / nkc, kc = t % nkc;
@@ -221,34 +217,12 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
             frag_b_kn_f<RW>(tb + T_TILE + (nb / (RW / 8)) * V_TILE, kk * 16, (nb % (RW / 8)) * 8, lane, b);
           mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
         }
-        if (SS) {
-#pragma unroll
-          for (int nb = 0; nb < 2; ++nb) {
-            uint32_t b[2];
-            frag_b_nk(tb, kk * 16, warp * 16 + nb * 8, lane, b);  // the same rows, as columns
-            mma_bf16_16816(ss[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
-          }
-        }
       }
       sk_release(bars, i, lane);
     }
     if (kc == nkc - 1 || i == nt - 1) {
       const int slot = c - sk_first(job.sp, rc);
       store_acc(job.part + static_cast<size_t>(rc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
-      if (SS) {
-        // Diagonal of the two 16 x 8 blocks: row q (0..7) sits in lane 4q + q/2, as
-        // element q & 1 of block 0 (row q) and element 2 + (q & 1) of block 1 (row q + 8).
-        const int q = lane >> 2;
-        if ((lane & 3) == (q >> 1)) {
-          float* d = job.ss_part + static_cast<size_t>(rc * job.slot_cap + slot) * 64 + warp * 16;
-          d[q] = ss[0][q & 1];
-          d[q + 8] = ss[1][2 + (q & 1)];
-        }
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) ss[nb][x] = 0.f;
-      }
     }
   }
 }
@@ -445,25 +419,13 @@ __global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ Red
       }
     }
   }
-  float rstd = 1.f;
-  if (j.ss_part != nullptr) {  // fused RMS norm: this row's statistic, from its slots in the same order
-    const float* ps = j.ss_part + static_cast<size_t>(g) * j.slot_cap * j.grows + r;
-    float ss = 0.f;
-    for (int s = 0; s < ns; ++s) ss += __ldg(ps + static_cast<size_t>(s) * j.grows);
-    rstd = __fdiv_rn(1.0f, sqrtf(__fdiv_rn(ss, j.ss_d) + j.ss_eps));
-    if (c == 0 && j.rstd_out != nullptr && row < j.rows) j.rstd_out[row] = rstd;
-  }
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const ReduceOut& o = j.outs.o[q];
     if (o.ptr == nullptr || c < o.col0 || c >= o.col0 + o.width) continue;
     const int cc = c - o.col0;
-    float f = o.scale;
-    if (o.by_rstd) f *= rstd;
-    if (o.rscale != nullptr) f *= __ldg(o.rscale + row);
-    if (o.gain != nullptr) f *= __bfloat162float(o.gain[row]) + (o.gain_plus_one ? 1.0f : 0.0f);
-    const bf16 b0 = __float2bfloat16_rn(f * acc.x), b1 = __float2bfloat16_rn(f * acc.y);
-    const bf16 b2 = __float2bfloat16_rn(f * acc.z), b3 = __float2bfloat16_rn(f * acc.w);
+    const bf16 b0 = __float2bfloat16_rn(o.scale * acc.x), b1 = __float2bfloat16_rn(o.scale * acc.y);
+    const bf16 b2 = __float2bfloat16_rn(o.scale * acc.z), b3 = __float2bfloat16_rn(o.scale * acc.w);
     if (o.transpose) {
       bf16* d = o.ptr + static_cast<size_t>(cc) * o.ld + row;
       d[0] = b0;
@@ -490,27 +452,24 @@ static cudaError_t set_smem(const void* f, int bytes) {
 }
 static int sk_smem(int stage) { return SK_STAGES * stage + 2 * SK_STAGES * 8 + 1024; }
 
-template <int RW, int NF, bool BT, bool SS = false>
+template <int RW, int NF, bool BT>
 static cudaError_t launch_rowproj_t(const CUtensorMap& t, const CUtensorMap& v0, const CUtensorMap& v1,
                                     const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
                                     cudaStream_t st) {
   const int vt = BT ? RW * 128 : FTile<RW>::BYTES;
   const int smem = sk_smem(T_TILE + NF * vt);
-  auto k = rowproj_kernel<RW, NF, BT, SS>;
+  auto k = rowproj_kernel<RW, NF, BT>;
   cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, v0, v1, v2, job, nkc, status);
 }
 
-// rank rw in {16, 32, 64}; nf factors (1 to 3), or bt: one factor given as B [rw, K];
-// job.ss_part set: also the rows' sums of squares (two factors only)
+// rank rw in {16, 32, 64}; nf factors (1 to 3), or bt: one factor given as B [rw, K]
 cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
                            const CUtensorMap& v1, const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
                            cudaStream_t st) {
-  if (job.ss_part != nullptr && (bt || nf != 2)) return cudaErrorInvalidValue;
 #define QL_ROW(RW_)                                                                              \
   if (rw == RW_) {                                                                               \
-    if (job.ss_part) return launch_rowproj_t<RW_, 2, false, true>(t, v0, v1, v2, job, nkc, status, st); \
     if (bt) return launch_rowproj_t<RW_, 1, true>(t, v0, v1, v2, job, nkc, status, st);          \
     if (nf == 1) return launch_rowproj_t<RW_, 1, false>(t, v0, v1, v2, job, nkc, status, st);    \
     if (nf == 2) return launch_rowproj_t<RW_, 2, false>(t, v0, v1, v2, job, nkc, status, st);    \

@@ -79,19 +79,6 @@ _SIGS = {
                                      ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
                                      ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
                                      ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
-    "qlora_norm_mlp_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-                                                         ctypes.c_int32]),
-    "qlora_norm_mlp_fwd": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_int32,
-                                          ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
-                                          ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
-                                          ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
-                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
-    "qlora_norm_mlp_bwd": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p, ctypes.c_int32,
-                                          ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
-                                          ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p,
-                                          ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p, ctypes.c_void_p,
-                                          ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t,
-                                                                                    ctypes.c_void_p]),
     "qlora_last_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_test_inject_timeout": (ctypes.c_int, []),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -390,51 +377,6 @@ def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, sa
 def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, saved, dY, ws: Workspace,
                     grads=None):
     return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
-
-
-def qlora_norm_mlp_workspace_bytes(M, d, h, r=16):
-    return int(lib().qlora_norm_mlp_workspace_bytes(M, d, h, r))
-
-
-def qlora_norm_mlp_fwd(act, norm_w, eps, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, ws: Workspace,
-                       plus_one=False, Y=None, saved=None, rstd=None):
-    """RMS norm (gain norm_w, or 1 + norm_w) fused into the gated MLP behind it: returns (Y, saved, rstd)."""
-    M, d = X.shape
-    h = _dims(gate)[0]
-    r = gate.A.shape[1]
-    if Y is None:
-        Y = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
-    if saved is None:
-        saved = make_mlp_saved(M, h, r, X.device)
-    if rstd is None:
-        rstd = torch.empty(M, dtype=torch.float32, device=X.device)
-    buf = ws.get(qlora_norm_mlp_workspace_bytes(M, d, h, r))
-    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
-    _check("qlora_norm_mlp_fwd", lib().qlora_norm_mlp_fwd(QLORA_ACT[act], _p(norm_w), float(eps), int(bool(plus_one)),
-                                                          ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X),
-                                                          M, _p(Y), ctypes.byref(sv), _p(rstd), _p(buf), buf.numel(),
-                                                          _stream()))
-    return Y, saved, rstd
-
-
-def qlora_norm_mlp_bwd(act, norm_w, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, rstd, dY,
-                       ws: Workspace, plus_one=False, grads=None):
-    """Backward of qlora_norm_mlp_fwd; grads["dX"] is the gradient with respect to the norm's input."""
-    M, d = X.shape
-    h = _dims(gate)[0]
-    if grads is None:
-        grads = {"dX": torch.empty(M, d, dtype=torch.bfloat16, device=X.device),
-                 "dA_g": torch.empty_like(gate.A), "dB_g": torch.empty_like(gate.B),
-                 "dA_u": torch.empty_like(up.A), "dB_u": torch.empty_like(up.B),
-                 "dA_d": torch.empty_like(down.A), "dB_d": torch.empty_like(down.B)}
-    buf = ws.get(qlora_norm_mlp_workspace_bytes(M, d, h, gate.A.shape[1]))
-    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
-    outs = [_p(grads[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
-    _check("qlora_norm_mlp_bwd", lib().qlora_norm_mlp_bwd(QLORA_ACT[act], _p(norm_w), int(bool(plus_one)),
-                                                          ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X),
-                                                          ctypes.byref(sv), _p(rstd), _p(dY), M, *outs, _p(buf),
-                                                          buf.numel(), _stream()))
-    return grads
 
 
 def qlora_rmsnorm_fwd(X, w, eps, plus_one=False, Y=None, rstd=None):

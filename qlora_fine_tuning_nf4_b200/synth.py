@@ -103,21 +103,3 @@ def make_qkv_problem(M, K, nq, nk, nv, r=16, alpha=16.0, seed=0):
     out["dY"] = _normal(ch[10], (M, nq + nk + nv))
     out.update({"s": float(alpha) / float(r), "M": M, "K": K, "nq": nq, "nk": nk, "nv": nv, "r": r})
     return out
-
-
-def make_norm_mlp_problem(M, d, h, r=16, alpha=16.0, seed=0, plus_one=False):
-    """RMS norm + gated MLP: the gated MLP's inputs with token rows whose norms
-    spread by 2x (hidden states entering a norm: X rows scaled by U(0.7, 1.4),
-    re-rounded to bf16) and the norm weight w [d]: N(1, 0.1) for the gain w,
-    N(0, 0.1) for the gain 1 + w (``plus_one``, Gemma's form).
-
-    Children of ``SeedSequence([seed, 1])``: row scales, w.
-    """
-    p = make_mlp_problem(M, d, h, r, alpha, seed)
-    ch = [np.random.default_rng(c) for c in np.random.SeedSequence([seed, 1]).spawn(2)]
-    scale = ch[0].uniform(0.7, 1.4, size=(M, 1)).astype(np.float32)
-    x32 = (p["X"].astype(np.uint32) << 16).view(np.float32)
-    p["X"] = bf16_bits(x32 * scale)
-    w = ch[1].standard_normal(d, dtype=np.float32) * np.float32(0.1)
-    p["w"] = bf16_bits(w + np.float32(0.0 if plus_one else 1.0))
-    return p

@@ -8,9 +8,8 @@ stores, in ``tests/golden/full_<workload>.npz``:
     quantiser must match them bit for bit);
   * the RMS of every returned tensor over the whole workload (the tolerance is
     2e-2 x RMS);
-  * a few sampled rows of Y, dX (and E, G, H for the MLP; rstd for the MLP
-    behind its RMS norm, stored as full_norm_<workload>.npz), including the
-    first and last row;
+  * a few sampled rows of Y, dX (and E, G, H for the MLP), including the first
+    and last row;
   * 4096 sampled entries of every adapter gradient dA / dB.
 The forward/backward runs in chunks of rows; the adapter gradients (sums over
 rows) are accumulated over the chunks.
@@ -29,7 +28,7 @@ sys.path.insert(0, ROOT)
 
 import oracle  # noqa: E402
 from oracle.nf4 import nf4_dequantize_f64  # noqa: E402
-from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem, make_norm_mlp_problem  # noqa: E402
+from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem  # noqa: E402
 from qlora_fine_tuning_nf4_b200.workloads import LINEAR_WORKLOADS, MLP_WORKLOADS  # noqa: E402
 
 CHUNK = 2048
@@ -97,38 +96,9 @@ def linear(name, cfg):
     return out
 
 
-# The RMS norm in front of the MLP (the fused norm + MLP entry points): gain w for
-# SwiGLU models, 1 + w for Gemma's GeGLU, as the pages describe them.
-NORM_EPS = {False: 1e-5, True: 1e-6}
-
-
-def saved_bound_rows(act, X, lin, E, G, H):
-    """Elementwise bounds of the bf16 E, G, H rows of an MLP whose GEMM operands
-    carry one bf16 rounding per input-side element (u = 2^-8): the stored
-    value's rounding, the rounded LoRA operand, fp32 accumulation, and the
-    rounding of the input side (u (|X||W|^T + s (|X||A|)|B|)); h = act(e) g
-    propagates |act'(e) g| |de| + |act(e)| |dg|."""
-    u = 2.0 ** -8
-    de = {}
-    for k, key, v in (("g", "E", E), ("u", "G", G)):
-        W, A, B, s = lin[k]
-        xw = np.abs(X) @ np.abs(W).T
-        de[key] = (4 * u * s * (np.abs(X @ A) @ np.abs(B)) + 2.0 ** -14 * xw +
-                   2 * u * (xw + s * ((np.abs(X) @ np.abs(A)) @ np.abs(B))))
-    return {"E": 2 * u * np.abs(E) + de["E"], "G": 2 * u * np.abs(G) + de["G"],
-            "H": 2 * u * np.abs(H) + np.abs(oracle.act_grad(act, E) * G) * de["E"] +
-            np.abs(oracle.act_fwd(act, E)) * de["G"]}
-
-
-def mlp(name, cfg, norm=False):
+def mlp(name, cfg):
     M, d, h, r, act = cfg["M"], cfg["d"], cfg["h"], cfg["r"], cfg["act"]
-    plus_one = act == "geglu_tanh"
-    if norm:
-        p = make_norm_mlp_problem(M, d, h, r, cfg["alpha"], cfg["seed"], plus_one=plus_one)
-        wn = oracle.bf16_bits_to_f64(p["w"])
-        eps = NORM_EPS[plus_one]
-    else:
-        p = make_mlp_problem(M, d, h, r, cfg["alpha"], cfg["seed"])
+    p = make_mlp_problem(M, d, h, r, cfg["alpha"], cfg["seed"])
     out = {}
     lin = {}
     for k in ("g", "u", "d"):
@@ -137,46 +107,28 @@ def mlp(name, cfg, norm=False):
     rows = sample_rows(M, N_ROWS, 1)
     rows_wide = rows[np.linspace(0, len(rows) - 1, N_ROWS_WIDE).astype(int)]
     widths = {"Y": d, "dX": d, "E": h, "G": h, "H": h}
-    if norm:
-        widths["rstd"] = 1
     ss = {k: 0.0 for k in widths}
-    row_vals = {k: np.zeros((len(rows if k in ("Y", "dX", "rstd") else rows_wide), w), np.float32)
+    row_vals = {k: np.zeros((len(rows if k in ("Y", "dX") else rows_wide), w), np.float32)
                 for k, w in widths.items()}
-    bounds = {k: np.zeros((len(rows_wide), h)) for k in ("E", "G", "H")}
     grads = {"dA_g": np.zeros((d, r)), "dB_g": np.zeros((r, h)), "dA_u": np.zeros((d, r)),
              "dB_u": np.zeros((r, h)), "dA_d": np.zeros((h, r)), "dB_d": np.zeros((r, d))}
     for m0 in range(0, M, CHUNK):
         m1 = min(M, m0 + CHUNK)
         X = oracle.bf16_bits_to_f64(p["X"][m0:m1])
         dY = oracle.bf16_bits_to_f64(p["dY"][m0:m1])
-        Xin = X
-        if norm:  # the norm, then the MLP on the normalised rows; backward in the reverse order
-            Xin, rstd = oracle.rmsnorm_fwd(X, wn, eps, plus_one=plus_one)
-        fwd = oracle.mlp_fwd(act, Xin, lin["g"], lin["u"], lin["d"])
-        bwd = oracle.mlp_bwd(act, Xin, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+        fwd = oracle.mlp_fwd(act, X, lin["g"], lin["u"], lin["d"])
+        bwd = oracle.mlp_bwd(act, X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
         for k in grads:
             grads[k] += bwd[k]
         vals = {"Y": fwd["Y"], "dX": bwd["dX"], "E": fwd["E"], "G": fwd["G"], "H": fwd["H"]}
-        if norm:
-            vals["dX"] = oracle.rmsnorm_bwd(X, wn, eps, bwd["dX"], plus_one=plus_one)
-            vals["rstd"] = rstd[:, None]
-            sel = (rows_wide >= m0) & (rows_wide < m1)
-            if sel.any():
-                i = rows_wide[sel] - m0
-                b = saved_bound_rows(act, Xin[i], lin, fwd["E"][i], fwd["G"][i], fwd["H"][i])
-                for k in ("E", "G", "H"):
-                    bounds[k][sel] = b[k]
         for k, v in vals.items():
             ss[k] += float(np.sum(v * v))
-            rr = rows if k in ("Y", "dX", "rstd") else rows_wide
+            rr = rows if k in ("Y", "dX") else rows_wide
             sel = (rr >= m0) & (rr < m1)
             row_vals[k][sel] = v[rr[sel] - m0]
         del fwd, bwd, vals
     out["rows"] = rows
     out["rows_wide"] = rows_wide
-    if norm:
-        for k, v in bounds.items():
-            out[f"bound_{k}"] = v
     for k, w in widths.items():
         out[f"rms_{k}"] = np.array(np.sqrt(ss[k] / (M * w)))
         out[f"rows_{k}"] = row_vals[k]
@@ -188,21 +140,11 @@ def mlp(name, cfg, norm=False):
     return out
 
 
-# workloads also stored behind their RMS norm (file full_norm_<workload>.npz)
-NORM_WORKLOADS = ["llama7b_swiglu_mlp", "gemma7b_geglu_mlp"]
-
-
 def main(names):
-    todo = names or ([n for n in LINEAR_WORKLOADS if n != "tiny_linear"] + list(MLP_WORKLOADS) +
-                     ["norm_" + n for n in NORM_WORKLOADS])
+    todo = names or [n for n in LINEAR_WORKLOADS if n != "tiny_linear"] + list(MLP_WORKLOADS)
     for name in todo:
         t0 = time.time()
-        if name.startswith("norm_"):
-            out = mlp(name, MLP_WORKLOADS[name[len("norm_"):]], norm=True)
-        elif name in LINEAR_WORKLOADS:
-            out = linear(name, LINEAR_WORKLOADS[name])
-        else:
-            out = mlp(name, MLP_WORKLOADS[name])
+        out = linear(name, LINEAR_WORKLOADS[name]) if name in LINEAR_WORKLOADS else mlp(name, MLP_WORKLOADS[name])
         np.savez(os.path.join(HERE, f"full_{name}.npz"), **out)
         print(f"{name}: {time.time() - t0:.1f} s", flush=True)
 

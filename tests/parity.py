@@ -44,7 +44,7 @@ def assert_close(name, gpu, ref, tol=TOL):
     return err / max(rms, 1e-300)
 
 
-def saved_bounds(o, p, input_round=False):
+def saved_bounds(o, p):
     """Elementwise error bounds of the saved bf16 activations E, G, H.
 
     bf16 keeps 8 significant bits, so one round-to-nearest-even costs at most
@@ -53,11 +53,6 @@ def saved_bounds(o, p, input_round=False):
     2^-16 |X||W|^T; both carry a safety factor 4, and the stored value's own
     rounding (u |e|) a factor 2.  h = act(e) g is formed from the fp32 e, g:
     |dh| <= 2u |h| + |act'(e) g| |de| + |act(e)| |dg|.
-
-    input_round: the GEMM's operands carry one bf16 rounding per element of the
-    input side (the fused RMS norm rounds the gain into the weight, W diag(g),
-    and into the factor, diag(g) A; the unfused chain rounds Xn instead), which
-    adds u (|X||W|^T + s (|X||A|)|B|) with X the MLP's input; factor 2.
     """
     u = 2.0 ** -8
     act = o["act"]
@@ -66,8 +61,6 @@ def saved_bounds(o, p, input_round=False):
     for k, key in (("g", "E"), ("u", "G")):
         W, A, B, s = o["lin"][k]
         de[key] = 4 * u * s * (np.abs(o["X"] @ A) @ np.abs(B)) + 2.0 ** -14 * (np.abs(o["X"]) @ np.abs(W).T)
-        if input_round:
-            de[key] = de[key] + 2 * u * (np.abs(o["X"]) @ np.abs(W).T + s * ((np.abs(o["X"]) @ np.abs(A)) @ np.abs(B)))
         out[key] = 2 * u * np.abs(o[key]) + de[key]
     out["H"] = (2 * u * np.abs(o["H"]) + np.abs(oracle.act_grad(act, o["E"]) * o["G"]) * de["E"]
                 + np.abs(oracle.act_fwd(act, o["E"])) * de["G"])

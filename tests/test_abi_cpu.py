@@ -104,25 +104,3 @@ def test_tile_config_setting(lib):
     assert ops.qlora_set_tile_config(prev) == 1
     assert ops.qlora_set_tile_config(7) == prev  # invalid values are ignored
     assert ops.qlora_set_tile_config(prev) == prev
-
-
-def test_norm_mlp_host_side_rejections(lib):
-    """The fused norm + MLP entry points validate on the host before any launch."""
-    g, u, d = _lin(n=512, k=256), _lin(n=512, k=256), _lin(n=256, k=512)
-    sv = ops.QloraMlpSaved(16, 16, 16, 16, 16, 16)
-    f = lib.qlora_norm_mlp_fwd
-    big = 1 << 40
-    args = lambda w, eps, rstd, M=8: (0, w, eps, 0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, M, 16,
-                                      ctypes.byref(sv), rstd, 16, big, None)
-    assert f(*args(16, 1e-5, 16, M=0)) == 0      # nothing to do
-    assert f(*args(None, 1e-5, 16)) == 1         # no norm weight
-    assert f(*args(16, -1.0, 16)) == 1           # negative epsilon
-    assert f(*args(16, 1e-5, None)) == 1         # no rstd output
-    assert f(*args(24, 1e-5, 16)) == 3           # misaligned norm weight
-    assert f(*(args(16, 1e-5, 16)[:-2] + (64, None))) == 4  # workspace too small
-    lib.qlora_set_tile_config(2)                 # the fusion needs the staged weight feed
-    try:
-        assert f(*args(16, 1e-5, 16)) == 2
-    finally:
-        lib.qlora_set_tile_config(4)
-    assert ops.qlora_norm_mlp_workspace_bytes(8192, 4096, 11008) > ops.qlora_mlp_workspace_bytes(8192, 4096, 11008)
