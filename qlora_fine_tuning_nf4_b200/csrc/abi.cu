@@ -171,10 +171,9 @@ bool map_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t
 // Skinny passes run up to four persistent CTAs per SM; a CTA's ring holds four
 // stages of one 64x64 tile of T plus 128 bytes per factor column (the grid
 // shrinks when wide factor tiles limit residency).
-constexpr int kSMs = 148;
 int skinny_target_ctas(int factor_cols) {
   const int smem = 4 * (8192 + 128 * factor_cols) + 64 + 1024;
-  return kSMs * std::max(1, std::min(4, 232448 / smem));
+  return num_sms() * std::max(1, std::min(4, 232448 / smem));  // the device's SMs (148 when none is present)
 }
 
 // Partition of `groups` output groups of `upg` units each over the CTAs:
