@@ -179,11 +179,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------ oracle arm ---
 
-def oracle_sample(wl, rows, seed_rows=0):
+def oracle_sample(wl, rows=None, seed_rows=0, target_s=12.0):
     """Time the fp64 oracle's MLP fwd+bwd on `rows` tokens of the workload.
 
-    Returns (seconds, flop, threads).  Weights are quantised/dequantised by the
-    oracle itself before timing (one-time, like the GPU side's quantisation).
+    With rows None, a 64-row probe sizes the sample to about `target_s` seconds
+    of CPU work (at most the whole batch).  Returns (seconds, flop, threads,
+    rows).  Weights are quantised/dequantised by the oracle itself before
+    timing (one-time, like the GPU side's quantisation).
     """
     import oracle
     from oracle.nf4 import nf4_dequantize_f64
@@ -196,13 +198,21 @@ def oracle_sample(wl, rows, seed_rows=0):
         c, a = oracle.nf4_quantize(p["W_" + k], n, kk)
         lin[k] = (nf4_dequantize_f64(c, a, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
                   oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
-    X = oracle.bf16_bits_to_f64(p["X"][seed_rows:seed_rows + rows])
-    dY = oracle.bf16_bits_to_f64(p["dY"][seed_rows:seed_rows + rows])
-    t0 = time.perf_counter()
-    fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
-    oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
-    dt = time.perf_counter() - t0
-    return dt, mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0))
+
+    def run(n):
+        X = oracle.bf16_bits_to_f64(p["X"][seed_rows:seed_rows + n])
+        dY = oracle.bf16_bits_to_f64(p["dY"][seed_rows:seed_rows + n])
+        t0 = time.perf_counter()
+        fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
+        oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+        return time.perf_counter() - t0
+
+    if rows is None:
+        per_row = run(64) / 64
+        rows = int(min(wl["M"] - seed_rows, max(64, target_s / max(per_row, 1e-9))))
+        rows -= rows % 64
+    dt = run(rows)
+    return dt, mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0)), rows
 
 
 def c_loop_oracle_sample():
@@ -616,8 +626,7 @@ def run_ours(args, wl):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "mlp":
-        rows = 512
-        dt, fl, cores = oracle_sample(wl, rows)
+        dt, fl, cores, rows = oracle_sample(wl)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{rows} of {M} token rows, one fwd+bwd (fp64 numpy, {dt:.1f} s)",
                "c_loop_oracle": c_loop_oracle_sample()}
