@@ -33,7 +33,9 @@
  *    _WORKSPACE_TOO_SMALL).  A failed launch returns QLORA_ERR_CUDA.  Errors
  *    found on the device (a pipeline wait that exceeded its time limit) are
  *    recorded in the status word and reported by qlora_last_device_status.
- *  - M = 0 is valid and enqueues nothing.
+ *  - M = 0 is valid.  A forward then enqueues nothing; a backward sets its
+ *    adapter gradients dA, dB to zero (sums over no tokens) with memsets on
+ *    the stream and reads or writes nothing else.
  */
 #ifndef QLORA_H_
 #define QLORA_H_

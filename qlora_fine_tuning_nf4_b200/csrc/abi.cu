@@ -132,6 +132,21 @@ int num_sms() {
 }
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// Backward of an empty batch (M = 0): every adapter gradient is a sum over no
+// tokens, so it is zero.  The gradients are cleared on the stream (a data-
+// parallel all-reduce then sums correct values from a rank whose shard is
+// empty); nothing else is read or written.
+qlora_status zero_adapter_grads(qlora_bf16* const* g, const int64_t* elems, int n, cudaStream_t st) {
+  for (int i = 0; i < n; ++i) {
+    if (!g[i]) return QLORA_ERR_INVALID_ARG;
+    if (misaligned(g[i])) return QLORA_ERR_MISALIGNED;
+  }
+  for (int i = 0; i < n; ++i)
+    if (cudaMemsetAsync(g[i], 0, static_cast<size_t>(elems[i]) * sizeof(qlora_bf16), st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -620,7 +635,11 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
   qlora_status s = check_linear(lin, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
-  if (M == 0) return QLORA_OK;  // NOTE: dA, dB are left untouched when there are no rows
+  if (M == 0) {
+    qlora_bf16* g[2] = {dA, dB};
+    const int64_t n[2] = {lin->w.k_in * lin->r, lin->w.n_out * lin->r};
+    return zero_adapter_grads(g, n, 2, reinterpret_cast<cudaStream_t>(stream));
+  }
   if (!X || !XA_saved || !dY || !dX || !dA || !dB || !ws) return QLORA_ERR_INVALID_ARG;
   if (misaligned(X) || misaligned(XA_saved) || misaligned(dY) || misaligned(dX) || misaligned(dA) ||
       misaligned(dB) || misaligned(ws))
@@ -822,7 +841,12 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
   qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
-  if (M == 0) return QLORA_OK;
+  if (M == 0) {
+    const int64_t dm = gate->w.k_in, hm = gate->w.n_out, rm = gate->r;
+    qlora_bf16* g[6] = {dA_g, dB_g, dA_u, dB_u, dA_d, dB_d};
+    const int64_t n[6] = {dm * rm, rm * hm, dm * rm, rm * hm, hm * rm, rm * dm};
+    return zero_adapter_grads(g, n, 6, reinterpret_cast<cudaStream_t>(stream));
+  }
   if (!X || !sv || !sv->E || !sv->G || !sv->H || !sv->XA_g || !sv->XA_u || !sv->HA_d || !dY || !dX || !dA_g ||
       !dB_g || !dA_u || !dB_u || !dA_d || !dB_d || !ws)
     return QLORA_ERR_INVALID_ARG;
@@ -1033,9 +1057,17 @@ qlora_status qlora_qkv_bwd(const qlora_lora_linear* q_, const qlora_lora_linear*
   qlora_status s = check_qkv(&lq, &lk, &lv);
   if (s != QLORA_OK) return s;
   if (M < 0) return QLORA_ERR_INVALID_ARG;
-  if (M == 0) return QLORA_OK;
   qlora_bf16* dA[3] = {dA_q, dA_k, dA_v};
   qlora_bf16* dB[3] = {dB_q, dB_k, dB_v};
+  if (M == 0) {
+    qlora_bf16* g[6] = {dA_q, dB_q, dA_k, dB_k, dA_v, dB_v};
+    int64_t n[6];
+    for (int p = 0; p < 3; ++p) {
+      n[2 * p] = L[p]->w.k_in * L[p]->r;       // dA [K, r]
+      n[2 * p + 1] = L[p]->r * L[p]->w.n_out;  // dB [r, n_p]
+    }
+    return zero_adapter_grads(g, n, 6, reinterpret_cast<cudaStream_t>(stream));
+  }
   if (!X || !XA_saved || !dY || !dX || !ws) return QLORA_ERR_INVALID_ARG;
   for (int p = 0; p < 3; ++p)
     if (!dA[p] || !dB[p]) return QLORA_ERR_INVALID_ARG;

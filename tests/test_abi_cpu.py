@@ -73,6 +73,9 @@ def test_host_side_rejections(lib):
     assert lib.nf4_dequantize(16, 16, 4, 100, 16, None) == 2                    # k_in % 64
     assert lib.nf4_dequantize(16, 16, 4, 64, 8, None) == 3
     assert lib.nf4_quantize(16, 0, 64, 16, 16, None) == 0                       # empty
+    b = lib.qlora_linear_bwd  # M = 0 clears dA, dB: their pointers are still checked before any CUDA call
+    assert b(ctypes.byref(c), None, None, None, 0, None, None, 16, None, 0, None) == 1  # null dA
+    assert b(ctypes.byref(c), None, None, None, 0, None, 16, 24, None, 0, None) == 3    # misaligned dB
     g, u, d = _lin(n=512, k=256), _lin(n=512, k=256), _lin(n=256, k=512)
     sv = ops.QloraMlpSaved(16, 16, 16, 16, 16, 16)
     mf = lib.qlora_mlp_fwd

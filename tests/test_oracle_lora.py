@@ -47,6 +47,32 @@ def test_s_zero_is_pure_dense_layer():
     assert np.all(dA == 0) and np.all(dB == 0)
 
 
+def test_adapter_gradients_add_over_token_shards_and_vanish_for_no_tokens():
+    """dA, dB are sums over tokens: the gradients of a batch equal the sum of
+    those of any split of its rows (what a data-parallel all-reduce relies
+    on), and an empty batch gives exactly zero."""
+    rng = np.random.default_rng(3)
+    X, W, A, B, s, dY = _lin(rng, 12, 64, 16, 4, s=2.0)
+    _, dA, dB = oracle.linear_bwd(X, W, A, B, s, dY)
+    _, dA1, dB1 = oracle.linear_bwd(X[:5], W, A, B, s, dY[:5])
+    _, dA2, dB2 = oracle.linear_bwd(X[5:], W, A, B, s, dY[5:])
+    assert np.allclose(dA, dA1 + dA2, rtol=0, atol=1e-12) and np.allclose(dB, dB1 + dB2, rtol=0, atol=1e-12)
+    Y0, XA0 = oracle.linear_fwd(X[:0], W, A, B, s)
+    dX0, dA0, dB0 = oracle.linear_bwd(X[:0], W, A, B, s, dY[:0])
+    assert Y0.shape == (0, 16) and XA0.shape == (0, 4) and dX0.shape == (0, 64)
+    assert dA0.shape == A.shape and dB0.shape == B.shape and not dA0.any() and not dB0.any()
+    lin = lambda n_out, k_in: (rng.standard_normal((n_out, k_in)) * 0.1, rng.uniform(-1, 1, (k_in, 4)) / np.sqrt(k_in),
+                               rng.standard_normal((4, n_out)) * 0.1, 2.0)
+    g, u, d = lin(32, 16), lin(32, 16), lin(16, 32)
+    Xm, dYm = rng.standard_normal((9, 16)), rng.standard_normal((9, 16))
+    full = oracle.mlp_bwd("swiglu", Xm, g, u, d, dYm)
+    parts = [oracle.mlp_bwd("swiglu", Xm[a:b], g, u, d, dYm[a:b]) for a, b in ((0, 4), (4, 9))]
+    empty = oracle.mlp_bwd("swiglu", Xm[:0], g, u, d, dYm[:0])
+    for k in ("dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert np.allclose(full[k], parts[0][k] + parts[1][k], rtol=0, atol=1e-12), k
+        assert empty[k].shape == full[k].shape and not empty[k].any(), k
+
+
 def test_zero_absmax_is_pure_lora():
     rng = np.random.default_rng(2)
     M, K, N, r = 6, 128, 8, 4
