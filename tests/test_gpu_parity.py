@@ -16,7 +16,7 @@ import oracle
 from qlora_fine_tuning_nf4_b200 import ops
 from qlora_fine_tuning_nf4_b200.synth import bf16_bits, make_linear_problem, make_mlp_problem
 
-from parity import (TOL_SMALL_MLP, assert_close, assert_saved, dev, gpu_weight, oracle_weight, run_linear_gpu,
+from parity import (TOL_SMALL_MLP, assert_close, assert_saved, gpu_weight, oracle_weight, run_linear_gpu,
                     run_linear_oracle, run_mlp_gpu, run_mlp_oracle, saved_bounds)
 
 pytestmark = pytest.mark.gpu

@@ -8,7 +8,7 @@ import pytest
 
 from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem
 
-from parity import (TOL, TOL_SMALL_MLP, assert_close, assert_saved, run_linear16_gpu, run_linear_gpu,
+from parity import (TOL_SMALL_MLP, assert_close, assert_saved, run_linear16_gpu, run_linear_gpu,
                     run_linear_oracle, run_mlp16_gpu, run_mlp_gpu, run_mlp_oracle, saved_bounds)
 
 pytestmark = pytest.mark.gpu

@@ -9,7 +9,6 @@ import math
 import os
 
 import numpy as np
-import pytest
 import torch
 
 import oracle
