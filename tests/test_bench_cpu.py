@@ -1,0 +1,25 @@
+"""Host logic of the benchmark: the FLOP counts it divides by and the choice
+of the roofline denominator (no GPU needed)."""
+
+import bench
+
+
+def test_mlp_flops_is_the_sum_of_its_gemms_and_lora_terms():
+    M, d, h, r = 8192, 4096, 11008, 16
+    dense = 4 * M * d * 2 * h + 4 * M * h * d          # fwd + dX of gate/up (N = 2h) and of down
+    lora = 6 * M * r * (d + h) * 2 + 6 * M * r * (h + d)  # 6 M r (K + N) per projection
+    assert bench.mlp_flops(M, d, h, r) == dense + lora
+    per_gemm = sum(bench.kernel_flops(k, M, d, h, r) for k in
+                   ("gemm_nf4_gateup_glu_fwd", "gemm_nf4_fwd", "gemm_nf4_down_bwd_glu", "gemm_nf4_bwd_dx"))
+    assert per_gemm <= bench.mlp_flops(M, d, h, r)     # the skinny passes carry the rest of the LoRA work
+    assert per_gemm >= dense
+
+
+def test_roofline_peak_follows_the_measured_clock():
+    pk = {"bf16": 1637.6, "bf16_sustained": 1390.6, "sustained_mhz": 1342.0, "max_mhz": 1965.0, "src": "measured"}
+    peak, kind = bench.tensor_peak(pk, {"sm_mhz": 1320.0})   # held at the power cap: the sustained loop's figure
+    assert peak == 1390.6 and "sustained" in kind
+    peak, kind = bench.tensor_peak(pk, {"sm_mhz": 1965.0})   # full clock: the burst figure
+    assert peak == 1637.6 and "burst" in kind
+    peak, kind = bench.tensor_peak(pk, {"sm_mhz": None})
+    assert peak == 1390.6 and "no clock record" in kind
