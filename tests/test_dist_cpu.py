@@ -1,6 +1,7 @@
-"""Multi-process (world size 2, gloo, CPU) check of the data-parallel step logic:
-each rank computes the adapter gradients of its token shard (oracle, fp64), the
-flat buffer is all-reduced, and the sum equals the full-batch gradients."""
+"""Multi-process (gloo, CPU) check of the data-parallel step logic: each rank
+computes the adapter gradients of its token shard (oracle, fp64), the flat
+buffer is all-reduced, and the sum equals the full-batch gradients.  One case
+leaves a rank with no tokens: its gradients are zero and the sum is unchanged."""
 
 import os
 import socket
@@ -23,9 +24,9 @@ def _free_port():
     return port
 
 
-def _problem():
+def _problem(M=24):
     rng = np.random.default_rng(0)
-    M, d, h, r = 24, 64, 96, 4
+    d, h, r = 64, 96, 4
     X = rng.standard_normal((M, d))
     proj = lambda K, N, s: (rng.standard_normal((N, K)) * 0.2, rng.uniform(-1, 1, (K, r)) / np.sqrt(K),
                             rng.standard_normal((r, N)) * 0.3, s)
@@ -34,12 +35,12 @@ def _problem():
     return M, d, h, r, X, gate, up, down, dY
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, M):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        M, d, h, r, X, gate, up, down, dY = _problem()
+        M, d, h, r, X, gate, up, down, dY = _problem(M)
         lo, hi = dp.shard_rows(M, rank, world)
         g = oracle.mlp_bwd("swiglu", X[lo:hi], gate, up, down, dY[lo:hi])
         flat, views = dp.flat_lora_grads(d, h, r, "cpu", dtype=torch.float64)
@@ -52,18 +53,19 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_sharded_gradients_sum_to_full_batch():
+@pytest.mark.parametrize("M,world", [(24, 2), (2, 3)])  # (2, 3): the third rank's shard is empty
+def test_sharded_gradients_sum_to_full_batch(M, world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(rk, 2, port, q)) for rk in range(2)]
+    procs = [ctx.Process(target=_worker, args=(rk, world, port, q, M)) for rk in range(world)]
     for p in procs:
         p.start()
     got = q.get(timeout=120)
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
-    M, d, h, r, X, gate, up, down, dY = _problem()
+    M, d, h, r, X, gate, up, down, dY = _problem(M)
     full = oracle.mlp_bwd("swiglu", X, gate, up, down, dY)
     for k in dp.GRAD_ORDER:
         np.testing.assert_allclose(got[k], full[k], rtol=1e-12, atol=1e-12)
