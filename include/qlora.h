@@ -36,6 +36,9 @@
  *  - M = 0 is valid.  A forward then enqueues nothing; a backward sets its
  *    adapter gradients dA, dB to zero (sums over no tokens) with memsets on
  *    the stream and reads or writes nothing else.
+ *  - M, k_in, n_out (and nq + nk + nv of the fused Q/K/V calls) are at most
+ *    2^23 = 8,388,608; larger values return QLORA_ERR_UNSUPPORTED_SHAPE (the
+ *    kernels index rank-side partials and output tiles with 32-bit integers).
  */
 #ifndef QLORA_H_
 #define QLORA_H_

@@ -67,6 +67,10 @@ int32_t g_tiles = 4;  // GEMM tile configuration (see qlora_set_tile_config)
 #define QL_GROUP_M 8
 #endif
 constexpr int kGroupM = QL_GROUP_M;  // output-row tiles per group of the GEMM tile order
+// Largest M, k_in, n_out (and nq + nk + nv) a call accepts.  The skinny
+// reductions index rows x factor columns (up to 192) and the GEMMs count
+// output tiles in 32-bit integers; at 2^23 both stay below 2^31.
+constexpr int64_t kMaxDim = int64_t(1) << 23;
 
 // Internal view of one projection: a frozen NF4 base (codes + absmax) or a
 // frozen bf16 base (w16), plus its LoRA factors.
@@ -472,7 +476,7 @@ qlora_status check_linear(const Lin* lin, int tiles) {
   if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
   if (!rank_ok(lin->r, tiles)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in % 256 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (lin->w.k_in > (1 << 30) || lin->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (lin->w.k_in > kMaxDim || lin->w.n_out > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->w.w16) || misaligned(lin->A) ||
       misaligned(lin->B))
     return QLORA_ERR_MISALIGNED;
@@ -611,7 +615,7 @@ static qlora_status linear_fwd(const Lin* lin, int tiles, const qlora_bf16* X, i
   if (M == 0) return QLORA_OK;
   if (!X || !Y || !XA_saved || !ws) return QLORA_ERR_INVALID_ARG;
   if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
   const int r = lin->r;
   const bool stage = is_staged(tiles) && !lin->w.w16;
@@ -644,7 +648,7 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
   if (misaligned(X) || misaligned(XA_saved) || misaligned(dY) || misaligned(dX) || misaligned(dA) ||
       misaligned(dB) || misaligned(ws))
     return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in, N = lin->w.n_out;
   const int r = lin->r;
   const bool stage_w = is_staged(tiles) && !lin->w.w16;
@@ -772,7 +776,7 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
   if (misaligned(X) || misaligned(Y) || misaligned(sv->E) || misaligned(sv->G) || misaligned(sv->H) ||
       misaligned(sv->XA_g) || misaligned(sv->XA_u) || misaligned(sv->HA_d) || misaligned(ws))
     return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
@@ -854,7 +858,7 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
                         dB_d, ws};
   for (const void* p : ptrs)
     if (misaligned(p)) return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t d = gate->w.k_in, h = gate->w.n_out;
   const int r = gate->r;
   const bool stage = is_staged(tiles) && !gate->w.w16;
@@ -967,7 +971,7 @@ qlora_status check_qkv(const Lin* q, const Lin* k, const Lin* v) {
   if (q->r != k->r || q->r != v->r) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (q->w.n_out % 256 || k->w.n_out % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;  // tiles never straddle
   if (q->w.w16 || k->w.w16 || v->w.w16) return QLORA_ERR_INVALID_ARG;
-  if (q->w.n_out + k->w.n_out + v->w.n_out > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (q->w.n_out + k->w.n_out + v->w.n_out > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   return QLORA_OK;
 }
 // the three weights dequantised into consecutive rows of one [nq + nk + nv, K] buffer
@@ -996,7 +1000,7 @@ qlora_status qlora_qkv_fwd(const qlora_lora_linear* q_, const qlora_lora_linear*
   if (M == 0) return QLORA_OK;
   if (!X || !Y || !XA_saved || !ws) return QLORA_ERR_INVALID_ARG;
   if (misaligned(X) || misaligned(Y) || misaligned(XA_saved) || misaligned(ws)) return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int r = lq.r;
   const int64_t K = lq.w.k_in, nq = lq.w.n_out, nk = lk.w.n_out, nv = lv.w.n_out, Nt = nq + nk + nv;
   if (ws_bytes < qkv_ws(M, K, nq, nk, nv, r)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
@@ -1074,7 +1078,7 @@ qlora_status qlora_qkv_bwd(const qlora_lora_linear* q_, const qlora_lora_linear*
   const void* ptrs[] = {X, XA_saved, dY, dX, dA_q, dB_q, dA_k, dB_k, dA_v, dB_v, ws};
   for (const void* p : ptrs)
     if (misaligned(p)) return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int r = lq.r;
   const int64_t K = lq.w.k_in, nq = lq.w.n_out, nk = lk.w.n_out, nv = lv.w.n_out, Nt = nq + nk + nv;
   const int64_t off[3] = {0, nq, nq + nk};
@@ -1342,7 +1346,7 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const ql
   if (M == 0) return QLORA_OK;
   if (!X || !Y || !XA_saved) return QLORA_ERR_INVALID_ARG;
   if (misaligned(X) || misaligned(Y) || misaligned(XA_saved)) return QLORA_ERR_MISALIGNED;
-  if (M > (1 << 30)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in;
   const size_t vec = align256(static_cast<size_t>(M) * 32);
   const size_t need = 256 + vec + align256(rowproj_part_bytes(M, K, 16));

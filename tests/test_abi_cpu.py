@@ -69,6 +69,9 @@ def test_host_side_rejections(lib):
     assert f(ctypes.byref(_lin(r=8)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # r != 16
     assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in % 256
     assert f(ctypes.byref(_lin(n=500)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # n_out % 8
+    assert f(ctypes.byref(c), 16, (1 << 23) + 1, 16, 16, 16, 1 << 62, None) == 2  # M above 2^23
+    assert f(ctypes.byref(_lin(k=(1 << 23) + 256)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in above 2^23
+    assert f(ctypes.byref(_lin(n=(1 << 23) + 8)), 16, 8, 16, 16, 16, 1 << 30, None) == 2    # n_out above 2^23
     assert f(ctypes.byref(_lin(codes=8)), 16, 8, 16, 16, 16, 1 << 30, None) == 3
     assert lib.nf4_dequantize(16, 16, 4, 100, 16, None) == 2                    # k_in % 64
     assert lib.nf4_dequantize(16, 16, 4, 64, 8, None) == 3
