@@ -156,6 +156,31 @@ def _dev(t, name):
     return t
 
 
+def _t(t, name, shape, dtype=torch.bfloat16):
+    """Marshalling check of one tensor argument: contiguous, on the current
+    CUDA device, of the expected dtype and shape.  The C ABI only sees raw
+    pointers, so a host tensor or a short buffer must be caught here."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor, got one on {t.device}")
+    if t.get_device() != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, not on the current device cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _rows(X, name="X"):
+    if not isinstance(X, torch.Tensor) or X.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor [M, features]")
+    return X.shape
+
+
 # ------------------------------------------------------------------ NF4 ----
 
 @dataclass
@@ -166,6 +191,8 @@ class NF4Weight:
     k_in: int
 
     def c(self):
+        _t(self.codes, "codes", (self.n_out * self.k_in // 2,), torch.uint8)
+        _t(self.absmax, "absmax", (self.n_out * self.k_in // 64,), torch.float32)
         return QloraNF4(self.codes.data_ptr(), self.absmax.data_ptr(), self.n_out, self.k_in)
 
 
@@ -177,8 +204,8 @@ def qlora_nf4_codebook():
 
 def nf4_quantize(w):
     """bf16 weight [n_out, k_in] on the GPU -> NF4Weight."""
-    _dev(w, "w")
-    n_out, k_in = w.shape
+    n_out, k_in = _rows(w, "w")
+    _t(w, "w", (n_out, k_in))
     codes = torch.empty(n_out * k_in // 2, dtype=torch.uint8, device=w.device)
     absmax = torch.empty(n_out * k_in // 64, dtype=torch.float32, device=w.device)
     _check("nf4_quantize", lib().nf4_quantize(_p(w), n_out, k_in, _p(codes), _p(absmax), _stream()))
@@ -189,6 +216,8 @@ def nf4_dequantize(w: NF4Weight, out=None):
     """NF4Weight -> bf16 [n_out, k_in] (bit-exact)."""
     if out is None:
         out = torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16, device=w.codes.device)
+    w.c()  # checks codes and absmax
+    _t(out, "out", (w.n_out, w.k_in))
     _check("nf4_dequantize", lib().nf4_dequantize(_p(w.codes), _p(w.absmax), w.n_out, w.k_in, _p(out), _stream()))
     return out
 
@@ -203,7 +232,10 @@ class LoraLinear:
     scale: float
 
     def c(self):
-        return QloraLoraLinear(self.w.c(), self.A.data_ptr(), self.B.data_ptr(), self.A.shape[1], self.scale)
+        r = self.A.shape[1] if self.A.dim() == 2 else -1
+        _t(self.A, "A", (self.w.k_in, r))
+        _t(self.B, "B", (r, self.w.n_out))
+        return QloraLoraLinear(self.w.c(), self.A.data_ptr(), self.B.data_ptr(), r, self.scale)
 
 
 @dataclass
@@ -223,8 +255,14 @@ class LoraLinear16:
         return self.w.shape[1]
 
     def c(self):
+        if self.w.dim() != 2:
+            raise ValueError("w must be a 2-D bf16 tensor [n_out, k_in]")
+        _t(self.w, "w", tuple(self.w.shape))
+        r = self.A.shape[1] if self.A.dim() == 2 else -1
+        _t(self.A, "A", (self.k_in, r))
+        _t(self.B, "B", (r, self.n_out))
         return QloraLoraLinear16(self.w.data_ptr(), self.n_out, self.k_in, self.A.data_ptr(), self.B.data_ptr(),
-                                 self.A.shape[1], self.scale)
+                                 r, self.scale)
 
 
 def _dims(lin):
@@ -262,14 +300,18 @@ def qlora_mlp16_workspace_bytes(M, d, h, r=16):
 
 
 def _linear_fwd(fn, wsq, lin, X, ws, Y, XA):
-    M = X.shape[0]
+    M = _rows(X)[0]
     n_out, k_in = _dims(lin)
+    r = lin.A.shape[1]
     if Y is None:
         Y = torch.empty(M, n_out, dtype=torch.bfloat16, device=X.device)
     if XA is None:
-        XA = torch.empty(M, lin.A.shape[1], dtype=torch.bfloat16, device=X.device)
-    buf = ws.get(wsq(M, k_in, n_out, lin.A.shape[1]))
+        XA = torch.empty(M, r, dtype=torch.bfloat16, device=X.device)
+    _t(X, "X", (M, k_in))
+    _t(Y, "Y", (M, n_out))
+    _t(XA, "XA", (M, r))
     c = lin.c()
+    buf = ws.get(wsq(M, k_in, n_out, r))
     _check(fn, getattr(lib(), fn)(ctypes.byref(c), _p(X), M, _p(Y), _p(XA), _p(buf), buf.numel(), _stream()))
     return Y, XA
 
@@ -286,11 +328,15 @@ def qlora_linear_fwd_noalloc(lin: LoraLinear, X, Y=None, XA=None):
     """qlora_linear_fwd without a workspace, for callers that cannot allocate
     device memory; its scratch is a fixed array inside the library (shared by
     all calls, so calls must not overlap on the GPU)."""
-    M = X.shape[0]
+    M = _rows(X)[0]
+    r = lin.A.shape[1]
     if Y is None:
         Y = torch.empty(M, lin.w.n_out, dtype=torch.bfloat16, device=X.device)
     if XA is None:
-        XA = torch.empty(M, lin.A.shape[1], dtype=torch.bfloat16, device=X.device)
+        XA = torch.empty(M, r, dtype=torch.bfloat16, device=X.device)
+    _t(X, "X", (M, lin.w.k_in))
+    _t(Y, "Y", (M, lin.w.n_out))
+    _t(XA, "XA", (M, r))
     c = lin.c()
     _check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(ctypes.byref(c), _p(X), M, _p(Y), _p(XA),
                                                                       _stream()))
@@ -298,16 +344,23 @@ def qlora_linear_fwd_noalloc(lin: LoraLinear, X, Y=None, XA=None):
 
 
 def _linear_bwd(fn, wsq, lin, X, XA, dY, ws, dX, dA, dB):
-    M = X.shape[0]
+    M = _rows(X)[0]
     n_out, k_in = _dims(lin)
+    r = lin.A.shape[1]
     if dX is None:
         dX = torch.empty(M, k_in, dtype=torch.bfloat16, device=X.device)
     if dA is None:
         dA = torch.empty_like(lin.A)
     if dB is None:
         dB = torch.empty_like(lin.B)
-    buf = ws.get(wsq(M, k_in, n_out, lin.A.shape[1]))
+    _t(X, "X", (M, k_in))
+    _t(XA, "XA", (M, r))
+    _t(dY, "dY", (M, n_out))
+    _t(dX, "dX", (M, k_in))
+    _t(dA, "dA", (k_in, r))
+    _t(dB, "dB", (r, n_out))
     c = lin.c()
+    buf = ws.get(wsq(M, k_in, n_out, r))
     _check(fn, getattr(lib(), fn)(ctypes.byref(c), _p(X), _p(XA), _p(dY), M, _p(dX), _p(dA), _p(dB), _p(buf),
                                   buf.numel(), _stream()))
     return dX, dA, dB
@@ -326,20 +379,33 @@ def make_mlp_saved(M, h, r, device):
     return {"E": e(M, h), "G": e(M, h), "H": e(M, h), "XA_g": e(M, r), "XA_u": e(M, r), "HA_d": e(M, r)}
 
 
-def _saved_c(sv):
+def _saved_c(sv, M, h, r):
+    for k in ("E", "G", "H"):
+        _t(sv[k], k, (M, h))
+    for k in ("XA_g", "XA_u", "HA_d"):
+        _t(sv[k], k, (M, r))
     return QloraMlpSaved(*[sv[k].data_ptr() for k in ("E", "G", "H", "XA_g", "XA_u", "HA_d")])
 
 
-def _mlp_fwd(fn, wsq, act, gate, up, down, X, ws, Y, saved):
-    M, d = X.shape
+def _mlp_dims(gate, up, down, d):
     h = _dims(gate)[0]
+    if _dims(gate) != (h, d) or _dims(up) != (h, d) or _dims(down) != (d, h):
+        raise ValueError(f"MLP weights must be gate, up [h, {d}] and down [{d}, h]")
+    return h
+
+
+def _mlp_fwd(fn, wsq, act, gate, up, down, X, ws, Y, saved):
+    M, d = _rows(X)
+    h = _mlp_dims(gate, up, down, d)
     r = gate.A.shape[1]
     if Y is None:
         Y = torch.empty(M, d, dtype=torch.bfloat16, device=X.device)
     if saved is None:
         saved = make_mlp_saved(M, h, r, X.device)
+    _t(X, "X", (M, d))
+    _t(Y, "Y", (M, d))
+    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved, M, h, r)
     buf = ws.get(wsq(M, d, h, r))
-    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
     _check(fn, getattr(lib(), fn)(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X), M,
                                   _p(Y), ctypes.byref(sv), _p(buf), buf.numel(), _stream()))
     return Y, saved
@@ -355,15 +421,22 @@ def qlora_mlp16_fwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear1
 
 
 def _mlp_bwd(fn, wsq, act, gate, up, down, X, saved, dY, ws, grads):
-    M, d = X.shape
-    h = _dims(gate)[0]
+    M, d = _rows(X)
+    h = _mlp_dims(gate, up, down, d)
+    r = gate.A.shape[1]
     if grads is None:
         grads = {"dX": torch.empty(M, d, dtype=torch.bfloat16, device=X.device),
                  "dA_g": torch.empty_like(gate.A), "dB_g": torch.empty_like(gate.B),
                  "dA_u": torch.empty_like(up.A), "dB_u": torch.empty_like(up.B),
                  "dA_d": torch.empty_like(down.A), "dB_d": torch.empty_like(down.B)}
-    buf = ws.get(wsq(M, d, h, gate.A.shape[1]))
-    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved)
+    _t(X, "X", (M, d))
+    _t(dY, "dY", (M, d))
+    _t(grads["dX"], "dX", (M, d))
+    for k, shp in (("dA_g", (d, r)), ("dB_g", (r, h)), ("dA_u", (d, r)), ("dB_u", (r, h)), ("dA_d", (h, r)),
+                   ("dB_d", (r, d))):
+        _t(grads[k], k, shp)
+    g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved, M, h, r)
+    buf = ws.get(wsq(M, d, h, r))
     outs = [_p(grads[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
     _check(fn, getattr(lib(), fn)(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X),
                                   ctypes.byref(sv), _p(dY), M, *outs, _p(buf), buf.numel(), _stream()))
@@ -381,20 +454,29 @@ def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear1
 
 def qlora_rmsnorm_fwd(X, w, eps, plus_one=False, Y=None, rstd=None):
     """RMS layer norm of X [M, d] with gain w (or 1 + w): returns (Y, rstd)."""
-    M, d = X.shape
+    M, d = _rows(X)
     if Y is None:
         Y = torch.empty_like(X)
     if rstd is None:
         rstd = torch.empty(M, dtype=torch.float32, device=X.device)
+    _t(X, "X", (M, d))
+    _t(w, "w", (d,))
+    _t(Y, "Y", (M, d))
+    _t(rstd, "rstd", (M,), torch.float32)
     _check("qlora_rmsnorm_fwd", lib().qlora_rmsnorm_fwd(_p(X), _p(w), M, d, float(eps), int(bool(plus_one)), _p(Y),
                                                         _p(rstd), _stream()))
     return Y, rstd
 
 
 def qlora_rmsnorm_bwd(X, w, rstd, dY, plus_one=False, dX=None):
-    M, d = X.shape
+    M, d = _rows(X)
     if dX is None:
         dX = torch.empty_like(X)
+    _t(X, "X", (M, d))
+    _t(w, "w", (d,))
+    _t(rstd, "rstd", (M,), torch.float32)
+    _t(dY, "dY", (M, d))
+    _t(dX, "dX", (M, d))
     _check("qlora_rmsnorm_bwd", lib().qlora_rmsnorm_bwd(_p(X), _p(w), _p(rstd), _p(dY), M, d, int(bool(plus_one)),
                                                         _p(dX), _stream()))
     return dX
@@ -406,30 +488,41 @@ def qlora_qkv_workspace_bytes(M, K, nq, nk, nv, r=16):
 
 def qlora_qkv_fwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, ws: Workspace, Y=None, XA=None):
     """Fused Q/K/V projection: Y = [Y_q | Y_k | Y_v] [M, nq + nk + nv], XA = [XA_q | XA_k | XA_v] [M, 3r]."""
-    M, K = X.shape
+    M, K = _rows(X)
     r = q.A.shape[1]
     nt = q.w.n_out + k.w.n_out + v.w.n_out
     if Y is None:
         Y = torch.empty(M, nt, dtype=torch.bfloat16, device=X.device)
     if XA is None:
         XA = torch.empty(M, 3 * r, dtype=torch.bfloat16, device=X.device)
-    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
+    _t(X, "X", (M, K))
+    _t(Y, "Y", (M, nt))
+    _t(XA, "XA", (M, 3 * r))
     cq, ck, cv = q.c(), k.c(), v.c()
+    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
     _check("qlora_qkv_fwd", lib().qlora_qkv_fwd(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv), _p(X), M,
                                                 _p(Y), _p(XA), _p(buf), buf.numel(), _stream()))
     return Y, XA
 
 
 def qlora_qkv_bwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, XA, dY, ws: Workspace, grads=None):
-    M, K = X.shape
+    M, K = _rows(X)
     r = q.A.shape[1]
+    nt = q.w.n_out + k.w.n_out + v.w.n_out
     if grads is None:
         grads = {"dX": torch.empty(M, K, dtype=torch.bfloat16, device=X.device)}
         for n, l in (("q", q), ("k", k), ("v", v)):
             grads["dA_" + n] = torch.empty_like(l.A)
             grads["dB_" + n] = torch.empty_like(l.B)
-    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
+    _t(X, "X", (M, K))
+    _t(XA, "XA", (M, 3 * r))
+    _t(dY, "dY", (M, nt))
+    _t(grads["dX"], "dX", (M, K))
+    for n, l in (("q", q), ("k", k), ("v", v)):
+        _t(grads["dA_" + n], "dA_" + n, (K, r))
+        _t(grads["dB_" + n], "dB_" + n, (r, l.w.n_out))
     cq, ck, cv = q.c(), k.c(), v.c()
+    buf = ws.get(qlora_qkv_workspace_bytes(M, K, q.w.n_out, k.w.n_out, v.w.n_out, r))
     outs = [_p(grads[n]) for n in ("dX", "dA_q", "dB_q", "dA_k", "dB_k", "dA_v", "dB_v")]
     _check("qlora_qkv_bwd", lib().qlora_qkv_bwd(ctypes.byref(cq), ctypes.byref(ck), ctypes.byref(cv), _p(X), _p(XA),
                                                 _p(dY), M, *outs, _p(buf), buf.numel(), _stream()))

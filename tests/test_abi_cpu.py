@@ -110,3 +110,26 @@ def test_tile_config_setting(lib):
     assert ops.qlora_set_tile_config(prev) == 1
     assert ops.qlora_set_tile_config(7) == prev  # invalid values are ignored
     assert ops.qlora_set_tile_config(prev) == prev
+
+
+def test_binding_rejects_host_tensors_before_any_library_call():
+    """The C ABI only sees raw pointers: the binding must refuse a host tensor
+    (whose address would be an illegal device access) before calling it."""
+    import torch
+    n, k, r = 512, 256, 16
+    w = ops.NF4Weight(torch.zeros(n * k // 2, dtype=torch.uint8), torch.zeros(n * k // 64, dtype=torch.float32), n, k)
+    lin = ops.LoraLinear(w, torch.zeros(k, r, dtype=torch.bfloat16), torch.zeros(r, n, dtype=torch.bfloat16), 1.0)
+    X = torch.zeros(8, k, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.qlora_linear_fwd(lin, X, ws=None)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.qlora_linear_bwd(lin, X, torch.zeros(8, r, dtype=torch.bfloat16), torch.zeros(8, n, dtype=torch.bfloat16),
+                             ws=None)
+    with pytest.raises(ValueError, match="2-D"):
+        ops.qlora_linear_fwd(lin, X.view(-1), ws=None)
+    down = ops.LoraLinear(ops.NF4Weight(w.codes, w.absmax, k, n), torch.zeros(n, r, dtype=torch.bfloat16),
+                          torch.zeros(r, k, dtype=torch.bfloat16), 1.0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        ops.qlora_mlp_fwd("swiglu", lin, lin, down, X, ws=None)
+    with pytest.raises(ValueError, match="MLP weights"):
+        ops.qlora_mlp_fwd("swiglu", lin, lin, lin, X, ws=None)
