@@ -1,6 +1,7 @@
 """Binding of the plain C oracle (``oracle/c/qlora_oracle.c``): the NF4
-codebook, quantiser and dequantiser and one QLoRA projection's forward and
-hand-derived backward as loops in binary64, for the tiny configuration.
+codebook, quantiser and dequantiser, one QLoRA projection's forward and
+hand-derived backward, and the gated MLP built from three projections, as
+loops in binary64, for small configurations.
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  ``build()`` compiles
 the C file with gcc (ISO C, no fast-math, so binary32 division and products
@@ -20,6 +21,13 @@ LIB = os.path.join(HERE, "c", "libqlora_oracle.so")
 
 _lib = None
 _D = ctypes.POINTER(ctypes.c_double)
+
+
+class _Proj(ctypes.Structure):
+    _fields_ = [("W", _D), ("A", _D), ("B", _D), ("s", ctypes.c_double)]
+
+
+_KIND = {"swiglu": 0, "geglu_tanh": 1}
 
 
 def build():
@@ -42,6 +50,10 @@ def lib():
         L.oracle_c_linear_fwd.argtypes = [_D, _D, _D, _D, ctypes.c_double] + [ctypes.c_long] * 4 + [_D, _D]
         L.oracle_c_linear_bwd.argtypes = ([_D, _D, _D, _D, ctypes.c_double, _D] + [ctypes.c_long] * 4 +
                                           [_D, _D, _D, _D, _D])
+        L.oracle_c_mlp_fwd.argtypes = [ctypes.c_int, _D] + [ctypes.c_long] * 4 + [_Proj] * 3 + [_D] * 4
+        L.oracle_c_mlp_fwd.restype = ctypes.c_int
+        L.oracle_c_mlp_bwd.argtypes = [ctypes.c_int, _D] + [ctypes.c_long] * 4 + [_Proj] * 3 + [_D] * 8
+        L.oracle_c_mlp_bwd.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -96,3 +108,39 @@ def linear_bwd(X, W, A, B, s, dY):
     lib().oracle_c_linear_bwd(_p(X), _p(W), _p(A), _p(B), float(s), _p(dY), M, K, N, r, _p(dX), _p(dA), _p(dB),
                               _p(G), _p(XA))
     return dX, dA, dB
+
+
+def _proj(p, keep):
+    W, A, B = (_f64(a) for a in p[:3])
+    keep.extend((W, A, B))  # the arrays must outlive the call
+    return _Proj(_p(W), _p(A), _p(B), float(p[3])), W.shape, A.shape[1]
+
+
+def mlp_fwd(kind, X, gate, up, down):
+    """Gated MLP forward; gate/up/down are (W, A, B, s).  Returns Y, E, G, H."""
+    keep = []
+    X = _f64(X)
+    M, d = X.shape
+    pg, (h, _), r = _proj(gate, keep)
+    pu, _, _ = _proj(up, keep)
+    pd, _, _ = _proj(down, keep)
+    E, G, H, Y = np.empty((M, h)), np.empty((M, h)), np.empty((M, h)), np.empty((M, d))
+    if lib().oracle_c_mlp_fwd(_KIND[kind], _p(X), M, d, h, r, pg, pu, pd, _p(E), _p(G), _p(H), _p(Y)):
+        raise MemoryError("oracle_c_mlp_fwd")
+    return {"Y": Y, "E": E, "G": G, "H": H}
+
+
+def mlp_bwd(kind, X, gate, up, down, dY):
+    """Gated MLP backward: dX and the six adapter gradients."""
+    keep = []
+    X, dY = _f64(X), _f64(dY)
+    M, d = X.shape
+    pg, (h, _), r = _proj(gate, keep)
+    pu, _, _ = _proj(up, keep)
+    pd, _, _ = _proj(down, keep)
+    out = {"dX": np.empty((M, d)), "dA_g": np.empty((d, r)), "dB_g": np.empty((r, h)), "dA_u": np.empty((d, r)),
+           "dB_u": np.empty((r, h)), "dA_d": np.empty((h, r)), "dB_d": np.empty((r, d))}
+    args = [_p(out[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
+    if lib().oracle_c_mlp_bwd(_KIND[kind], _p(X), M, d, h, r, pg, pu, pd, _p(dY), *args):
+        raise MemoryError("oracle_c_mlp_bwd")
+    return out

@@ -4,8 +4,10 @@ Two independent statements of the same definitions (different languages,
 quantile routines, loop orders and summation orders) must agree: the NF4
 codebook, codes and absmax bit for bit, the dequantised weight exactly, and
 the projection's forward and backward to binary64 rounding on the tiny
-configuration (256 x 512 -> 1024, rank 16).  A mistake in either (a dropped
-LoRA term, a transposed operand, a wrong nibble order or tie rule) fails here.
+configuration (256 x 512 -> 1024, rank 16), and the gated MLP's forward and
+backward (both activations, with derivatives written separately in each) on a
+small MLP.  A mistake in either (a dropped LoRA term, a transposed operand, a
+wrong nibble order or tie rule, a wrong activation derivative) fails here.
 """
 
 import numpy as np
@@ -14,7 +16,7 @@ import pytest
 import oracle
 from oracle import c_oracle
 from oracle.nf4 import nf4_dequantize_f64
-from qlora_fine_tuning_nf4_b200.synth import bf16_bits, make_linear_problem
+from qlora_fine_tuning_nf4_b200.synth import bf16_bits, make_linear_problem, make_mlp_problem
 from qlora_fine_tuning_nf4_b200.workloads import LINEAR_WORKLOADS
 
 
@@ -63,5 +65,27 @@ def test_linear_forward_and_backward_agree():
     c_b = c_oracle.linear_bwd(X, W, A, B, s, dY)
     n_b = oracle.linear_bwd(X, W, A, B, s, dY)
     for name, c, o in [("Y", cy, ny), ("XA", cxa, nxa)] + list(zip(("dX", "dA", "dB"), c_b, n_b)):
+        rms = np.sqrt(np.mean(o * o))
+        assert np.max(np.abs(c - o)) <= 1e-12 * rms, name
+
+
+@pytest.mark.parametrize("kind", ["swiglu", "geglu_tanh"])
+def test_gated_mlp_forward_and_backward_agree(kind):
+    """The C loops' gated MLP (their own activations and derivatives, written
+    from the definitions) against the numpy oracle, on bf16-valued inputs of a
+    small MLP with the pages' structure (d -> h -> d, rank r, s = alpha / r)."""
+    p = make_mlp_problem(48, 256, 512, r=16, alpha=32.0, seed=9)
+    lin = {}
+    for k in ("g", "u", "d"):
+        n, kk = p["W_" + k].shape
+        codes, absmax = oracle.nf4_quantize(p["W_" + k], n, kk)
+        lin[k] = (nf4_dequantize_f64(codes, absmax, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
+                  oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
+    X, dY = oracle.bf16_bits_to_f64(p["X"]), oracle.bf16_bits_to_f64(p["dY"])
+    cf = c_oracle.mlp_fwd(kind, X, lin["g"], lin["u"], lin["d"])
+    nf = oracle.mlp_fwd(kind, X, lin["g"], lin["u"], lin["d"])
+    cb = c_oracle.mlp_bwd(kind, X, lin["g"], lin["u"], lin["d"], dY)
+    nb = oracle.mlp_bwd(kind, X, lin["g"], lin["u"], lin["d"], dY)
+    for name, c, o in [(k, cf[k], nf[k]) for k in ("Y", "E", "G", "H")] + [(k, cb[k], nb[k]) for k in cb]:
         rms = np.sqrt(np.mean(o * o))
         assert np.max(np.abs(c - o)) <= 1e-12 * rms, name
