@@ -21,6 +21,15 @@ TOL = 2e-2  # max |gpu - oracle| <= TOL * RMS(oracle), per tensor (every workloa
 # at M = 200-1024 tokens, because the max over elements of few-row sums is
 # dominated by single heavy-tailed products.  These cases use 3e-2.
 TOL_SMALL_MLP = 3e-2
+# (M, d, h) of the small gated-MLP parity cases (seed M + d + h): several tiles of
+# every kernel, ragged M and a width that is not a multiple of the 256-wide tile.
+# tests/test_tolerance_emulation.py derives TOL_SMALL_MLP on exactly these.
+SMALL_MLP_CASES = [
+    (256, 256, 512),
+    (200, 512, 768),
+    (384, 768, 1280),
+    (1100, 512, 768),
+]
 
 
 def f64(bits):

@@ -16,8 +16,8 @@ import oracle
 from qlora_fine_tuning_nf4_b200 import ops
 from qlora_fine_tuning_nf4_b200.synth import bf16_bits, make_linear_problem, make_mlp_problem
 
-from parity import (TOL_SMALL_MLP, assert_close, assert_saved, gpu_weight, oracle_weight, run_linear_gpu,
-                    run_linear_oracle, run_mlp_gpu, run_mlp_oracle, saved_bounds)
+from parity import (SMALL_MLP_CASES, TOL_SMALL_MLP, assert_close, assert_saved, gpu_weight, oracle_weight,
+                    run_linear_gpu, run_linear_oracle, run_mlp_gpu, run_mlp_oracle, saved_bounds)
 
 pytestmark = pytest.mark.gpu
 
@@ -133,12 +133,7 @@ def test_linear_zero_B_gives_zero_dA(tiles):
 
 # ------------------------------------------------------------------ MLP ----
 
-MLP_CASES = [
-    (256, 256, 512),
-    (200, 512, 768),
-    (384, 768, 1280),
-    (1100, 512, 768),
-]
+MLP_CASES = SMALL_MLP_CASES
 
 
 @pytest.mark.parametrize("tiles", [1, 2, 3, 4])
