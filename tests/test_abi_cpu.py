@@ -133,3 +133,26 @@ def test_binding_rejects_host_tensors_before_any_library_call():
         ops.qlora_mlp_fwd("swiglu", lin, lin, down, X, ws=None)
     with pytest.raises(ValueError, match="MLP weights"):
         ops.qlora_mlp_fwd("swiglu", lin, lin, lin, X, ws=None)
+
+
+def test_workspace_holds_the_staged_weight_only_under_the_staged_feed(lib):
+    """Configuration 4 dequantises each weight once per call into the workspace
+    (n_out * k_in bf16 for a projection, the gate and up weights side by side
+    for the MLP); the in-mainloop configurations and the 16-bit base need no
+    such room."""
+    M, d, h = 8192, 4096, 11008
+    prev = ops.qlora_set_tile_config(4)
+    try:
+        lin4 = ops.qlora_linear_workspace_bytes(M, d, d)
+        mlp4 = ops.qlora_mlp_workspace_bytes(M, d, h)
+        ops.qlora_set_tile_config(2)
+        lin2 = ops.qlora_linear_workspace_bytes(M, d, d)
+        mlp2 = ops.qlora_mlp_workspace_bytes(M, d, h)
+    finally:
+        ops.qlora_set_tile_config(prev)
+    assert lin4 - lin2 >= d * d * 2
+    assert mlp4 - mlp2 >= 2 * h * d * 2
+    assert ops.qlora_linear16_workspace_bytes(M, d, d) < lin4
+    assert ops.qlora_mlp16_workspace_bytes(M, d, h) < mlp4
+    sizes = [ops.qlora_mlp_workspace_bytes(m, d, h) for m in (1, 256, 1024, 8192, 16384)]
+    assert sizes == sorted(sizes)
