@@ -144,7 +144,8 @@ QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t k_in, int64_t n
 /* Forward of one QLoRA projection (Mistral blog "10、11. 手动 Autograd"):
  *   XA = X A                      -> XA_saved [M, r]  (kept for the backward)
  *   Y  = X dequant(W)^T + s XA B  -> Y [M, n_out]
- * X [M, k_in].  Requires k_in % 256 == 0, n_out % 8 == 0, r == 16. */
+ * X [M, k_in].  Requires k_in % 256 == 0, n_out % 8 == 0, and r = 16, 32 or
+ * 64 under tile configuration 4 (the default), r = 16 under 1-3. */
 QLORA_API qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                               qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
@@ -170,7 +171,9 @@ QLORA_API size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int3
  * act = SiLU (QLORA_ACT_SWIGLU) or tanh-approximate GELU
  * (QLORA_ACT_GEGLU_TANH).  gate/up: n_out = h, k_in = d; down: n_out = d,
  * k_in = h.  X [M, d], Y [M, d]; `saved` receives E, G, H, XA_g, XA_u, HA_d.
- * Requires d % 256 == 0, h % 256 == 0, r == 16. */
+ * Requires d % 256 == 0, h % 256 == 0, the same r for the three projections,
+ * and r = 16, 32 or 64 under tile configuration 4 (the default), r = 16 under
+ * 1-3. */
 QLORA_API qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
                            const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                            const qlora_mlp_saved* saved, void* workspace, size_t workspace_bytes,
