@@ -23,3 +23,20 @@ def test_roofline_peak_follows_the_measured_clock():
     assert peak == 1637.6 and "burst" in kind
     peak, kind = bench.tensor_peak(pk, {"sm_mhz": None})
     assert peak == 1390.6 and "no clock record" in kind
+
+
+def test_cpu_baseline_repeats_whole_batches_until_the_target_time():
+    """A batch the probe finds cheap is timed as whole-batch steps repeated
+    until the target has passed, and the FLOP count covers every step."""
+    wl = {"M": 128, "d": 256, "h": 512, "r": 16, "alpha": 16.0, "seed": 0, "act": "swiglu"}
+    dt, flop, cores, rows, steps = bench.oracle_sample(wl, target_s=0.5)
+    assert rows == 128 and steps >= 1 and dt >= 0.5
+    assert flop == steps * bench.mlp_flops(128, 256, 512, 16)
+    assert cores >= 1
+    dt, flop, _, rows, steps = bench.oracle_sample(wl, rows=64)
+    assert rows == 64 and steps == 1 and flop == bench.mlp_flops(64, 256, 512, 16)
+
+
+def test_c_loop_baseline_record():
+    rec = bench.c_loop_oracle_sample()
+    assert rec["value"] > 0 and rec["ms"] > 0 and rec["threads"] == 1 and rec["unit"] == bench.UNIT
