@@ -321,9 +321,8 @@ def run_reference(args, wl):
 def setup_mlp(args, wl, M, d, h, r, act, rank, world, dev):
     """Tensors and step of the gated MLP fwd + bwd (the metric's workload)."""
     import torch
-    import torch.distributed as dist
 
-    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200 import dp, ops
     from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_mlp_problem
 
     # Inputs: same seeded recipe as the tests; each rank draws its own batch.
@@ -343,21 +342,16 @@ def setup_mlp(args, wl, M, d, h, r, act, rank, world, dev):
     ws = ops.Workspace(dev)
     saved = ops.make_mlp_saved(M, h, r, dev)
     Y = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-    # LoRA gradients as views of one flat buffer -> one all-reduce per step
-    sizes = [("dA_g", (d, r)), ("dB_g", (r, h)), ("dA_u", (d, r)), ("dB_u", (r, h)), ("dA_d", (h, r)),
-             ("dB_d", (r, d))]
-    flat = torch.empty(sum(a * b for _, (a, b) in sizes), dtype=torch.bfloat16, device=dev)
-    grads, off = {}, 0
-    for name, (a, b) in sizes:
-        grads[name] = flat[off:off + a * b].view(a, b)
-        off += a * b
+    # LoRA gradients as views of one flat buffer; with N > 1 ranks the four that are final before the gate/up
+    # dX GEMM are summed on a side stream while it runs, the other two after the backward
+    flat, views, early = dp.flat_lora_grads(d, h, r, dev)
+    grads = dict(views)
     grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-
-    def step():
-        mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws, Y=Y, saved=saved)
-        mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads)
-        if world > 1:
-            dist.all_reduce(flat)
+    sync = dp.GradAllReduce(flat, early)
+    step = dp.make_step(lambda: mlp_fwd(act, lins["g"], lins["u"], lins["d"], X, ws, Y=Y, saved=saved),
+                        lambda ev: mlp_bwd(act, lins["g"], lins["u"], lins["d"], X, saved, dY, ws, grads=grads,
+                                           early_event=ev),
+                        sync)
 
     kflops = {k: kernel_flops(k, M, d, h, r) for k in ("gemm_nf4_gateup_glu_fwd", "gemm_nf4_fwd",
                                                          "gemm_nf4_down_bwd_glu", "gemm_nf4_bwd_dx")}
@@ -396,9 +390,8 @@ def setup_norm_mlp(args, wl, M, d, h, r, act, rank, world, dev):
 def setup_qkv(args, wl, M, d, r, rank, world, dev):
     """Tensors and step of the fused Q/K/V projection fwd + bwd at the workload's attention widths."""
     import torch
-    import torch.distributed as dist
 
-    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200 import dp, ops
     from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_qkv_problem
     from qlora_fine_tuning_nf4_b200.workloads import linear_flops
 
@@ -417,18 +410,12 @@ def setup_qkv(args, wl, M, d, r, rank, world, dev):
     XA = torch.empty(M, 3 * r, dtype=torch.bfloat16, device=dev)
     sizes = [(f"d{m}_{n}", (d, r) if m == "A" else (r, wn)) for n, wn in (("q", nq), ("k", nkv), ("v", nkv))
              for m in "AB"]
-    flat = torch.empty(sum(a * b for _, (a, b) in sizes), dtype=torch.bfloat16, device=dev)
-    grads, off = {}, 0
-    for name, (a, b) in sizes:
-        grads[name] = flat[off:off + a * b].view(a, b)
-        off += a * b
+    flat, views, _ = dp.flat_buffer(sizes, dev)
+    grads = dict(views)
     grads["dX"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-
-    def step():
-        ops.qlora_qkv_fwd(lins["q"], lins["k"], lins["v"], X, ws, Y=Y, XA=XA)
-        ops.qlora_qkv_bwd(lins["q"], lins["k"], lins["v"], X, XA, dY, ws, grads=grads)
-        if world > 1:
-            dist.all_reduce(flat)
+    step = dp.make_step(lambda: ops.qlora_qkv_fwd(lins["q"], lins["k"], lins["v"], X, ws, Y=Y, XA=XA),
+                        lambda ev: ops.qlora_qkv_bwd(lins["q"], lins["k"], lins["v"], X, XA, dY, ws, grads=grads),
+                        dp.GradAllReduce(flat))
 
     flop = sum(linear_flops(M, d, n, r) for n in (nq, nkv, nkv))
     kflops = {"gemm_nf4_fwd": 2 * M * d * nt + 2 * M * r * nt, "gemm_nf4_bwd_dx": 2 * M * nt * d + 2 * M * 3 * r * d}
@@ -439,9 +426,8 @@ def setup_qkv(args, wl, M, d, r, rank, world, dev):
 def setup_linear(args, wl, rank, world, dev):
     """Tensors and step of one QLoRA projection fwd + bwd (qlora_linear_fwd / qlora_linear_bwd)."""
     import torch
-    import torch.distributed as dist
 
-    from qlora_fine_tuning_nf4_b200 import ops
+    from qlora_fine_tuning_nf4_b200 import dp, ops
     from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_linear_problem
     from qlora_fine_tuning_nf4_b200.workloads import linear_flops
 
@@ -460,15 +446,11 @@ def setup_linear(args, wl, rank, world, dev):
     ws = ops.Workspace(dev)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     XA = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    flat = torch.empty(K * r + r * N, dtype=torch.bfloat16, device=dev)
-    grads = {"dA": flat[:K * r].view(K, r), "dB": flat[K * r:].view(r, N),
-             "dX": torch.empty(M, K, dtype=torch.bfloat16, device=dev)}
-
-    def step():
-        fwd(lin, X, ws, Y=Y, XA=XA)
-        bwd(lin, X, XA, dY, ws, dX=grads["dX"], dA=grads["dA"], dB=grads["dB"])
-        if world > 1:
-            dist.all_reduce(flat)
+    flat, views, _ = dp.flat_buffer([("dA", (K, r)), ("dB", (r, N))], dev)
+    grads = dict(views, dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev))
+    step = dp.make_step(lambda: fwd(lin, X, ws, Y=Y, XA=XA),
+                        lambda ev: bwd(lin, X, XA, dY, ws, dX=grads["dX"], dA=grads["dA"], dB=grads["dB"]),
+                        dp.GradAllReduce(flat))
 
     kflops = {"gemm_nf4_fwd": 2 * M * K * N + 2 * M * r * N, "gemm_nf4_bwd_dx": 2 * M * N * K + 2 * M * r * K}
     dq = 2 * N * K * (0.5 + 4 / 64 + 2) if args.weights == "nf4" else 0  # the forward's and the backward's
@@ -485,6 +467,8 @@ def run_ours(args, wl):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but {world} rank(s) were started (WORLD_SIZE)")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -562,64 +546,86 @@ def run_ours(args, wl):
     pk = peaks()
 
     # ---- end-to-end through the public API with host buffers ----
-    # Every step copies its inputs (X, dY) from pinned host memory and reads its result (the adapter
-    # gradients, what the optimiser consumes; Y and dX feed neighbouring layers on the device) back to
-    # pinned host memory, inside the timed region.  As a training loop prefetches its next batch, the
-    # next step's inputs are copied on a second stream into the other of two device buffers while the
-    # current step computes; the read-back follows each step on that stream.
+    # Every step copies its inputs (X, dY) from pinned host memory and reads its result back to pinned host
+    # memory, inside the timed region.  `e2e`: the result is the adapter gradients (what the optimiser
+    # consumes; Y and dX feed neighbouring layers on the device).  `e2e_outputs`: Y and dX are read back every
+    # step as well.  As a training loop prefetches its next batch, the next step's inputs are copied on one
+    # copy stream into the other of two device buffers while the current step computes; the read-backs go on
+    # a second copy stream (the two PCIe directions overlap), the gradients first, then Y and dX from the
+    # step's own slot of two output buffers.
+    Yt, dXt = Y, grads["dX"]
     hX = torch.empty(X.shape, dtype=torch.bfloat16, pin_memory=True)
     hdY = torch.empty(dY.shape, dtype=torch.bfloat16, pin_memory=True)
     hX.copy_(X.cpu())
     hdY.copy_(dY.cpu())
-    hflat = torch.empty(flat.numel(), dtype=torch.bfloat16, pin_memory=True)
+    hflat = torch.empty(flat.numel(), dtype=flat.dtype, pin_memory=True)
+    hY = torch.empty(Yt.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdX = torch.empty(dXt.shape, dtype=torch.bfloat16, pin_memory=True)
     bufX = [torch.empty_like(X), torch.empty_like(X)]
     bufdY = [torch.empty_like(dY), torch.empty_like(dY)]
-    copy_stream = torch.cuda.Stream(device=dev)
+    bufY = [torch.empty_like(Yt), torch.empty_like(Yt)]
+    bufdX = [torch.empty_like(dXt), torch.empty_like(dXt)]
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
     ev_in = [torch.cuda.Event(), torch.cuda.Event()]
     ev_used = [torch.cuda.Event(), torch.cuda.Event()]
-    ev_out = torch.cuda.Event()
+    ev_outs = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_grads = torch.cuda.Event()
     e2e_steps = max(3, args.steps)  # as many as the timed region, so that both see the same clocks
 
     def h2d(slot):
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(ev_used[slot])  # the step that last read this buffer is done
+        with torch.cuda.stream(h2d_stream):
+            h2d_stream.wait_event(ev_used[slot])  # the step that last read this buffer is done
             bufX[slot].copy_(hX, non_blocking=True)
             bufdY[slot].copy_(hdY, non_blocking=True)
-            ev_in[slot].record(copy_stream)
+            ev_in[slot].record(h2d_stream)
 
-    def run_e2e(n):
-        copy_stream.wait_stream(stream)
+    def run_e2e(n, outputs):
+        h2d_stream.wait_stream(stream)
+        d2h_stream.wait_stream(stream)
         h2d(0)
         for i in range(n):
             sl = i % 2
             stream.wait_event(ev_in[sl])
             X.set_(bufX[sl])
             dY.set_(bufdY[sl])
+            if outputs:
+                stream.wait_event(ev_outs[sl])  # step i - 2's Y and dX have left this slot
+                Yt.set_(bufY[sl])
+                dXt.set_(bufdX[sl])
             step()
             ev_used[sl].record(stream)
             if i + 1 < n:
                 h2d((i + 1) % 2)
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(ev_used[sl])
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(ev_used[sl])
                 hflat.copy_(flat, non_blocking=True)
-                ev_out.record(copy_stream)
-            stream.wait_event(ev_out)  # the next step's backward rewrites the gradients
-        stream.wait_stream(copy_stream)
+                ev_grads.record(d2h_stream)
+                if outputs:
+                    hY.copy_(bufY[sl], non_blocking=True)
+                    hdX.copy_(bufdX[sl], non_blocking=True)
+                    ev_outs[sl].record(d2h_stream)
+            stream.wait_event(ev_grads)  # the next step's backward rewrites the gradients
+        stream.wait_stream(h2d_stream)
+        stream.wait_stream(d2h_stream)
 
-    run_e2e(2)
-    barrier()
-    e0.record(stream)
-    run_e2e(e2e_steps)
-    e1.record(stream)
-    barrier()
-    ems = e0.elapsed_time(e1)
-    t = torch.tensor([ems], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ems = float(t.item())
-    e2e_value = flop_step * e2e_steps * world / (ems / 1e3) / 1e12
+    def time_e2e(outputs):
+        run_e2e(2, outputs)
+        barrier()
+        e0.record(stream)
+        run_e2e(e2e_steps, outputs)
+        e1.record(stream)
+        barrier()
+        t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return flop_step * e2e_steps * world / (float(t.item()) / 1e3) / 1e12
+
+    e2e_value = time_e2e(False)
+    e2e_out_value = time_e2e(True)
     h2d_bytes = (X.numel() + dY.numel()) * 2
-    d2h_bytes = flat.numel() * 2
+    d2h_bytes = flat.numel() * flat.element_size()
+    d2h_out_bytes = d2h_bytes + (Yt.numel() + dXt.numel()) * 2
 
     # ---- roofline of the dominant kernel (live CUDA-event times) ----
     roof = None
@@ -675,8 +681,13 @@ def run_ours(args, wl):
                    "base_weights": args.weights, "l2": l2_note(args.op, M, d, h, cfg_extra)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "steps": e2e_steps,
-                "io": "inputs X, dY from pinned host memory every step (the next step's copied on a second stream "
-                      "during the current one); result read back every step: the adapter gradients"},
+                "io": "inputs X, dY from pinned host memory every step (the next step's copied on a copy stream "
+                      "during the current one); result read back every step on a second copy stream: the adapter "
+                      "gradients"},
+        "e2e_outputs": {"value": e2e_out_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
+                        "d2h_bytes_per_step": d2h_out_bytes, "steps": e2e_steps,
+                        "io": "as e2e, and Y and dX (the step's own outputs) read back every step too, from two "
+                              "alternating device output buffers"},
         "gpu_launches": launches,
         "roofline": roof,
         "dequant": dq,
@@ -687,8 +698,31 @@ def run_ours(args, wl):
     }), flush=True)
 
 
+def torchrun_command(argv, gpus, port, limit_s=1800):
+    """The command that runs this script as `gpus` ranks on one node (one process per GPU), bounded by
+    `timeout` well above the process group's own 120 s collective timeout."""
+    import shutil
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    if shutil.which("timeout"):
+        cmd = ["timeout", "-k", "60", str(limit_s)] + cmd
+    return cmd
+
+
+def free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
 def main():
     args = parse()
+    if args.impl == "ours" and args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started as a plain process: start the ranks (the driver's torchrun launch sets WORLD_SIZE itself)
+        sys.exit(subprocess.call(torchrun_command(sys.argv[1:], args.gpus, free_port())))
     if (args.op == "linear") != (args.workload in LINEAR_WORKLOADS):
         sys.exit(f"--op {args.op} needs {'a single-projection' if args.op == 'linear' else 'an MLP'} workload")
     if args.op == "linear" and args.impl == "reference":

@@ -57,12 +57,13 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st* qlora_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+typedef struct CUevent_st* qlora_event_t;   /* a cudaEvent_t */
 typedef uint16_t qlora_bf16;                /* bf16 bit pattern */
 
 typedef enum {
   QLORA_OK = 0,
   QLORA_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum */
-  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* k_in % 256 != 0 for the GEMM paths, n_out % 8 != 0, unsupported rank ... */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* k_in % 64 != 0, n_out % 8 != 0, unsupported rank ... */
   QLORA_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
   QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
   QLORA_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
@@ -144,8 +145,10 @@ QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t k_in, int64_t n
 /* Forward of one QLoRA projection (Mistral blog "10、11. 手动 Autograd"):
  *   XA = X A                      -> XA_saved [M, r]  (kept for the backward)
  *   Y  = X dequant(W)^T + s XA B  -> Y [M, n_out]
- * X [M, k_in].  Requires k_in % 256 == 0, n_out % 8 == 0, and r = 16, 32 or
- * 64 under tile configuration 4 (the default), r = 16 under 1-3. */
+ * X [M, k_in].  Requires k_in % 64 == 0 (one NF4 block), n_out % 8 == 0, and
+ * r = 16, 32 or 64 under tile configuration 4 (the default).  Tile
+ * configurations 1-3 further require k_in % 256 == 0 (their GEMM loads each
+ * weight row's absmax values by TMA, in 16-byte pieces) and r = 16. */
 QLORA_API qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                               qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
@@ -171,9 +174,9 @@ QLORA_API size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int3
  * act = SiLU (QLORA_ACT_SWIGLU) or tanh-approximate GELU
  * (QLORA_ACT_GEGLU_TANH).  gate/up: n_out = h, k_in = d; down: n_out = d,
  * k_in = h.  X [M, d], Y [M, d]; `saved` receives E, G, H, XA_g, XA_u, HA_d.
- * Requires d % 256 == 0, h % 256 == 0, the same r for the three projections,
- * and r = 16, 32 or 64 under tile configuration 4 (the default), r = 16 under
- * 1-3. */
+ * Requires d % 64 == 0, h % 256 == 0, the same r for the three projections,
+ * and r = 16, 32 or 64 under tile configuration 4 (the default); tile
+ * configurations 1-3 require d % 256 == 0 and r = 16. */
 QLORA_API qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
                            const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                            const qlora_mlp_saved* saved, void* workspace, size_t workspace_bytes,
@@ -189,6 +192,20 @@ QLORA_API qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gat
                            const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
                            qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* workspace,
                            size_t workspace_bytes, qlora_stream_t stream);
+
+/* qlora_mlp_bwd that also records `early_grads` (a cudaEvent_t created by the
+ * caller; NULL = none) on `stream` as soon as dA_d, dB_d, dB_g and dB_u are
+ * final, before the gate/up dX GEMM is enqueued (for M = 0, after their
+ * memsets).  A data-parallel caller can make a second stream wait for that
+ * event and start summing those four gradients across ranks while the rest of
+ * the backward runs (the pages' DDP gradient sync; Mistral blog, 2 x T4 DDP
+ * tables).  Everything else is exactly qlora_mlp_bwd. */
+QLORA_API qlora_status qlora_mlp_bwd_ev(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                                        const qlora_lora_linear* down, const qlora_bf16* X,
+                                        const qlora_mlp_saved* saved, const qlora_bf16* dY, int64_t M, qlora_bf16* dX,
+                                        qlora_bf16* dA_g, qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u,
+                                        qlora_bf16* dA_d, qlora_bf16* dB_d, void* workspace, size_t workspace_bytes,
+                                        qlora_stream_t stream, qlora_event_t early_grads);
 
 /* The same four computations with bf16 base weights (qlora_lora_linear16):
  * outputs, saved tensors, shapes, workspace rules and errors as the NF4 calls
@@ -216,6 +233,14 @@ QLORA_API qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16*
                                        int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
                                        qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
                                        void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+/* qlora_mlp16_bwd with the `early_grads` event of qlora_mlp_bwd_ev. */
+QLORA_API qlora_status qlora_mlp16_bwd_ev(qlora_act act, const qlora_lora_linear16* gate,
+                                          const qlora_lora_linear16* up, const qlora_lora_linear16* down,
+                                          const qlora_bf16* X, const qlora_mlp_saved* saved, const qlora_bf16* dY,
+                                          int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                                          qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
+                                          void* workspace, size_t workspace_bytes, qlora_stream_t stream,
+                                          qlora_event_t early_grads);
 
 /* Fused Q/K/V projection (the pages' manual-autograd QKV, with grouped-query
  * K/V widths, e.g. Mistral's 4096 / 1024 / 1024): three NF4 projections q, k,
@@ -228,7 +253,7 @@ QLORA_API qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16*
  *   dX = sum_p dY_p dequant(W_p) + s_p (dY_p B_p^T) A_p^T   (one GEMM over the
  *   concatenated reduction, three LoRA steps), dA_p, dB_p as qlora_linear_bwd.
  * Requires nq % 256 == 0 and nk % 256 == 0 (an output tile never spans two
- * projections), k_in % 256 == 0, r in {16, 32, 64}.  Always runs the staged
+ * projections), k_in % 64 == 0, r in {16, 32, 64}.  Always runs the staged
  * feed (tile configuration 4); the workspace also holds the stacked bf16
  * weight ((nq + nk + nv) * k_in * 2 bytes). */
 QLORA_API size_t qlora_qkv_workspace_bytes(int64_t M, int64_t k_in, int64_t nq, int64_t nk, int64_t nv, int32_t r);
@@ -272,6 +297,37 @@ QLORA_API qlora_status qlora_last_device_status(void* workspace, qlora_stream_t 
  * the timeout, and the next call computes normally. */
 QLORA_API qlora_status qlora_test_inject_timeout(void);
 
+/* Test hook (not needed in normal use; host side, not thread-safe): caps the
+ * number of CTAs of every persistent launch -- the GEMMs (rounded down to
+ * whole CTA pairs), the rank-side passes and the weight dequantisation -- at
+ * `max_ctas` (0 = no cap, the default; negative values are ignored).  With a
+ * small cap every CTA or CTA pair walks many output tiles and work units on
+ * small problems, so tests reach the persistent scheduling paths (accumulator
+ * ping-pong, ring phases across tiles, tile-group wrap, multi-unit ranges)
+ * without full-size inputs.  Results stay within the same tolerance; the
+ * rank-side sums may change in their last bits because their split changes.
+ * Workspace queries follow the cap current when they are called.  Returns the
+ * previous cap. */
+QLORA_API int32_t qlora_test_set_grid_cap(int32_t max_ctas);
+
+/* Checked debug build.  lib/libqlora_check.so is the same library compiled
+ * with QLORA_CHECK: its kernels check the indices they derive from their
+ * arguments (partial-sum slots and groups of the rank-side passes and their
+ * reduction, the GEMMs' tile-walk arguments) and, on a failed check, record
+ * QL_DEV_BAD_CONFIG in the workspace status word and skip the access instead
+ * of touching memory out of range; nothing traps.  qlora_last_device_status
+ * then returns QLORA_ERR_DEVICE.  In the normal build the checks compile away.
+ * qlora_checked_build returns 1 in the checked build, 0 otherwise. */
+QLORA_API int32_t qlora_checked_build(void);
+
+/* Test hook for the checked build (host side, one shot): the next rank-side
+ * pass whose plan gives some output group more than one partial slot tells
+ * its kernels one slot fewer than planned.  The partial buffer keeps the
+ * planned size, so every access stays inside the workspace; the checked build
+ * reports the mismatch (QLORA_ERR_DEVICE), the normal build silently computes
+ * wrong adapter values for that call. */
+QLORA_API qlora_status qlora_test_shrink_next_slot_cap(void);
+
 /* Human-readable name of a status code (static string). */
 QLORA_API const char* qlora_status_string(qlora_status status);
 
@@ -308,17 +364,25 @@ QLORA_API uint64_t qlora_launch_count(void);
  * that owns all device memory, or a path where allocating is not permitted.
  * (The pages describe no such call; it has no counterpart there.)
  * Its scratch is a fixed 4 MiB array inside the library that every GPU which
- * loads the library keeps until the process exits; problems that need more
- * (M above about 43,000 rows) return QLORA_ERR_WORKSPACE_TOO_SMALL before
- * anything is enqueued.  It allocates nothing and frees nothing.
+ * loads the library keeps until the process exits.  A call uses at most
+ * 256 + 32 M + 4096 ceil(M / 64) bytes of it (each term rounded up to a
+ * multiple of 256): the status word, the s-scaled X A and the partial sums of
+ * the X A pass.  So M <= 43,648 rows is accepted for any k_in, and larger M
+ * returns QLORA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  It
+ * allocates nothing and frees nothing.
+ * The fixed array has no room for a staged weight, so this call always runs a
+ * GEMM that dequantises the weight in its mainloop: tile configuration 2 when
+ * configuration 4 (the default) is selected, else the selected 1-3.  Those
+ * take rank-16 adapters only; other ranks return QLORA_ERR_UNSUPPORTED_SHAPE
+ * before anything is enqueued.
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array: calls whose GPU work overlaps (on
- * different streams, or from different threads) race and must not be issued.
- * Each call zeroes the status word it uses; device-side timeouts are recorded
- * there and are not reported back through this call.  The fixed array has no
- * room for a staged weight, so under tile configuration 4 this call uses
- * configuration 2 (weight dequantised in the GEMM mainloop). */
+ * device current) and caches it by device ordinal for the life of the
+ * process; make that first call before any stream capture.  The cached
+ * address does not survive cudaDeviceReset: do not use this call on a device
+ * after resetting it.  All calls share the one array: calls whose GPU work
+ * overlaps (on different streams, or from different threads) race and must
+ * not be issued.  Each call zeroes the status word it uses; device-side
+ * timeouts are recorded there and are not reported back through this call. */
 QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M,
                                                 qlora_bf16* Y, qlora_bf16* XA_saved, qlora_stream_t stream);
 

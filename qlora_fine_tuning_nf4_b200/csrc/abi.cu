@@ -32,12 +32,13 @@ cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, co
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
 cudaError_t arm_inject_timeout();
-cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st);
+cudaError_t launch_reduce(const ReduceJob* jobs, int n, cudaStream_t st);
 cudaError_t launch_rmsnorm_fwd(const bf16* X, const bf16* w, int M, int d, float eps, int plus_one, bf16* Y,
                                float* rstd, cudaStream_t st);
 cudaError_t launch_rmsnorm_bwd(const bf16* X, const bf16* w, const float* rstd, const bf16* dY, int M, int d,
                                int plus_one, bf16* dX, cudaStream_t st);
 extern const uint32_t h_nf4_bits[16];
+int g_grid_cap = 0;
 }  // namespace ql
 
 using namespace ql;
@@ -192,7 +193,8 @@ bool map_bf16(CUtensorMap* m, const void* p, int64_t cols, int64_t rows, int64_t
 // shrinks when wide factor tiles limit residency).
 int skinny_target_ctas(int factor_cols) {
   const int smem = 4 * (8192 + 128 * factor_cols) + 64 + 1024;
-  return num_sms() * std::max(1, std::min(4, 232448 / smem));  // the device's SMs (148 when none is present)
+  // the device's SMs (148 when none is present)
+  return apply_grid_cap(num_sms() * std::max(1, std::min(4, 232448 / smem)), 1);
 }
 
 // Partition of `groups` output groups of `upg` units each over the CTAs:
@@ -218,8 +220,10 @@ SkPlan plan_skinny(int64_t groups, int64_t upg, int target) {
 }
 constexpr int kDyCC = 4;  // column chunks of 64 per dypass unit (matches the kernel)
 // rowproj: T [M, K] times factors of `fcols` columns in all; reduction over K (padded to 64)
-SkPlan plan_rowproj(int64_t M, int64_t K, int fcols) {
-  return plan_skinny(cdiv(M, 64), cdiv(K, 64), skinny_target_ctas(fcols));
+// `target` > 0 overrides the CTA count (at most one CTA per 64-row group then
+// gives every group a single partial slot).
+SkPlan plan_rowproj(int64_t M, int64_t K, int fcols, int target = 0) {
+  return plan_skinny(cdiv(M, 64), cdiv(K, 64), target > 0 ? target : skinny_target_ctas(fcols));
 }
 SkPlan plan_colproj(int64_t M, int64_t ncols, int R) {
   return plan_skinny(cdiv(ncols, 64), cdiv(M, 64), skinny_target_ctas(R));
@@ -227,8 +231,8 @@ SkPlan plan_colproj(int64_t M, int64_t ncols, int R) {
 SkPlan plan_dypass(int64_t M, int64_t N) {
   return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64), skinny_target_ctas(32));
 }
-size_t rowproj_part_bytes(int64_t M, int64_t K, int R) {
-  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K, R).slot_cap * 64 * R * 4;
+size_t rowproj_part_bytes(int64_t M, int64_t K, int R, int target = 0) {
+  return static_cast<size_t>(cdiv(M, 64)) * plan_rowproj(M, K, R, target).slot_cap * 64 * R * 4;
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
   R = R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 128));  // the kernel's tile width
@@ -243,6 +247,19 @@ size_t dypass_part_bytes(int64_t M, int64_t N, int r) {
   const int64_t ncb = cdiv(cdiv(N, 64), kDyCC);
   return dypass_gpart_bytes(M, N) + static_cast<size_t>(ncb) * plan_dypass(M, N).slot_cap * kDyCC * 64 * 16 * 4;
 }
+// Test hook (qlora_test_shrink_next_slot_cap): the next skinny pass whose plan
+// gives some group more than one partial slot tells its kernels one slot fewer
+// than the plan has (the partial buffer keeps the plan's size, so every access
+// stays inside it).  The checked build's kernels then report QL_DEV_BAD_CONFIG.
+int g_shrink_slot_cap = 0;
+int planned_slot_cap(int cap) {
+  if (g_shrink_slot_cap && cap > 1) {
+    g_shrink_slot_cap = 0;
+    return cap - 1;
+  }
+  return cap;
+}
+
 ReduceJob reduce_job(float* part, int64_t groups, int grows, int64_t rows, int R, int slot_cap, int nslots,
                      const SkPart& sp, const ReduceOuts& outs) {
   ReduceJob j;
@@ -273,26 +290,51 @@ bool map_factor(CUtensorMap* m, const void* p, int64_t rows, int cols, int64_t l
   return map_bf16(m, p, cols, rows, ld, subw, 64, swz);
 }
 
+// Reductions collected for one launch: those of passes whose results nothing
+// reads until later, each with its own partial region.
+struct ReduceBatch {
+  ReduceJob j[kMaxReduceJobs];
+  int n = 0;
+};
+// Runs the reductions of a pass now, or appends them to `batch` (flush_reduce launches them).
+qlora_status reduce_now_or_later(const ReduceJob* jobs, int n, ReduceBatch* batch, cudaStream_t st) {
+  if (batch) {
+    if (batch->n + n > kMaxReduceJobs) return QLORA_ERR_CUDA;  // planning error inside the library
+    for (int i = 0; i < n; ++i) batch->j[batch->n++] = jobs[i];
+    return QLORA_OK;
+  }
+  KScope k(K_REDUCE, st);
+  return cuda_status(launch_reduce(jobs, n, st));
+}
+qlora_status flush_reduce(ReduceBatch& b, cudaStream_t st) {
+  if (b.n == 0) return QLORA_OK;
+  KScope k(K_REDUCE, st);
+  const qlora_status s = cuda_status(launch_reduce(b.j, b.n, st));
+  b.n = 0;
+  return s;
+}
+
 // P = T V (V = up to three [K, r] LoRA A factors side by side) -> outs (bf16, optional scaled copies)
 qlora_status pass_rowproj(const bf16* T, int64_t M, int64_t K, const bf16* V0, const bf16* V1, int r, float* part,
-                          ReduceOuts outs, int* status, cudaStream_t st, const bf16* V2 = nullptr) {
+                          ReduceOuts outs, int* status, cudaStream_t st, const bf16* V2 = nullptr,
+                          int target = 0) {
   CUtensorMap mt, mv0, mv1, mv2;
   const int nv = V2 ? 3 : (V1 ? 2 : 1);
   if (!map_bf16(&mt, T, K, M, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_factor(&mv0, V0, K, r, r)) return QLORA_ERR_CUDA;
   if (!map_factor(&mv1, V1 ? V1 : V0, K, r, r)) return QLORA_ERR_CUDA;
   if (!map_factor(&mv2, V2 ? V2 : V0, K, r, r)) return QLORA_ERR_CUDA;
-  const SkPlan p = plan_rowproj(M, K, nv * r);
+  const SkPlan p = plan_rowproj(M, K, nv * r, target);
   const int64_t nrc = cdiv(M, 64);
-  const ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, p.slot_cap, 0, p.sp, outs);
+  ReduceJob j = reduce_job(part, nrc, 64, M, nv * r, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
+  j.status = status;
   {
     KScope k(K_ROWPROJ, st);
     const qlora_status s =
         cuda_status(launch_rowproj(r, nv, false, mt, mv0, mv1, mv2, j, (int)cdiv(K, 64), status, st));
     if (s != QLORA_OK) return s;
   }
-  KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(j, nullptr, st));
+  return reduce_now_or_later(&j, 1, nullptr, st);
 }
 
 // G = T B^T (B = LoRA right factor [r, N]) -> outs
@@ -303,14 +345,14 @@ qlora_status pass_rowproj_bt(const bf16* T, int64_t M, int64_t N, const bf16* B,
   if (!map_bf16(&mb, B, N, r, N, 64, r, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   const SkPlan p = plan_rowproj(M, N, r);
   const int64_t nrc = cdiv(M, 64);
-  const ReduceJob j = reduce_job(part, nrc, 64, M, r, p.slot_cap, 0, p.sp, outs);
+  ReduceJob j = reduce_job(part, nrc, 64, M, r, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
+  j.status = status;
   {
     KScope k(K_ROWPROJ, st);
     const qlora_status s = cuda_status(launch_rowproj(r, 1, true, mt, mb, mb, mb, j, (int)cdiv(N, 64), status, st));
     if (s != QLORA_OK) return s;
   }
-  KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(j, nullptr, st));
+  return reduce_now_or_later(&j, 1, nullptr, st);
 }
 
 // Supported factor-tile widths of the colproj kernel: R rounded up to 16, 32, 64 or 128.
@@ -318,28 +360,30 @@ int colproj_width(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 :
 
 // Q = T^T U (U [M, R] with row stride ldu, R <= 128) -> outs
 qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U, int R, float* part,
-                          ReduceOuts outs, int* status, cudaStream_t st, int64_t ldt = 0, int64_t ldu = 0) {
+                          ReduceOuts outs, int* status, cudaStream_t st, int64_t ldt = 0, int64_t ldu = 0,
+                          ReduceBatch* batch = nullptr) {
   CUtensorMap mt, mu;
   if (!map_bf16(&mt, T, ncols, M, ldt ? ldt : ncols, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
   if (!map_factor(&mu, U, M, R, ldu ? ldu : R, colproj_width(R))) return QLORA_ERR_CUDA;
   R = colproj_width(R);
   const SkPlan p = plan_colproj(M, ncols, R);
   const int64_t ncc = cdiv(ncols, 64);
-  const ReduceJob j = reduce_job(part, ncc, 64, ncols, R, p.slot_cap, 0, p.sp, outs);
+  ReduceJob j = reduce_job(part, ncc, 64, ncols, R, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
+  j.status = status;
   {
     KScope k(K_COLPROJ, st);
     const qlora_status s = cuda_status(launch_colproj(R, mt, mu, j, (int)cdiv(M, 64), status, st));
     if (s != QLORA_OK) return s;
   }
-  KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(j, nullptr, st));
+  return reduce_now_or_later(&j, 1, batch, st);
 }
 
 // G = T Bl^T ([M, r]) and Q = T^T U ([N, r]) for T [M, N]: one fused read of T
-// at rank 16, a G pass and a Q pass at larger ranks.
+// at rank 16 (its two reductions may go to `batch`), a G pass and a Q pass at
+// larger ranks (which reuse `part`, so they are reduced at once).
 qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, const bf16* Bl, int r, float* part,
                          ReduceOuts gouts, ReduceOuts qouts, int* status, cudaStream_t st, int64_t ldt = 0,
-                         int64_t ldu = 0) {
+                         int64_t ldu = 0, ReduceBatch* batch = nullptr) {
   if (r != 16) {
     const qlora_status s = pass_rowproj_bt(T, M, N, Bl, r, part, gouts, status, st, ldt);
     if (s != QLORA_OK) return s;
@@ -353,15 +397,16 @@ qlora_status pass_dypass(const bf16* T, int64_t M, int64_t N, const bf16* U, con
   const int64_t nrc = cdiv(M, 64), nch = cdiv(N, 64), ncb = cdiv(nch, kDyCC);
   float* gpart = part;
   float* qpart = reinterpret_cast<float*>(reinterpret_cast<char*>(part) + dypass_gpart_bytes(M, N));
-  const ReduceJob jg = reduce_job(gpart, nrc, 64, M, 16, (int)ncb, (int)ncb, p.sp, gouts);
-  const ReduceJob jq = reduce_job(qpart, ncb, kDyCC * 64, N, 16, p.slot_cap, 0, p.sp, qouts);
+  ReduceJob jg = reduce_job(gpart, nrc, 64, M, 16, (int)ncb, (int)ncb, p.sp, gouts);
+  ReduceJob jq = reduce_job(qpart, ncb, kDyCC * 64, N, 16, planned_slot_cap(p.slot_cap), 0, p.sp, qouts);
+  jg.status = jq.status = status;
   {
     KScope k(K_DYPASS, st);
     const qlora_status s = cuda_status(launch_dypass(mt, mu, mb, jg, jq, (int)nch, status, st));
     if (s != QLORA_OK) return s;
   }
-  KScope k(K_REDUCE, st);
-  return cuda_status(launch_reduce(jg, &jq, st));
+  const ReduceJob both[2] = {jg, jq};
+  return reduce_now_or_later(both, 2, batch, st);
 }
 
 // One reduction output: columns [col0, col0 + width) of the partials, scaled, bf16
@@ -475,7 +520,11 @@ qlora_status check_linear(const Lin* lin, int tiles) {
   if (lin->w.w16 ? false : (!lin->w.codes || !lin->w.absmax)) return QLORA_ERR_INVALID_ARG;
   if (lin->w.n_out <= 0 || lin->w.k_in <= 0) return QLORA_ERR_INVALID_ARG;
   if (!rank_ok(lin->r, tiles)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (lin->w.k_in % 256 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (lin->w.k_in % 64 || lin->w.n_out % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  // The feeds that dequantise in the GEMM mainloop load each weight row's
+  // absmax values by TMA, whose row stride (k_in / 64 binary32 values) must be
+  // a multiple of 16 bytes.
+  if (!is_staged(tiles) && !lin->w.w16 && lin->w.k_in % 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (lin->w.k_in > kMaxDim || lin->w.n_out > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (misaligned(lin->w.codes) || misaligned(lin->w.absmax) || misaligned(lin->w.w16) || misaligned(lin->A) ||
       misaligned(lin->B))
@@ -540,6 +589,19 @@ qlora_status qlora_nf4_codebook(float out[16]) {
   if (!out) return QLORA_ERR_INVALID_ARG;
   for (int i = 0; i < 16; ++i) std::memcpy(&out[i], &h_nf4_bits[i], 4);
   return QLORA_OK;
+}
+
+int32_t qlora_checked_build(void) { return kChecked ? 1 : 0; }
+
+qlora_status qlora_test_shrink_next_slot_cap(void) {
+  g_shrink_slot_cap = 1;
+  return QLORA_OK;
+}
+
+int32_t qlora_test_set_grid_cap(int32_t max_ctas) {
+  const int32_t prev = g_grid_cap;
+  if (max_ctas >= 0) g_grid_cap = max_ctas;
+  return prev;
 }
 
 int32_t qlora_set_tile_config(int32_t tiles) {
@@ -701,6 +763,10 @@ static qlora_status linear_bwd(const Lin* lin, int tiles, const qlora_bf16* X, c
 }
 
 namespace {
+// The backward reduces the dA_d pass and the two passes over dE and dG in one
+// launch, so their partials sit side by side: [dA_d | dE pass | dG pass].
+size_t mlp_bwd_part_dad(int64_t M, int64_t h, int r) { return align256(colproj_part_bytes(M, h, r)); }
+size_t mlp_bwd_part_dy(int64_t M, int64_t h, int r) { return align256(dypass_part_bytes(M, h, r)); }
 // MLP workspace: [status | 256 B][dE][dG][5 rank vectors][partials][two staged weights, if `stage`]
 size_t mlp_ws(int64_t M, int64_t d, int64_t h, int r, bool stage) {
   const size_t big = align256(static_cast<size_t>(M) * h * 2);
@@ -708,8 +774,7 @@ size_t mlp_ws(int64_t M, int64_t d, int64_t h, int r, bool stage) {
   size_t part = rowproj_part_bytes(M, d, 2 * r);
   part = std::max(part, rowproj_part_bytes(M, h, r));
   part = std::max(part, dypass_part_bytes(M, d, r));
-  part = std::max(part, dypass_part_bytes(M, h, r));
-  part = std::max(part, colproj_part_bytes(M, h, r));
+  part = std::max(part, mlp_bwd_part_dad(M, h, r) + 2 * mlp_bwd_part_dy(M, h, r));
   part = std::max(part, colproj_part_bytes(M, d, 2 * r));
   return 256 + 2 * big + 5 * vec + align256(part) + (stage ? 2 * stage_bytes(h, d) : 0);
 }
@@ -840,7 +905,7 @@ static qlora_status mlp_fwd(qlora_act act, const Lin* gate, const Lin* up, const
 static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const Lin* down, int tiles, const qlora_bf16* X,
                      const qlora_mlp_saved* sv, const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g,
                      qlora_bf16* dB_g, qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d,
-                     void* ws, size_t ws_bytes, qlora_stream_t stream) {
+                     void* ws, size_t ws_bytes, qlora_stream_t stream, qlora_event_t early = nullptr) {
   if (act != QLORA_ACT_SWIGLU && act != QLORA_ACT_GEGLU_TANH) return QLORA_ERR_INVALID_ARG;
   qlora_status s = check_mlp(gate, up, down, tiles);
   if (s != QLORA_OK) return s;
@@ -849,7 +914,11 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     const int64_t dm = gate->w.k_in, hm = gate->w.n_out, rm = gate->r;
     qlora_bf16* g[6] = {dA_g, dB_g, dA_u, dB_u, dA_d, dB_d};
     const int64_t n[6] = {dm * rm, rm * hm, dm * rm, rm * hm, hm * rm, rm * dm};
-    return zero_adapter_grads(g, n, 6, reinterpret_cast<cudaStream_t>(stream));
+    s = zero_adapter_grads(g, n, 6, reinterpret_cast<cudaStream_t>(stream));
+    if (s == QLORA_OK && early &&
+        cudaEventRecord(reinterpret_cast<cudaEvent_t>(early), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return s;
   }
   if (!X || !sv || !sv->E || !sv->G || !sv->H || !sv->XA_g || !sv->XA_u || !sv->HA_d || !dY || !dX || !dA_g ||
       !dB_g || !dA_u || !dB_u || !dA_d || !dB_d || !ws)
@@ -906,18 +975,31 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
     if (s != QLORA_OK) return s;
   }
   // 3. dA_d = H^T (s_d G_d)
-  s = pass_colproj(reinterpret_cast<const bf16*>(sv->H), M, h, sGd, r, w.part,
-                   routs(rout(reinterpret_cast<bf16*>(dA_d), 0, r, r, 0, 1.f)), w.status, st);
-  if (s != QLORA_OK) return s;
   // 4. G_g = dE B_g^T, dB_g = s_g XA_g^T dE ; G_u = dG B_u^T, dB_u = s_u XA_u^T dG
-  s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), r,
-                  w.part, routs(rout(w.gu, 0, r, 2 * r, 0, gate->scale)),
-                  routs(rout(reinterpret_cast<bf16*>(dB_g), 0, r, (int)h, 1, gate->scale)), w.status, st);
-  if (s != QLORA_OK) return s;
-  s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), r,
-                  w.part, routs(rout(w.gu + r, 0, r, 2 * r, 0, up->scale)),
-                  routs(rout(reinterpret_cast<bf16*>(dB_u), 0, r, (int)h, 1, up->scale)), w.status, st);
-  if (s != QLORA_OK) return s;
+  // Nothing reads dA_d before the end of the call, so its partial sums are
+  // reduced in one launch with those of the two passes of step 4.
+  {
+    ReduceBatch rb;
+    float* part_dad = w.part;
+    float* part_de = reinterpret_cast<float*>(reinterpret_cast<char*>(w.part) + mlp_bwd_part_dad(M, h, r));
+    float* part_dg = reinterpret_cast<float*>(reinterpret_cast<char*>(part_de) + mlp_bwd_part_dy(M, h, r));
+    s = pass_colproj(reinterpret_cast<const bf16*>(sv->H), M, h, sGd, r, part_dad,
+                     routs(rout(reinterpret_cast<bf16*>(dA_d), 0, r, r, 0, 1.f)), w.status, st, 0, 0, &rb);
+    if (s != QLORA_OK) return s;
+    s = pass_dypass(w.dE, M, h, reinterpret_cast<const bf16*>(sv->XA_g), reinterpret_cast<const bf16*>(gate->B), r,
+                    part_de, routs(rout(w.gu, 0, r, 2 * r, 0, gate->scale)),
+                    routs(rout(reinterpret_cast<bf16*>(dB_g), 0, r, (int)h, 1, gate->scale)), w.status, st, 0, 0,
+                    &rb);
+    if (s != QLORA_OK) return s;
+    s = pass_dypass(w.dG, M, h, reinterpret_cast<const bf16*>(sv->XA_u), reinterpret_cast<const bf16*>(up->B), r,
+                    part_dg, routs(rout(w.gu + r, 0, r, 2 * r, 0, up->scale)),
+                    routs(rout(reinterpret_cast<bf16*>(dB_u), 0, r, (int)h, 1, up->scale)), w.status, st, 0, 0,
+                    &rb);
+    if (s != QLORA_OK) return s;
+    if ((s = flush_reduce(rb, st)) != QLORA_OK) return s;
+  }
+  // dA_d, dB_d, dB_g and dB_u are final: a data-parallel caller may start summing them across ranks
+  if (early && cudaEventRecord(reinterpret_cast<cudaEvent_t>(early), st) != cudaSuccess) return QLORA_ERR_CUDA;
   // 5. dX = [dE | dG] [W_g ; W_u] + [sG_g | sG_u] [A_g^T ; A_u^T]
   {
     GemmMaps maps;
@@ -1208,6 +1290,17 @@ qlora_status qlora_mlp_bwd(qlora_act act, const qlora_lora_linear* gate, const q
                  stream);
 }
 
+qlora_status qlora_mlp_bwd_ev(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
+                              const qlora_lora_linear* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
+                              const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                              qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
+                              size_t ws_bytes, qlora_stream_t stream, qlora_event_t early_grads) {
+  if (!gate || !up || !down) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_bwd(act, &g, &u, &d, g_tiles, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes,
+                 stream, early_grads);
+}
+
 // 16-bit entry points: bf16 base weights, always the staged-feed pair tile
 // (the weight is already what the GEMM streams; nothing is dequantised).
 size_t qlora_linear16_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
@@ -1248,6 +1341,16 @@ qlora_status qlora_mlp16_bwd(qlora_act act, const qlora_lora_linear16* gate, con
   if (!gate || !up || !down || !gate->w || !up->w || !down->w) return QLORA_ERR_INVALID_ARG;
   const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
   return mlp_bwd(act, &g, &u, &d, 4, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes, stream);
+}
+qlora_status qlora_mlp16_bwd_ev(qlora_act act, const qlora_lora_linear16* gate, const qlora_lora_linear16* up,
+                                const qlora_lora_linear16* down, const qlora_bf16* X, const qlora_mlp_saved* sv,
+                                const qlora_bf16* dY, int64_t M, qlora_bf16* dX, qlora_bf16* dA_g, qlora_bf16* dB_g,
+                                qlora_bf16* dA_u, qlora_bf16* dB_u, qlora_bf16* dA_d, qlora_bf16* dB_d, void* ws,
+                                size_t ws_bytes, qlora_stream_t stream, qlora_event_t early_grads) {
+  if (!gate || !up || !down || !gate->w || !up->w || !down->w) return QLORA_ERR_INVALID_ARG;
+  const Lin g = lin_of(*gate), u = lin_of(*up), d = lin_of(*down);
+  return mlp_bwd(act, &g, &u, &d, 4, X, sv, dY, M, dX, dA_g, dB_g, dA_u, dB_u, dA_d, dB_d, ws, ws_bytes, stream,
+                 early_grads);
 }
 
 qlora_status qlora_test_inject_timeout(void) {
@@ -1349,7 +1452,14 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const ql
   if (M > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int64_t K = lin->w.k_in;
   const size_t vec = align256(static_cast<size_t>(M) * 32);
-  const size_t need = 256 + vec + align256(rowproj_part_bytes(M, K, 16));
+  // The X A pass normally splits its work over all resident CTAs, which can
+  // give a 64-row group several partial sums.  When those do not fit, each
+  // group goes to one CTA (one partial per group), so the scratch needed is
+  // 256 + 32 M + 4096 ceil(M / 64) bytes (rounded up to 256) for any k_in.
+  int target = 0;
+  if (256 + vec + align256(rowproj_part_bytes(M, K, 16)) > kNoAllocScratchBytes)
+    target = static_cast<int>(std::min<int64_t>(cdiv(M, 64), skinny_target_ctas(16)));
+  const size_t need = 256 + vec + align256(rowproj_part_bytes(M, K, 16, target));
   if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   void* base = nullptr;
   if ((s = noalloc_scratch(&base)) != QLORA_OK) return s;
@@ -1363,7 +1473,7 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_lora_linear* lin_nf4, const ql
   float* part = reinterpret_cast<float*>(w + 256 + vec);
   s = pass_rowproj(reinterpret_cast<const bf16*>(X), M, K, reinterpret_cast<const bf16*>(lin->A), nullptr, 16, part,
                    routs(rout(xa, 0, 16, 16, 0, 1.f), rout(XAs != xa ? XAs : nullptr, 0, 16, 16, 0, lin->scale)),
-                   status, st);
+                   status, st, nullptr, target);
   if (s != QLORA_OK) return s;
   return gemm_fwd(*lin, reinterpret_cast<const bf16*>(X), M, XAs, reinterpret_cast<bf16*>(Y), status, tiles, nullptr,
                   st);

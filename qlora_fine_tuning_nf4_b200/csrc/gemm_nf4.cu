@@ -186,6 +186,16 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
   const int cluster = blockIdx.x / CG;
   const int clusters = gridDim.x / CG;
   const int nk = args.nkb0 + args.nkb1;
+  // Checked build: the arguments the tile walk and the rings depend on.  They are
+  // the same for every CTA, so on failure the whole grid leaves here, before any
+  // barrier, TMEM or cluster operation.
+  if (!dev_check(args.M > 0 && args.N > 0 && args.nkb0 > 0 && args.nkb1 >= 0 && args.group_m >= 1 &&
+                     args.lora >= 0 && args.lora <= (ST ? 3 : 2) && args.ldo >= args.N &&
+                     (!ST || args.lora == 0 || (args.lora_k16 >= 1 && args.lora_k16 <= 4)),
+                 args.status)) {
+    grid_dep_wait();
+    return;
+  }
 
   // barriers
   const uint32_t bar0 = sbase + C::OFF_BAR;
@@ -843,7 +853,7 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& args, cudaSt
     resident[dev] = n * CG;
   }
   const int total = m_tiles * n_tiles;
-  const int ctas = (total * CG < resident[dev]) ? total * CG : resident[dev];
+  const int ctas = apply_grid_cap((total * CG < resident[dev]) ? total * CG : resident[dev], CG);
   cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
   return cudaLaunchKernelEx(&cfg, kern, maps, args);
 }

@@ -11,6 +11,17 @@ namespace ql {
 
 using bf16 = __nv_bfloat16;
 
+// Upper bound on the CTAs of every persistent launch (GEMM, skinny passes,
+// weight dequantisation); 0 = none.  Set only by the test hook
+// qlora_test_set_grid_cap, so that small problems make every CTA (pair) walk
+// several tiles or work units.
+extern int g_grid_cap;
+inline int apply_grid_cap(int ctas, int multiple) {
+  if (g_grid_cap <= 0 || ctas <= g_grid_cap) return ctas;
+  const int c = g_grid_cap - g_grid_cap % multiple;
+  return c > multiple ? c : multiple;
+}
+
 // ------------------------------------------------------------------ GEMM ---
 // D = A * op(dequant(W)) + LoRA, on tcgen05 tensor cores.
 //   MODE_FWD:     reduction over k_in, W [N, K] is the K-major B operand.
@@ -107,7 +118,11 @@ struct ReduceJob {
   int groups, grows, rows, R, slot_cap, nslots;
   SkPart sp;
   ReduceOuts outs;
+  int* status;  // device status word (the checked build's bounds checks report there)
 };
+
+// Reductions one launch of the reduction kernel can serve.
+constexpr int kMaxReduceJobs = 6;
 
 // Launch with programmatic stream serialisation (the kernel calls
 // grid_dep_wait() before reading what earlier kernels wrote).

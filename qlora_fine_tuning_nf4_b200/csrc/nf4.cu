@@ -21,38 +21,70 @@ const uint32_t h_nf4_bits[16] = {0xbf800000u, 0xbf3239b1u, 0xbf066b2eu, 0xbeca32
                                  0xbdba7869u, 0x00000000u, 0x3da2fb01u, 0x3e24cadfu, 0x3e7c04dau, 0x3ead0336u,
                                  0x3ee1a4b5u, 0x3f1007a9u, 0x3f3913b0u, 0x3f800000u};
 
-// One warp per 64-element block: lane l owns elements 2l and 2l+1.
-// absmax = max |w| (exact); v = w / absmax rounded once to binary32; the
-// level index is the number of midpoints (exact in binary64) strictly below
-// v, so a value on a midpoint takes the lower level; absmax 0 -> level 7.
-__global__ void nf4_quantize_kernel(const bf16* __restrict__ w, int64_t nblocks, uint8_t* __restrict__ codes,
-                                    float* __restrict__ absmax) {
+// Level index of v = w / absmax (binary32): the number of level midpoints
+// strictly below v.  The midpoints m_i = (c_i + c_{i+1}) / 2 are exact in
+// binary64; with t_i = m_i rounded toward -inf to binary32, a binary32 v has
+// v > m_i exactly when v > t_i (if m_i is a binary32 value, t_i = m_i; if
+// not, t_i < m_i < the next binary32 after t_i, and v cannot lie strictly
+// between those two).  So the comparisons run in binary32 against t and take
+// the same decisions as the binary64 ones, ties (v = m_i) to the lower level
+// included.  Four comparisons: a binary search over the 15 thresholds.
+QL_DEV int nf4_level_index(float v, const float* t) {
+  int q = v > t[7] ? 8 : 0;
+  q += v > t[q + 3] ? 4 : 0;
+  q += v > t[q + 1] ? 2 : 0;
+  q += v > t[q] ? 1 : 0;
+  return q;
+}
+
+// Eight threads per 64-element block (one 16-byte load of 8 bf16 each), eight
+// blocks per warp.  absmax = max |w| (exact: bf16 values are binary32 values);
+// v = w / absmax rounded once to binary32 (IEEE division); absmax 0 -> level 7.
+// Each thread stores its 8 level indices as 4 bytes (even element in the high
+// nibble) and the block's first thread its absmax.
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const bf16* __restrict__ w, int64_t nblocks,
+                                                           uint8_t* __restrict__ codes, float* __restrict__ absmax) {
+  __shared__ float thr[15];
+  if (threadIdx.x < 15) {
+    const double mid = 0.5 * (static_cast<double>(__uint_as_float(c_nf4_bits[threadIdx.x])) +
+                              static_cast<double>(__uint_as_float(c_nf4_bits[threadIdx.x + 1])));
+    thr[threadIdx.x] = __double2float_rd(mid);
+  }
+  __syncthreads();
   grid_dep_wait();
   grid_dep_launch();
-  const int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (blk >= nblocks) return;
-  const uint32_t pair = reinterpret_cast<const uint32_t*>(w + blk * 64)[lane];
-  const float x0 = __uint_as_float(pair << 16), x1 = __uint_as_float(pair & 0xFFFF0000u);
-  float m = fmaxf(fabsf(x0), fabsf(x1));
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t blk = t >> 3;
+  const int part = static_cast<int>(t & 7);
+  const bool valid = blk < nblocks;
+  uint4 raw = make_uint4(0, 0, 0, 0);
+  if (valid) raw = __ldg(reinterpret_cast<const uint4*>(w + blk * 64 + part * 8));
+  const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+  float x[8];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  int q0 = 7, q1 = 7;
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = bf16_lo(wv[i]);
+    x[2 * i + 1] = bf16_hi(wv[i]);
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+  // the block's eight threads are lanes 8j .. 8j + 7 of one warp
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (!valid) return;
+  uint32_t packed = 0x77777777u;  // all-zero block: level 7 everywhere
   if (m > 0.f) {
-    const double v0 = static_cast<double>(__fdiv_rn(x0, m));
-    const double v1 = static_cast<double>(__fdiv_rn(x1, m));
-    q0 = 0;
-    q1 = 0;
+    packed = 0;
 #pragma unroll
-    for (int i = 0; i < 15; ++i) {
-      const double mid = 0.5 * (static_cast<double>(__uint_as_float(c_nf4_bits[i])) +
-                                static_cast<double>(__uint_as_float(c_nf4_bits[i + 1])));
-      q0 += v0 > mid;
-      q1 += v1 > mid;
+    for (int i = 0; i < 8; ++i) {
+      const int q = nf4_level_index(__fdiv_rn(x[i], m), thr);
+      // element 2b in the high nibble of byte b, element 2b + 1 in its low nibble
+      packed |= static_cast<uint32_t>(q) << (8 * (i >> 1) + ((i & 1) ? 0 : 4));
     }
   }
-  codes[blk * 32 + lane] = static_cast<uint8_t>((q0 << 4) | q1);
-  if (lane == 0) absmax[blk] = m;
+  reinterpret_cast<uint32_t*>(codes + blk * 32)[part] = packed;
+  if (part == 0) absmax[blk] = m;
 }
 
 // Dequantisation of up to two tensors in one launch.  A warp takes runs of
@@ -102,7 +134,7 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, con
 
 cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st) {
   const int64_t nblocks = numel / 64;
-  const int64_t threads = nblocks * 32;
+  const int64_t threads = nblocks * 8;
   const int64_t grid = (threads + 255) / 256;
   return launch_pdl(nf4_quantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, w, nblocks, codes,
                     absmax);
@@ -117,6 +149,7 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, i
   int64_t grid = (j0.runs + j1.runs + 7) / 8;             // one run per warp, 8 warps per CTA
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 CTAs of 256 threads per SM
   if (grid > cap) grid = cap;
+  grid = apply_grid_cap(static_cast<int>(grid), 1);
   if (grid < 1) grid = 1;
   return launch_pdl(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, j0, j1);
 }

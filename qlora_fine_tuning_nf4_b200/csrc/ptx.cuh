@@ -99,6 +99,24 @@ QL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
   }
 }
 
+// Debug bounds checks.  In the checked build (libqlora_check.so, compiled with
+// -DQLORA_CHECK) a failed check records QL_DEV_BAD_CONFIG in the status word
+// and returns false, and the caller skips the access it guards instead of
+// touching memory out of range; nothing traps.  In the normal build every
+// check is the constant true and compiles away.
+#ifdef QLORA_CHECK
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+QL_DEV bool dev_check(bool ok, int* status) {
+  if constexpr (kChecked) {
+    if (!ok) atomicOr(status, QL_DEV_BAD_CONFIG);
+    return ok;
+  }
+  return true;
+}
+
 // Waits used on the way out after an error, for this thread's own operations
 // still in flight.  Unlike mbar_wait they do not give up when the status word
 // already holds a timeout (that is why they run), but they are bounded too.

@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
     }
     if (kc == nkc - 1 || i == nt - 1) {
       const int slot = c - sk_first(job.sp, rc);
-      store_acc(job.part + static_cast<size_t>(rc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
+      if (dev_check(rc < job.groups && slot >= 0 && slot < job.slot_cap, status))
+        store_acc(job.part + static_cast<size_t>(rc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
     }
   }
 }
@@ -282,7 +283,8 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
     }
     if (mc == nmc - 1 || i == nt - 1) {
       const int slot = c - sk_first(job.sp, cc);
-      store_acc(job.part + static_cast<size_t>(cc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
+      if (dev_check(cc < job.groups && slot >= 0 && slot < job.slot_cap, status))
+        store_acc(job.part + static_cast<size_t>(cc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
     }
   }
 }
@@ -373,11 +375,15 @@ __global__ void __launch_bounds__(SK_THREADS) dypass_kernel(const __grid_constan
       }
       ++i;
     }
-    store_acc(gjob.part + static_cast<size_t>(rc * ncb + cb) * 64 * 16, 16, warp * 16, lane, gacc);
+    if (dev_check(rc < nrc && cb < gjob.slot_cap, status))
+      store_acc(gjob.part + static_cast<size_t>(rc * ncb + cb) * 64 * 16, 16, warp * 16, lane, gacc);
     if (u == u1 - 1 || (u + 1) / nrc != cb) {
-      float* qb = qjob.part + static_cast<size_t>(cb * qjob.slot_cap + c - sk_first(sp, cb)) * (CC * 64) * 16;
+      const int slot = c - sk_first(sp, cb);
+      float* qb = qjob.part + static_cast<size_t>(cb * qjob.slot_cap + slot) * (CC * 64) * 16;
+      if (dev_check(cb < ncb && slot >= 0 && slot < qjob.slot_cap, status)) {
 #pragma unroll
-      for (int q = 0; q < CC; ++q) store_acc(qb + q * 64 * 16, 16, warp * 16, lane, qacc[q]);
+        for (int q = 0; q < CC; ++q) store_acc(qb + q * 64 * 16, 16, warp * 16, lane, qacc[q]);
+      }
     }
   }
 }
@@ -385,22 +391,27 @@ __global__ void __launch_bounds__(SK_THREADS) dypass_kernel(const __grid_constan
 // ------------------------------------------------------------- reduce ----
 // out = bf16(scale * sum over the group's slots of part), summed in slot
 // order.  One thread per four consecutive partial columns; its slot loads are
-// issued sixteen at a time.  One launch serves up to two reductions.
+// issued sixteen at a time.  One launch serves up to kMaxReduceJobs
+// reductions (each with its own partial region): job k takes the threads
+// [start[k], start[k + 1]).
 struct ReduceJobs {
-  ReduceJob j[2];
-  int n0, n1;  // float4 elements (rows * R / 4) of each job
+  ReduceJob j[kMaxReduceJobs];
+  int start[kMaxReduceJobs + 1];  // prefix sums of rows * R / 4 (float4 elements)
+  int n;                          // jobs in use
 };
 __global__ void __launch_bounds__(256) reduce_kernel(const __grid_constant__ ReduceJobs js) {
   grid_dep_wait();
   grid_dep_launch();
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const int k = idx < js.n0 ? 0 : 1;
-  if (k == 1) idx -= js.n0;
-  if (idx >= (k ? js.n1 : js.n0)) return;
+  if (idx >= js.start[js.n]) return;
+  int k = 0;
+  while (k + 1 < js.n && idx >= js.start[k + 1]) ++k;
+  idx -= js.start[k];
   const ReduceJob& j = js.j[k];
   const int row = (idx * 4) / j.R, c = (idx * 4) % j.R;
   const int g = row / j.grows, r = row % j.grows;
-  const int ns = j.nslots > 0 ? j.nslots : sk_slots(j.sp, g);
+  int ns = j.nslots > 0 ? j.nslots : sk_slots(j.sp, g);
+  if (!dev_check(g < j.groups && ns <= j.slot_cap, j.status)) ns = g < j.groups ? j.slot_cap : 0;
   const size_t slot_stride = static_cast<size_t>(j.grows) * j.R;
   const float* p = j.part + static_cast<size_t>(g) * j.slot_cap * slot_stride + static_cast<size_t>(r) * j.R + c;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -514,17 +525,22 @@ cudaError_t arm_inject_timeout() {
   return cudaMemcpyToSymbol(g_inject_timeout, &one, sizeof(one));
 }
 
-cudaError_t launch_reduce(const ReduceJob& j0, const ReduceJob* j1, cudaStream_t st) {
+// One launch for `n` reductions (1 <= n <= kMaxReduceJobs).
+cudaError_t launch_reduce(const ReduceJob* jobs, int n, cudaStream_t st) {
+  if (n < 1 || n > kMaxReduceJobs) return cudaErrorInvalidValue;
   ReduceJobs js;
   std::memset(&js, 0, sizeof(js));
-  js.j[0] = j0;
-  js.n0 = j0.rows * j0.R / 4;
-  if (j1) {
-    js.j[1] = *j1;
-    js.n1 = j1->rows * j1->R / 4;
+  js.n = n;
+  int64_t total = 0;
+  for (int k = 0; k < n; ++k) {
+    js.j[k] = jobs[k];
+    js.start[k] = static_cast<int>(total);
+    total += static_cast<int64_t>(jobs[k].rows) * jobs[k].R / 4;
   }
-  const int n = js.n0 + js.n1;
-  return launch_pdl(reduce_kernel, dim3((n + 255) / 256), dim3(256), 0, st, js);
+  if (total >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  js.start[n] = static_cast<int>(total);
+  if (total == 0) return cudaSuccess;
+  return launch_pdl(reduce_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, st, js);
 }
 
 }  // namespace ql

@@ -14,6 +14,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "libqlora.so")
+CHECK_LIB_PATH = os.path.join(_PKG, "lib", "libqlora_check.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
 
 QLORA_OK = 0
@@ -79,8 +80,21 @@ _SIGS = {
                                      ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
                                      ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
                                      ctypes.c_int64] + [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_mlp_bwd_ev": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear),
+                                        ctypes.POINTER(QloraLoraLinear), ctypes.POINTER(QloraLoraLinear),
+                                        ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
+                                        ctypes.c_int64] + [ctypes.c_void_p] * 8 +
+                         [ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_mlp16_bwd_ev": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(QloraLoraLinear16),
+                                          ctypes.POINTER(QloraLoraLinear16), ctypes.POINTER(QloraLoraLinear16),
+                                          ctypes.c_void_p, ctypes.POINTER(QloraMlpSaved), ctypes.c_void_p,
+                                          ctypes.c_int64] + [ctypes.c_void_p] * 8 +
+                           [ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_last_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_test_inject_timeout": (ctypes.c_int, []),
+    "qlora_test_set_grid_cap": (ctypes.c_int32, [ctypes.c_int32]),
+    "qlora_test_shrink_next_slot_cap": (ctypes.c_int, []),
+    "qlora_checked_build": (ctypes.c_int32, []),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_tile_config": (ctypes.c_int32, [ctypes.c_int32]),
     "qlora_trace_begin": (ctypes.c_int, []),
@@ -122,19 +136,55 @@ _SIGS = {
 }
 
 
+def _load(path):
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m qlora_fine_tuning_nf4_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
 def lib():
     """Load libqlora.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m qlora_fine_tuning_nf4_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in _SIGS.items():
-            f = getattr(L, name)
-            f.restype = res
-            f.argtypes = args
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+_check_lib = None
+
+
+def checked_lib():
+    """Load the bounds-checked debug build, libqlora_check.so (same ABI; its
+    kernels report out-of-range indices as QLORA_ERR_DEVICE instead of
+    touching memory out of range)."""
+    global _check_lib
+    if _check_lib is None:
+        _check_lib = _load(CHECK_LIB_PATH)
+    return _check_lib
+
+
+class use_library:
+    """Context manager that routes every wrapper of this module to another
+    build of the library (e.g. checked_lib()) and restores the previous one."""
+
+    def __init__(self, L):
+        self.L = L
+
+    def __enter__(self):
+        global _lib
+        self.prev = lib()
+        _lib = self.L
+        return self.L
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.prev
+        return False
 
 
 def _check(fn, status):
@@ -420,7 +470,7 @@ def qlora_mlp16_fwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear1
     return _mlp_fwd("qlora_mlp16_fwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, ws, Y, saved)
 
 
-def _mlp_bwd(fn, wsq, act, gate, up, down, X, saved, dY, ws, grads):
+def _mlp_bwd(fn, wsq, act, gate, up, down, X, saved, dY, ws, grads, early_event=0):
     M, d = _rows(X)
     h = _mlp_dims(gate, up, down, d)
     r = gate.A.shape[1]
@@ -438,18 +488,27 @@ def _mlp_bwd(fn, wsq, act, gate, up, down, X, saved, dY, ws, grads):
     g, u, dn, sv = gate.c(), up.c(), down.c(), _saved_c(saved, M, h, r)
     buf = ws.get(wsq(M, d, h, r))
     outs = [_p(grads[k]) for k in ("dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d")]
-    _check(fn, getattr(lib(), fn)(QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X),
-                                  ctypes.byref(sv), _p(dY), M, *outs, _p(buf), buf.numel(), _stream()))
+    args = [QLORA_ACT[act], ctypes.byref(g), ctypes.byref(u), ctypes.byref(dn), _p(X), ctypes.byref(sv), _p(dY), M,
+            *outs, _p(buf), buf.numel(), _stream()]
+    if early_event:
+        _check(fn + "_ev", getattr(lib(), fn + "_ev")(*args, ctypes.c_void_p(early_event)))
+    else:
+        _check(fn, getattr(lib(), fn)(*args))
     return grads
 
 
-def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, dY, ws: Workspace, grads=None):
-    return _mlp_bwd("qlora_mlp_bwd", qlora_mlp_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
+def qlora_mlp_bwd(act, gate: LoraLinear, up: LoraLinear, down: LoraLinear, X, saved, dY, ws: Workspace, grads=None,
+                  early_event=0):
+    """MLP backward; with `early_event` (a raw cudaEvent_t, e.g. torch.cuda.Event().cuda_event after its first
+    record) the library records it once dA_d, dB_d, dB_g and dB_u are final (qlora_mlp_bwd_ev)."""
+    return _mlp_bwd("qlora_mlp_bwd", qlora_mlp_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads,
+                    early_event)
 
 
 def qlora_mlp16_bwd(act, gate: LoraLinear16, up: LoraLinear16, down: LoraLinear16, X, saved, dY, ws: Workspace,
-                    grads=None):
-    return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads)
+                    grads=None, early_event=0):
+    return _mlp_bwd("qlora_mlp16_bwd", qlora_mlp16_workspace_bytes, act, gate, up, down, X, saved, dY, ws, grads,
+                    early_event)
 
 
 def qlora_rmsnorm_fwd(X, w, eps, plus_one=False, Y=None, rstd=None):
@@ -534,6 +593,20 @@ def qlora_qkv_bwd(q: LoraLinear, k: LoraLinear, v: LoraLinear, X, XA, dY, ws: Wo
 def qlora_test_inject_timeout():
     """Arms the library's one-shot timeout injection (test hook; see include/qlora.h)."""
     _check("qlora_test_inject_timeout", lib().qlora_test_inject_timeout())
+
+
+def qlora_test_shrink_next_slot_cap():
+    """Arms the one-shot plan-mismatch hook (test only; see include/qlora.h)."""
+    _check("qlora_test_shrink_next_slot_cap", lib().qlora_test_shrink_next_slot_cap())
+
+
+def qlora_checked_build():
+    return int(lib().qlora_checked_build())
+
+
+def qlora_test_set_grid_cap(max_ctas):
+    """Caps the CTAs of every persistent launch (test hook; 0 = no cap); returns the previous cap."""
+    return int(lib().qlora_test_set_grid_cap(int(max_ctas)))
 
 
 def qlora_last_device_status(ws: Workspace):

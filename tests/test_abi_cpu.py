@@ -67,7 +67,15 @@ def test_host_side_rejections(lib):
     assert f(ctypes.byref(c), 24, 8, 16, 16, 16, 1 << 30, None) == 3          # misaligned X
     assert f(ctypes.byref(c), 16, 8, 16, 16, 16, 64, None) == 4               # workspace too small
     assert f(ctypes.byref(_lin(r=8)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # r != 16
-    assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in % 256
+    assert f(ctypes.byref(_lin(k=100)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in % 64
+    # k_in = 320 (a multiple of 64, not of 256) passes the shape check under the default staged feed
+    # (rejected next for the 64-byte workspace, still before any CUDA call) ...
+    assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, 16, 64, None) == 4
+    prev = ops.qlora_set_tile_config(2)
+    try:  # ... and is unsupported by the feeds that dequantise in the mainloop
+        assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, 16, 1 << 30, None) == 2
+    finally:
+        ops.qlora_set_tile_config(prev)
     assert f(ctypes.byref(_lin(n=500)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # n_out % 8
     assert f(ctypes.byref(c), 16, (1 << 23) + 1, 16, 16, 16, 1 << 62, None) == 2  # M above 2^23
     assert f(ctypes.byref(_lin(k=(1 << 23) + 256)), 16, 8, 16, 16, 16, 1 << 30, None) == 2  # k_in above 2^23
@@ -87,6 +95,31 @@ def test_host_side_rejections(lib):
     assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(bad_d), 16, 8, 16, ctypes.byref(sv), 16, 1 << 40,
               None) == 1                                                        # shapes do not chain
     assert mf(0, ctypes.byref(g), ctypes.byref(u), ctypes.byref(d), 16, 8, 16, ctypes.byref(sv), 16, 10, None) == 4
+
+
+def test_noalloc_host_side_rejections(lib):
+    """qlora_linear_fwd_noalloc rejects, before any CUDA call, what its fixed
+    scratch or its in-mainloop GEMM cannot run (fake device addresses: none of
+    these calls reaches the GPU)."""
+    f = lib.qlora_linear_fwd_noalloc
+    c = _lin(k=256)
+    assert f(ctypes.byref(c), 16, (43648 // 64 + 1) * 64, 16, 16, None) == 4  # beyond the documented 43,648 rows
+    assert f(ctypes.byref(c), 16, 43649, 16, 16, None) == 4
+    assert f(ctypes.byref(_lin(r=32)), 16, 8, 16, 16, None) == 2            # rank 16 only
+    assert f(ctypes.byref(_lin(k=320)), 16, 8, 16, 16, None) == 2           # in-mainloop feed: k_in % 256
+    assert f(ctypes.byref(c), 16, 0, 16, 16, None) == 0                     # M = 0: nothing to do
+    assert f(None, 16, 8, 16, 16, None) == 1
+
+
+def _noalloc_need(M):
+    a256 = lambda x: (x + 255) & ~255
+    return 256 + a256(32 * M) + a256(4096 * -(-M // 64))
+
+
+def test_noalloc_documented_limit_is_the_scratch_formula():
+    """43,648 is the largest M whose scratch, 256 + 32 M + 4096 ceil(M / 64)
+    bytes rounded per term to 256, fits the 4 MiB array."""
+    assert _noalloc_need(43648) <= 4 << 20 < _noalloc_need(43649)
 
 
 def test_rank_support_follows_the_tile_configuration(lib):
@@ -156,3 +189,15 @@ def test_workspace_holds_the_staged_weight_only_under_the_staged_feed(lib):
     assert ops.qlora_mlp16_workspace_bytes(M, d, h) < mlp4
     sizes = [ops.qlora_mlp_workspace_bytes(m, d, h) for m in (1, 256, 1024, 8192, 16384)]
     assert sizes == sorted(sizes)
+
+
+def test_checked_build_exports_the_same_abi():
+    """libqlora_check.so (QLORA_CHECK) exports every symbol the normal build
+    does and says it is the checked build (a host-only call)."""
+    import subprocess
+    syms = lambda path: {l.split()[-1] for l in subprocess.run(["nm", "-D", "--defined-only", path], check=True,
+                                                                  capture_output=True, text=True).stdout.splitlines()
+                         if " T " in l}
+    assert syms(ops.CHECK_LIB_PATH) == syms(ops.LIB_PATH)
+    assert ops.checked_lib().qlora_checked_build() == 1
+    assert ops.lib().qlora_checked_build() == 0

@@ -40,3 +40,15 @@ def test_cpu_baseline_repeats_whole_batches_until_the_target_time():
 def test_c_loop_baseline_record():
     rec = bench.c_loop_oracle_sample()
     assert rec["value"] > 0 and rec["ms"] > 0 and rec["threads"] == 1 and rec["unit"] == bench.UNIT
+
+
+def test_gpus_n_starts_n_ranks_on_one_node():
+    """`bench.py --gpus N` started as one process re-runs itself under torchrun
+    with N ranks on this node (rendezvous on 127.0.0.1), bounded by `timeout`."""
+    cmd = bench.torchrun_command(["--gpus", "4", "--steps", "20"], 4, 29511)
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    i = cmd.index("--master-addr")
+    assert cmd[i + 1] == "127.0.0.1" and cmd[cmd.index("--master-port") + 1] == "29511"
+    assert cmd[-3:] == ["4", "--steps", "20"] and cmd[-5].endswith("bench.py")
+    if cmd[0] == "timeout":
+        assert cmd[1:3] == ["-k", "60"] and int(cmd[3]) > 120  # well above the process group's own timeout

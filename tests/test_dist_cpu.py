@@ -1,7 +1,11 @@
 """Multi-process (gloo, CPU) check of the data-parallel step logic: each rank
 computes the adapter gradients of its token shard (oracle, fp64), the flat
 buffer is all-reduced, and the sum equals the full-batch gradients.  One case
-leaves a rank with no tokens: its gradients are zero and the sum is unchanged."""
+leaves a rank with no tokens: its gradients are zero and the sum is unchanged.
+
+The second test runs the step plumbing the benchmark times (dp.make_step with
+dp.GradAllReduce's two-part sum over dp.flat_lora_grads), with the oracle
+standing in for the library's forward and backward."""
 
 import os
 import socket
@@ -43,7 +47,7 @@ def _worker(rank, world, port, q, M):
         M, d, h, r, X, gate, up, down, dY = _problem(M)
         lo, hi = dp.shard_rows(M, rank, world)
         g = oracle.mlp_bwd("swiglu", X[lo:hi], gate, up, down, dY[lo:hi])
-        flat, views = dp.flat_lora_grads(d, h, r, "cpu", dtype=torch.float64)
+        flat, views, _ = dp.flat_lora_grads(d, h, r, "cpu", dtype=torch.float64)
         for k in dp.GRAD_ORDER:
             views[k].copy_(torch.from_numpy(g[k]))
         dp.allreduce_lora_grads(flat)
@@ -51,6 +55,73 @@ def _worker(rank, world, port, q, M):
             q.put({k: views[k].numpy().copy() for k in dp.GRAD_ORDER})
     finally:
         dist.destroy_process_group()
+
+
+def _step_worker(rank, world, port, q, M):
+    """The benchmark's step (dp.make_step) on this rank's shard, oracle kernels."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        M, d, h, r, X, gate, up, down, dY = _problem(M)
+        lo, hi = dp.shard_rows(M, rank, world)
+        flat, views, early = dp.flat_lora_grads(d, h, r, "cpu", dtype=torch.float64)
+        sync = dp.GradAllReduce(flat, early)
+        state = {"bwd": 0}
+
+        def forward():
+            state["fwd"] = oracle.mlp_fwd("swiglu", X[lo:hi], gate, up, down)
+
+        def backward(ready):
+            assert ready == 0  # no CUDA event on the CPU: both parts are summed after the backward
+            g = oracle.mlp_bwd("swiglu", X[lo:hi], gate, up, down, dY[lo:hi], saved=state["fwd"])
+            for k in dp.GRAD_ORDER:
+                views[k].copy_(torch.from_numpy(g[k]))
+            state["bwd"] += 1
+
+        step = dp.make_step(forward, backward, sync)
+        step()
+        step()  # a second step rewrites the gradients: the sums must not accumulate across steps
+        if rank == 0:
+            q.put(({k: views[k].numpy().copy() for k in dp.GRAD_ORDER}, state["bwd"]))
+    finally:
+        dist.destroy_process_group()
+
+
+def _spawn(target, M, world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=target, args=(rk, world, port, q, M)) for rk in range(world)]
+    for p in procs:
+        p.start()
+    got = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    return got
+
+
+@pytest.mark.parametrize("M,world", [(24, 2), (2, 3)])
+def test_benchmark_step_plumbing_sums_shards_to_full_batch(M, world):
+    got, nbwd = _spawn(_step_worker, M, world)
+    assert nbwd == 2
+    M, d, h, r, X, gate, up, down, dY = _problem(M)
+    full = oracle.mlp_bwd("swiglu", X, gate, up, down, dY)
+    for k in dp.GRAD_ORDER:
+        np.testing.assert_allclose(got[k], full[k], rtol=1e-12, atol=1e-12)
+
+
+def test_early_part_of_the_flat_buffer_is_the_four_gradients_final_before_the_gate_up_dx_gemm():
+    d, h, r = 4096, 11008, 16
+    flat, views, early = dp.flat_lora_grads(d, h, r, "cpu")
+    first = dp.GRAD_ORDER[:dp.MLP_EARLY]
+    assert set(first) == {"dA_d", "dB_d", "dB_g", "dB_u"}
+    assert early == sum(views[k].numel() for k in first)
+    for k in first:
+        assert views[k].data_ptr() < flat.data_ptr() + early * flat.element_size()
+    for k in dp.GRAD_ORDER[dp.MLP_EARLY:]:
+        assert views[k].data_ptr() >= flat.data_ptr() + early * flat.element_size()
 
 
 @pytest.mark.parametrize("M,world", [(24, 2), (2, 3)])  # (2, 3): the third rank's shard is empty
@@ -72,7 +143,7 @@ def test_sharded_gradients_sum_to_full_batch(M, world):
 
 
 def test_flat_buffer_views_are_aligned_and_disjoint():
-    flat, views = dp.flat_lora_grads(4096, 11008, 16, "cpu")
+    flat, views, _ = dp.flat_lora_grads(4096, 11008, 16, "cpu")
     offs = []
     for k in dp.GRAD_ORDER:
         v = views[k]

@@ -153,3 +153,35 @@ def test_mlp_fwd_bwd_parity(tiles, act, M, d, h):
         assert_close(k, g[k], o[k])
     for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
         assert_close(k, g[k], o[k], TOL_SMALL_MLP)
+
+
+# ------------------------------------------- k_in a multiple of 64 only ----
+
+@pytest.mark.parametrize("M,K,N", [(300, 320, 520), (129, 576, 264), (1, 64, 8)])
+def test_linear_k_in_multiple_of_64(M, K, N):
+    """k_in = 64 j with j not a multiple of 4 (the contract is one NF4 block):
+    the default staged feed takes it; the feeds that dequantise in the mainloop
+    reject it before anything is enqueued."""
+    p = make_linear_problem(M, K, N, r=16, alpha=16.0, seed=M + K + N)
+    g = run_linear_gpu(p, 4)
+    o = run_linear_oracle(p)
+    assert g["status"] == 0
+    assert np.array_equal(g["codes"], o["codes"]) and np.array_equal(g["absmax"], o["absmax"])
+    for k in ("XA", "Y", "dX", "dA", "dB"):
+        assert_close(k, g[k], o[k])
+    with pytest.raises(ops.QloraError, match="UNSUPPORTED_SHAPE"):
+        run_linear_gpu(p, 2)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
+def test_mlp_d_multiple_of_64(act):
+    M, d, h = 200, 320, 512
+    p = make_mlp_problem(M, d, h, seed=M + d + h)
+    g = run_mlp_gpu(p, act, 4)
+    o = run_mlp_oracle(p, act)
+    assert g["status"] == 0
+    bounds = saved_bounds(o, p)
+    for k in ("E", "G", "H"):
+        assert_saved(k, g[k], o[k], bounds[k])
+    for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert_close(k, g[k], o[k], TOL_SMALL_MLP)

@@ -1,0 +1,96 @@
+"""Element-by-element parity of the persistent scheduling paths against the
+fp64 oracle: every element of every returned tensor, at sizes where each GEMM
+CTA pair and each rank-side CTA works through several tiles or units.
+
+What these sizes reach that the small parity cases do not:
+  * M = 2344 = 9 x 256 + 40 rows: 10 output-row tiles per GEMM, so the
+    8-row-tile groups of the tile order wrap once and end on a ragged tile;
+  * the gated MLP's gate/up GEMM has 10 x 22 = 220 output tiles against the
+    74 CTA pairs of a B200, so pairs run three tiles and both accumulators;
+  * with the persistent grids capped at 14 CTAs (qlora_test_set_grid_cap; 7
+    GEMM pairs), every GEMM's pairs run 5-32 tiles each, so the accumulator
+    ping-pong, the operand ring's phases across tiles and the group wrap all
+    happen inside one CTA pair, and every rank-side CTA walks a range of many
+    64 x 64 units (42 for X A over X [2344, 1024]) with partial sums spanning
+    several groups; the weight dequantisation's warps loop over many runs;
+  * N = 2824 for the projection: a ragged last output-column tile.
+
+Bars (max |gpu - oracle| <= bar x RMS(oracle), per tensor):
+  * projection outputs: 2e-2;
+  * gated-MLP outputs at these sizes: 2.5e-2.  The design stores X A, E, G, H,
+    dE, dG and s G in bf16 (inputs of later tensor-core contractions); the CPU
+    emulation of exactly those roundings on exact products, with no kernel
+    involved, already gives 1.9-2.2e-2 x RMS over whole tensors at every size
+    tried between 2088 and 4136 rows (tests/test_tolerance_emulation.py pins
+    one of these cases above 2e-2), so an exact implementation of this
+    arithmetic cannot meet 2e-2 on full-tensor maxima.
+  * saved E, G, H: elementwise against the bf16 rounding bound of
+    tests/parity.py (saved_bounds).
+"""
+
+import numpy as np
+import pytest
+
+from qlora_fine_tuning_nf4_b200 import ops
+from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem
+
+from parity import (TOL, assert_close, assert_saved, run_linear_gpu, run_linear_oracle, run_mlp_gpu,
+                    run_mlp_oracle, saved_bounds)
+
+pytestmark = pytest.mark.gpu
+
+TOL_MLP_FULL_TENSOR = 2.5e-2
+MLP_SHAPE = (2344, 1024, 2816)
+LINEAR_SHAPE = (2344, 1024, 2824)
+GRID_CAP = 14  # 7 CTA pairs; not a divisor of any tile count here
+
+_oracle = {}
+
+
+def _mlp(act):
+    key = ("mlp", act)
+    if key not in _oracle:
+        M, d, h = MLP_SHAPE
+        p = make_mlp_problem(M, d, h, seed=M + d + h)
+        o = run_mlp_oracle(p, act)
+        _oracle[key] = (p, o, saved_bounds(o, p))
+    return _oracle[key]
+
+
+def _linear(alpha):
+    key = ("linear", alpha)
+    if key not in _oracle:
+        M, K, N = LINEAR_SHAPE
+        p = make_linear_problem(M, K, N, r=16, alpha=alpha, seed=M + K + N)
+        _oracle[key] = (p, run_linear_oracle(p))
+    return _oracle[key]
+
+
+@pytest.mark.parametrize("cap", [0, GRID_CAP])
+@pytest.mark.parametrize("tiles", [4, 2])
+@pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
+def test_mlp_every_element_multi_tile(act, tiles, cap):
+    p, o, bounds = _mlp(act)
+    ops.qlora_test_set_grid_cap(cap)
+    g = run_mlp_gpu(p, act, tiles)
+    assert g["status"] == 0
+    for k in ("g", "u", "d"):
+        assert np.array_equal(g["q"][k][0], o["q"][k][0]) and np.array_equal(g["q"][k][1], o["q"][k][1])
+    for k in ("E", "G", "H"):
+        assert_saved(k, g[k], o[k], bounds[k])
+    for k in ("XA_g", "XA_u", "HA_d"):
+        assert_close(k, g[k], o[k], TOL)
+    for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert_close(k, g[k], o[k], TOL_MLP_FULL_TENSOR)
+
+
+@pytest.mark.parametrize("cap", [0, GRID_CAP])
+@pytest.mark.parametrize("tiles", [1, 2, 3, 4])
+def test_linear_every_element_multi_tile(tiles, cap):
+    p, o = _linear(32.0)
+    ops.qlora_test_set_grid_cap(cap)
+    g = run_linear_gpu(p, tiles)
+    assert g["status"] == 0
+    assert np.array_equal(g["codes"], o["codes"]) and np.array_equal(g["absmax"], o["absmax"])
+    for k in ("XA", "Y", "dX", "dA", "dB"):
+        assert_close(k, g[k], o[k], TOL)

@@ -194,3 +194,25 @@ def test_dequant_is_rne_of_binary32_product():
     ref16 = torch.from_numpy(ref32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(w32, ref32.astype(np.float64))
     assert np.array_equal(wb, ref16)
+
+
+def test_binary32_thresholds_take_the_binary64_midpoint_decisions():
+    """The quantiser may compare v = RN_binary32(w / absmax) with t_i, the
+    midpoint m_i rounded toward -inf to binary32, instead of with m_i in
+    binary64: for every binary32 v near each midpoint (and at it), v > m_i and
+    v > t_i agree."""
+    mids = oracle.nf4_midpoints()
+    for m in mids:
+        t = np.float32(m)
+        if np.float64(t) > m:
+            t = np.nextafter(t, np.float32(-np.inf))
+        assert np.float64(t) <= m < np.float64(np.nextafter(t, np.float32(np.inf)))
+        v = np.float32(m)
+        near = [v]
+        lo = hi = v
+        for _ in range(6):
+            lo = np.nextafter(lo, np.float32(-np.inf))
+            hi = np.nextafter(hi, np.float32(np.inf))
+            near += [lo, hi]
+        for x in near:
+            assert (np.float64(x) > m) == (x > t), (m, x)

@@ -11,7 +11,10 @@ the oracle.  Rounding each returned tensor alone already costs up to about
 land on single heavy-tailed products, where half a bf16 ulp is large against
 the RMS.  With the stored intermediates the chain reaches 2.25e-2, so an exact
 implementation of this arithmetic would fail the 2e-2 bar, while 3e-2 holds with
-room.  Every full-size workload meets 2e-2 (tests/test_gpu_full.py).
+room.  More rows do not cure it: over whole tensors of 2088-4136 rows the chain
+stays at 1.9-2.2e-2 (one multi-tile case is pinned below), so the multi-tile
+parity cases use 2.5e-2.  The full-size workloads meet 2e-2 on the rows they
+sample (tests/test_gpu_full.py), where the maximum runs over fewer elements.
 """
 
 import numpy as np
@@ -84,6 +87,19 @@ def test_bf16_chain_explains_the_small_mlp_bar():
     assert output_only_min >= 0.7 * TOL
     # ... and the design's stored bf16 intermediates push some case past it
     assert chain_max > TOL
+
+
+def test_bf16_chain_explains_the_multi_tile_mlp_bar():
+    """The multi-tile parity case of tests/test_gpu_persistent.py (2344 tokens,
+    d = 1024, h = 2816, SwiGLU): more rows do not bring the whole-tensor
+    maximum under 2e-2.  The design's own bf16 roundings put Y above 2e-2 x RMS
+    there, so that case's bar is 2.5e-2 (still below the small-M 3e-2)."""
+    from test_gpu_persistent import MLP_SHAPE, TOL_MLP_FULL_TENSOR
+    M, d, h = MLP_SHAPE
+    X, dY, lin, ref = _case(M, d, h, "swiglu")
+    em = _chain("swiglu", X, dY, lin)
+    worst = max(_ratio(em[k], ref[k]) for k in OUTS)
+    assert TOL < worst <= 0.9 * TOL_MLP_FULL_TENSOR, worst
 
 
 @pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
