@@ -158,8 +158,10 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self, t0, t1):
-        """Summary of the samples stamped in [t0, t1] (host wall-clock seconds)."""
+    def stop(self, t0, t1, slack=0.3):
+        """Summary of the samples stamped in [t0, t1] (host wall-clock seconds).  A window shorter than the
+        sampling interval may hold no sample; then the samples within `slack` seconds of it are used (the GPU is
+        busy with the same steps just before and after) and the summary says so."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
@@ -171,8 +173,13 @@ class ClockSampler:
         self.out.seek(0)
         out = self.out.read()
         self.out.close()
-        sm, pw, mx, reasons = [], [], None, set()
+        return self.summarize(out, t0, t1, slack)
+
+    @staticmethod
+    def summarize(out, t0, t1, slack=0.3):
+        """Median SM clock, power and the throttle reasons seen in nvidia-smi's CSV lines `out`."""
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 10:
@@ -182,16 +189,18 @@ class ClockSampler:
                 clk, top, power = float(f[2]), float(f[3]), float(f[4])
             except ValueError:
                 continue
-            if not t0 <= ts <= t1:
-                continue
-            sm.append(clk)
-            pw.append(power)
-            mx = top
-            for n, v in zip(names, f[6:10]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "power_w": statistics.median(pw) if pw else None, "samples": len(sm)}
+            rows.append((ts, clk, top, power, [n for n, v in zip(names, f[6:10]) if v.lower().startswith("active")]))
+        window = "timed region"
+        sel = [r for r in rows if t0 <= r[0] <= t1]
+        if not sel:
+            sel = [r for r in rows if t0 - slack <= r[0] <= t1 + slack]
+            window = f"no sample inside the {1e3 * (t1 - t0):.0f} ms timed region; samples within {slack} s of it"
+        sm = [r[1] for r in sel]
+        pw = [r[3] for r in sel]
+        reasons = sorted({n for r in sel for n in r[4]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": sel[-1][2] if sel else None,
+                "reasons": reasons, "power_w": statistics.median(pw) if pw else None, "samples": len(sm),
+                "window": window}
 
 
 # ------------------------------------------------------------ oracle arm ---

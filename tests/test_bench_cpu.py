@@ -52,3 +52,19 @@ def test_gpus_n_starts_n_ranks_on_one_node():
     assert cmd[-3:] == ["4", "--steps", "20"] and cmd[-5].endswith("bench.py")
     if cmd[0] == "timeout":
         assert cmd[1:3] == ["-k", "60"] and int(cmd[3]) > 120  # well above the process group's own timeout
+
+
+def test_clock_summary_uses_the_timed_window_or_its_nearest_samples():
+    import datetime
+    base = datetime.datetime(2026, 1, 1, 12, 0, 0)
+    line = lambda dt, mhz, cap: (f"{(base + datetime.timedelta(seconds=dt)).strftime('%Y/%m/%d %H:%M:%S.%f')[:-3]}, "
+                                 f"0, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, "
+                                 f"{'Active' if cap else 'Not Active'}")
+    out = "\n".join([line(0.00, 1965, False), line(0.05, 1800, True), line(0.10, 1700, True), line(0.40, 1965, False)])
+    t = base.timestamp()
+    inside = bench.ClockSampler.summarize(out, t + 0.04, t + 0.11)
+    assert inside["samples"] == 2 and inside["sm_mhz"] == 1750 and inside["reasons"] == ["sw_power_cap"]
+    assert inside["window"] == "timed region"
+    short = bench.ClockSampler.summarize(out, t + 0.65, t + 0.655)  # a 5 ms window holds no sample
+    assert short["samples"] == 1 and short["sm_mhz"] == 1965 and short["reasons"] == []
+    assert "no sample inside" in short["window"]

@@ -13,7 +13,10 @@ What these sizes reach that the small parity cases do not:
     happen inside one CTA pair, and every rank-side CTA walks a range of many
     64 x 64 units (42 for X A over X [2344, 1024]) with partial sums spanning
     several groups; the weight dequantisation's warps loop over many runs;
-  * N = 2824 for the projection: a ragged last output-column tile.
+  * N = 2824 for the projection: a ragged last output-column tile;
+  * the same paths at ranks 32 and 64 (the LoRA term as up to four 16-wide
+    MMA steps, rank-side passes split into G and dB passes), with a frozen bf16
+    base, and for the fused Q/K/V projection.
 
 Bars (max |gpu - oracle| <= bar x RMS(oracle), per tensor):
   * projection outputs: 2e-2;
@@ -32,9 +35,9 @@ import numpy as np
 import pytest
 
 from qlora_fine_tuning_nf4_b200 import ops
-from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem
+from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem, make_qkv_problem
 
-from parity import (TOL, assert_close, assert_saved, run_linear_gpu, run_linear_oracle, run_mlp_gpu,
+from parity import (TOL, assert_close, assert_saved, run_linear_gpu, run_linear_oracle, run_mlp16_gpu, run_mlp_gpu,
                     run_mlp_oracle, saved_bounds)
 
 pytestmark = pytest.mark.gpu
@@ -94,3 +97,58 @@ def test_linear_every_element_multi_tile(tiles, cap):
     assert np.array_equal(g["codes"], o["codes"]) and np.array_equal(g["absmax"], o["absmax"])
     for k in ("XA", "Y", "dX", "dA", "dB"):
         assert_close(k, g[k], o[k], TOL)
+
+
+# Ranks 32 and 64, the 16-bit base and the fused Q/K/V projection on the same
+# persistent paths: multi-tile sizes with the grid capped, every element.
+
+@pytest.mark.parametrize("r", [32, 64])
+def test_linear_higher_rank_every_element_multi_tile(r):
+    M, K, N = LINEAR_SHAPE
+    p = make_linear_problem(M, K, N, r=r, alpha=float(r), seed=M + K + N + r)
+    o = run_linear_oracle(p)
+    ops.qlora_test_set_grid_cap(GRID_CAP)
+    g = run_linear_gpu(p, 4)
+    assert g["status"] == 0
+    for k in ("XA", "Y", "dX", "dA", "dB"):
+        assert_close(k, g[k], o[k], TOL)
+
+
+def test_mlp_rank64_every_element_multi_tile():
+    M, d, h = MLP_SHAPE
+    p = make_mlp_problem(M, d, h, r=64, alpha=64.0, seed=M + d + h + 64)
+    o = run_mlp_oracle(p, "swiglu")
+    ops.qlora_test_set_grid_cap(GRID_CAP)
+    g = run_mlp_gpu(p, "swiglu", 4)
+    assert g["status"] == 0
+    bounds = saved_bounds(o, p)
+    for k in ("E", "G", "H"):
+        assert_saved(k, g[k], o[k], bounds[k])
+    for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert_close(k, g[k], o[k], TOL_MLP_FULL_TENSOR)
+
+
+@pytest.mark.parametrize("cap", [0, GRID_CAP])
+def test_mlp16_every_element_multi_tile(cap):
+    p, _, _ = _mlp("swiglu")
+    o = run_mlp_oracle(p, "swiglu", base="bf16")
+    ops.qlora_test_set_grid_cap(cap)
+    g = run_mlp16_gpu(p, "swiglu")
+    assert g["status"] == 0
+    for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert_close(k, g[k], o[k], TOL_MLP_FULL_TENSOR)
+
+
+def test_qkv_every_element_multi_tile():
+    """Fused Q/K/V at grouped-query widths (q 2048, k 512, v 264: a ragged v tile) over 2344 tokens, grid capped."""
+    from test_gpu_qkv import run_qkv_gpu, run_qkv_oracle
+    p = make_qkv_problem(2344, 1024, 2048, 512, 264, r=16, alpha=16.0, seed=77)
+    o = run_qkv_oracle(p)
+    ops.qlora_test_set_grid_cap(GRID_CAP)
+    g = run_qkv_gpu(p)
+    assert g["status"] == 0
+    for k in ("Y", "XA", "dX"):
+        assert_close(k, g[k], o[k], TOL)
+    for n in "qkv":
+        for k in ("dA_" + n, "dB_" + n):
+            assert_close(k, g[k], o[k], TOL)
