@@ -352,6 +352,11 @@ typedef struct {
   double total_ms;  /* summed device time between the bracketing events */
 } qlora_trace_entry;
 QLORA_API qlora_status qlora_trace_begin(void);
+/* As qlora_trace_begin, but only launches of the kernel named `kernel_name`
+ * (one of the names qlora_trace_end reports, e.g. "gemm_nf4_gateup_glu_fwd")
+ * are bracketed; every other launch keeps its programmatic overlap with its
+ * neighbours.  QLORA_ERR_INVALID_ARG for an unknown name. */
+QLORA_API qlora_status qlora_trace_begin_only(const char* kernel_name);
 /* Stops tracing, waits for the recorded events and fills up to `max_entries`
  * per-kernel totals; returns the number of distinct kernels (or -1). */
 QLORA_API int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries);

@@ -56,6 +56,7 @@ const char* const kKernelNames[K_COUNT] = {
 
 std::atomic<uint64_t> g_launches{0};
 bool g_trace = false;
+int g_trace_only = -1;  // kernel id traced alone (qlora_trace_begin_only), -1 = every kernel
 struct TraceRec {
   int id;
   cudaEvent_t a, b;
@@ -106,7 +107,7 @@ struct KScope {
   cudaEvent_t b = nullptr;
   KScope(int id_, cudaStream_t st_) : id(id_), st(st_) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (g_trace) {
+    if (g_trace && (g_trace_only < 0 || g_trace_only == id)) {
       cudaEvent_t a = pool_event();
       b = pool_event();
       if (a && b) {
@@ -1375,8 +1376,21 @@ qlora_status qlora_last_device_status(void* ws, qlora_stream_t stream) {
 qlora_status qlora_trace_begin(void) {
   g_recs.clear();
   g_pool_used = 0;
+  g_trace_only = -1;
   g_trace = true;
   return QLORA_OK;
+}
+
+qlora_status qlora_trace_begin_only(const char* kernel_name) {
+  if (!kernel_name) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < K_COUNT; ++i) {
+    if (std::strcmp(kernel_name, kKernelNames[i]) == 0) {
+      qlora_status s = qlora_trace_begin();
+      g_trace_only = i;
+      return s;
+    }
+  }
+  return QLORA_ERR_INVALID_ARG;
 }
 
 int32_t qlora_trace_end(qlora_trace_entry* out, int32_t max_entries) {

@@ -98,6 +98,7 @@ _SIGS = {
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_tile_config": (ctypes.c_int32, [ctypes.c_int32]),
     "qlora_trace_begin": (ctypes.c_int, []),
+    "qlora_trace_begin_only": (ctypes.c_int, [ctypes.c_char_p]),
     "qlora_trace_end": (ctypes.c_int32, [ctypes.POINTER(QloraTraceEntry), ctypes.c_int32]),
     "qlora_launch_count": (ctypes.c_uint64, []),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(QloraLoraLinear), ctypes.c_void_p, ctypes.c_int64,
@@ -629,8 +630,12 @@ def qlora_launch_count():
     return int(lib().qlora_launch_count())
 
 
-def qlora_trace_begin():
-    _check("qlora_trace_begin", lib().qlora_trace_begin())
+def qlora_trace_begin(only=None):
+    """Start tracing every kernel launch, or only the kernel named `only`."""
+    if only is None:
+        _check("qlora_trace_begin", lib().qlora_trace_begin())
+    else:
+        _check("qlora_trace_begin_only", lib().qlora_trace_begin_only(only.encode()))
 
 
 def qlora_trace_end(max_entries=64):
