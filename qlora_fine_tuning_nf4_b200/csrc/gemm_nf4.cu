@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(GemmCfg<MODE, CG, MH, ST>::THREADS, 1)
           // ranks below 64 leave the rest of the boxes to the TMA's zero fill.
           // plain forward of fused projections: the tile's columns belong to one of them
           const int fop = (args.ncut[1] > 0 && n0 >= args.ncut[1]) ? 2 : ((args.ncut[0] > 0 && n0 >= args.ncut[0]) ? 1 : 0);
-          const int fcol0 = fop == 0 ? 0 : args.ncut[fop - 1];
+          const int fcol0 = fop == 0 ? 0 : (fop == 1 ? args.ncut[0] : args.ncut[1]);
           for (int i = 0; i < args.lora; ++i, ++j) {
             const int s = j % C::S;
             const int op = MODE == MODE_FWD ? fop : i;
