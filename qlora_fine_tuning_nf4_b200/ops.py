@@ -4,6 +4,11 @@ Argument marshalling only: tensors are PyTorch CUDA tensors (device memory and
 streams), their data pointers and the current stream are passed to the C ABI,
 and every step of the computation runs in the library's CUDA kernels.  There
 is no CPU fallback: if ``lib/libqlora.so`` is missing, every call raises.
+
+With the environment variable QLORA_LIBRARY=checked the binding loads the
+bounds-checked debug build ``lib/libqlora_check.so`` instead (same ABI; its
+kernels report an out-of-range index through the status word rather than
+touching memory out of range).
 """
 
 import ctypes
@@ -149,10 +154,13 @@ def _load(path):
 
 
 def lib():
-    """Load libqlora.so (raises if it has not been built)."""
+    """Load libqlora.so, or libqlora_check.so under QLORA_LIBRARY=checked (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        _lib = _load(LIB_PATH)
+        choice = os.environ.get("QLORA_LIBRARY", "")
+        if choice not in ("", "checked"):
+            raise RuntimeError(f"QLORA_LIBRARY={choice!r}: expected unset or 'checked'")
+        _lib = _load(CHECK_LIB_PATH if choice == "checked" else LIB_PATH)
     return _lib
 
 
