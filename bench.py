@@ -62,7 +62,9 @@ def parse():
     ap.add_argument("--workload", default="llama7b_swiglu_mlp", choices=sorted(MLP_WORKLOADS) + sorted(LINEAR_WORKLOADS),
                     help="an MLP workload (ops mlp, norm_mlp, qkv) or a single-projection one (op linear)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--tiles", type=int, default=4, help="GEMM tile configuration (1-4)")
+    ap.add_argument("--tiles", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="GEMM tile configuration: 0 = the library's automatic choice (the default), 1-3 dequantise "
+                         "in the mainloop, 4 = staged bf16 weight")
     ap.add_argument("--op", default="mlp", choices=["mlp", "norm_mlp", "qkv", "linear"],
                     help="the timed step: the gated MLP (the metric), the MLP behind its RMS layer norm (norm "
                          "forward and backward added), the fused Q/K/V projection (GQA widths), or one QLoRA "
@@ -703,7 +705,7 @@ def run_ours(args, wl):
         "frac_of_bf16_peak_sustained": value / world / pk["bf16_sustained"],
         "config": {"workload": args.workload, "op": args.op, "M_per_gpu": M, "d": d, **cfg_extra, "r": r,
                    "nf4_block": 64, "global_batch_tokens": M * world, "parallelism": f"dp{world}",
-                   "gemm_tiles": ops.TILE_CONFIGS[4 if args.weights == "bf16" else args.tiles],
+                   "gemm_tiles": ops.TILE_CONFIGS[effective_tiles(args, ops, M, d, h, r)],
                    "base_weights": args.weights, "l2": l2_note(args.op, M, d, h, cfg_extra)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "steps": e2e_steps,
@@ -722,6 +724,15 @@ def run_ours(args, wl):
         "cpu_baseline": cpu,
         "clocks": clocks,
     }), flush=True)
+
+
+def effective_tiles(args, ops, M, d, h, r):
+    """The GEMM configuration the timed step's calls use (the automatic setting resolved)."""
+    if args.weights == "bf16" or args.op == "qkv":
+        return 4  # the 16-bit and fused Q/K/V calls always stream a bf16 weight by TMA
+    if args.op in ("mlp", "norm_mlp"):
+        return ops.qlora_mlp_tile_config(M, d, h, r)
+    return args.tiles or 4
 
 
 def torchrun_command(argv, gpus, port, limit_s=1800):

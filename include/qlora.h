@@ -146,9 +146,10 @@ QLORA_API size_t qlora_linear_workspace_bytes(int64_t M, int64_t k_in, int64_t n
  *   XA = X A                      -> XA_saved [M, r]  (kept for the backward)
  *   Y  = X dequant(W)^T + s XA B  -> Y [M, n_out]
  * X [M, k_in].  Requires k_in % 64 == 0 (one NF4 block), n_out % 8 == 0, and
- * r = 16, 32 or 64 under tile configuration 4 (the default).  Tile
- * configurations 1-3 further require k_in % 256 == 0 (their GEMM loads each
- * weight row's absmax values by TMA, in 16-byte pieces) and r = 16. */
+ * r = 16, 32 or 64 under tile configuration 4 (what the default, automatic
+ * setting uses here).  Tile configurations 1-3 further require k_in % 256 ==
+ * 0 (their GEMM loads each weight row's absmax values by TMA, in 16-byte
+ * pieces) and r = 16. */
 QLORA_API qlora_status qlora_linear_fwd(const qlora_lora_linear* lin, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                               qlora_bf16* XA_saved, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
@@ -175,8 +176,9 @@ QLORA_API size_t qlora_mlp_workspace_bytes(int64_t M, int64_t d, int64_t h, int3
  * (QLORA_ACT_GEGLU_TANH).  gate/up: n_out = h, k_in = d; down: n_out = d,
  * k_in = h.  X [M, d], Y [M, d]; `saved` receives E, G, H, XA_g, XA_u, HA_d.
  * Requires d % 64 == 0, h % 256 == 0, the same r for the three projections,
- * and r = 16, 32 or 64 under tile configuration 4 (the default); tile
- * configurations 1-3 require d % 256 == 0 and r = 16. */
+ * and r = 16, 32 or 64 under tile configuration 4; tile configurations 1-3
+ * require d % 256 == 0 and r = 16 (the automatic setting picks 2 only when
+ * they hold; see qlora_set_tile_config). */
 QLORA_API qlora_status qlora_mlp_fwd(qlora_act act, const qlora_lora_linear* gate, const qlora_lora_linear* up,
                            const qlora_lora_linear* down, const qlora_bf16* X, int64_t M, qlora_bf16* Y,
                            const qlora_mlp_saved* saved, void* workspace, size_t workspace_bytes,
@@ -335,14 +337,22 @@ QLORA_API const char* qlora_status_string(qlora_status status);
  * Configurations 1-3 dequantise the weight tile by tile in shared memory
  * inside the GEMM mainloop: 1 = one CTA per 128 x 256 tile, 2 = a CTA pair
  * (cta_group::2) per 256 x 256 tile, 3 = a CTA pair per 512 x 128 tile whose
- * dequantised weight tile feeds two M = 256 MMAs.  Configuration 4 (default)
- * = a CTA pair per 256 x 256 tile whose weight is first dequantised once per
- * call into the workspace (the nf4_dequantize kernel) and then streamed by TMA:
- * each weight element is decoded once instead of once per 256-row tile, at the
- * price of that bf16 copy in the workspace.  The workspace size queries follow
- * the configuration current when they are called.  Invalid values are ignored.
- * Returns the previous value.  Not thread-safe. */
+ * dequantised weight tile feeds two M = 256 MMAs.  Configuration 4 = a CTA
+ * pair per 256 x 256 tile whose weight is first dequantised once per call
+ * into the workspace (the nf4_dequantize kernel) and then streamed by TMA:
+ * each weight element is decoded once instead of once per 256-row tile, at
+ * the price of that bf16 copy in the workspace.  0 (the default) = automatic:
+ * the NF4 gated-MLP calls use configuration 2 for at most 512 tokens (rank
+ * 16, d % 256 == 0), where decoding in the mainloop is faster than staging
+ * the three weights, and configuration 4 otherwise; the projection and Q/K/V
+ * calls use 4.  The workspace size queries follow the configuration current
+ * when they are called.  Invalid values are ignored.  Returns the previous
+ * value.  Not thread-safe. */
 QLORA_API int32_t qlora_set_tile_config(int32_t tiles);
+/* The tile configuration (1-4) that qlora_mlp_fwd / qlora_mlp_bwd use for M
+ * tokens, width d, MLP width h and rank r under the current setting.  Host
+ * only. */
+QLORA_API int32_t qlora_mlp_tile_config(int64_t M, int64_t d, int64_t h, int32_t r);
 
 /* Kernel tracing (host side, not thread-safe).  While enabled, every kernel
  * launch of the library is bracketed by CUDA events on its stream. */
@@ -376,8 +386,9 @@ QLORA_API uint64_t qlora_launch_count(void);
  * returns QLORA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  It
  * allocates nothing and frees nothing.
  * The fixed array has no room for a staged weight, so this call always runs a
- * GEMM that dequantises the weight in its mainloop: tile configuration 2 when
- * configuration 4 (the default) is selected, else the selected 1-3.  Those
+ * GEMM that dequantises the weight in its mainloop: tile configuration 2 under
+ * the automatic setting (the default) or when configuration 4 is selected,
+ * else the selected 1-3.  Those
  * take rank-16 adapters only; other ranks return QLORA_ERR_UNSUPPORTED_SHAPE
  * before anything is enqueued.
  * The first call on a device looks up the array's device address (with that

@@ -102,6 +102,7 @@ _SIGS = {
     "qlora_checked_build": (ctypes.c_int32, []),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_tile_config": (ctypes.c_int32, [ctypes.c_int32]),
+    "qlora_mlp_tile_config": (ctypes.c_int32, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32]),
     "qlora_trace_begin": (ctypes.c_int, []),
     "qlora_trace_begin_only": (ctypes.c_int, [ctypes.c_char_p]),
     "qlora_trace_end": (ctypes.c_int32, [ctypes.POINTER(QloraTraceEntry), ctypes.c_int32]),
@@ -626,12 +627,17 @@ def qlora_status_string(status):
     return lib().qlora_status_string(status).decode()
 
 
-TILE_CONFIGS = {1: "1 CTA, 128x256", 2: "CTA pair, 256x256", 3: "CTA pair, 512x128",
+TILE_CONFIGS = {0: "automatic", 1: "1 CTA, 128x256", 2: "CTA pair, 256x256", 3: "CTA pair, 512x128",
                 4: "CTA pair, 256x256, staged bf16 weight"}
 
 
 def qlora_set_tile_config(tiles):
     return int(lib().qlora_set_tile_config(tiles))
+
+
+def qlora_mlp_tile_config(M, d, h, r=16):
+    """The tile configuration the NF4 MLP calls use for these sizes under the current setting."""
+    return int(lib().qlora_mlp_tile_config(M, d, h, r))
 
 
 def qlora_launch_count():

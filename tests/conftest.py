@@ -16,8 +16,10 @@ def pytest_configure(config):
 @pytest.fixture(autouse=True)
 def _restore_library_state(request):
     """The GEMM tile configuration and the persistent-grid cap are process-wide
-    settings of the library; every GPU test gets the defaults (configuration 4,
-    no cap) and leaves them as it found them, whatever order the tests run in."""
+    settings of the library; every GPU test starts with configuration 4 (the
+    staged feed; a test that wants another, or the automatic setting, sets it)
+    and no cap, and leaves both as it found them, whatever order the tests run
+    in."""
     if request.node.get_closest_marker("gpu") is None:
         yield
         return

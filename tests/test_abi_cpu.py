@@ -201,3 +201,23 @@ def test_checked_build_exports_the_same_abi():
     assert syms(ops.CHECK_LIB_PATH) == syms(ops.LIB_PATH)
     assert ops.checked_lib().qlora_checked_build() == 1
     assert ops.lib().qlora_checked_build() == 0
+
+
+def test_automatic_tile_configuration(lib):
+    """Configuration 0 (the default): the NF4 MLP calls dequantise in the mainloop
+    (configuration 2) up to 512 tokens when rank and width allow it, and stage
+    the weights (configuration 4) otherwise; an explicit choice is kept."""
+    prev = ops.qlora_set_tile_config(0)
+    try:
+        assert ops.qlora_mlp_tile_config(256, 4096, 11008, 16) == 2
+        assert ops.qlora_mlp_tile_config(512, 4096, 11008, 16) == 2
+        assert ops.qlora_mlp_tile_config(513, 4096, 11008, 16) == 4
+        assert ops.qlora_mlp_tile_config(8192, 4096, 11008, 16) == 4
+        assert ops.qlora_mlp_tile_config(256, 4096, 11008, 32) == 4   # configuration 2 takes rank 16 only
+        assert ops.qlora_mlp_tile_config(256, 320, 512, 16) == 4      # ... and d % 256 == 0
+        # the workspace follows: no staging room below the threshold
+        assert ops.qlora_mlp_workspace_bytes(256, 4096, 11008) < ops.qlora_mlp_workspace_bytes(256, 4096, 11008, 32)
+        ops.qlora_set_tile_config(3)
+        assert ops.qlora_mlp_tile_config(8192, 4096, 11008, 16) == 3
+    finally:
+        ops.qlora_set_tile_config(prev)

@@ -185,3 +185,18 @@ def test_mlp_d_multiple_of_64(act):
         assert_saved(k, g[k], o[k], bounds[k])
     for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
         assert_close(k, g[k], o[k], TOL_SMALL_MLP)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "geglu_tanh"])
+@pytest.mark.parametrize("M", [256, 1100])
+def test_mlp_automatic_configuration(act, M):
+    """The default, automatic setting: 256 tokens take the pair tile that
+    dequantises in the mainloop, 1100 the staged feed; both match the oracle."""
+    d, h = 512, 768
+    p = make_mlp_problem(M, d, h, seed=M + d + h + 1)
+    g = run_mlp_gpu(p, act, tiles=0)
+    assert ops.qlora_mlp_tile_config(M, d, h, 16) == (2 if M <= 512 else 4)
+    o = run_mlp_oracle(p, act)
+    assert g["status"] == 0
+    for k in ("Y", "dX", "dA_g", "dB_g", "dA_u", "dB_u", "dA_d", "dB_d"):
+        assert_close(k, g[k], o[k], TOL_SMALL_MLP)

@@ -55,11 +55,13 @@ def test_noalloc_forward_is_bitwise_the_workspace_forward_twice(alpha):
         assert_close("XA", gpu_f64(XA), o["XA"], TOL)
 
 
-def test_noalloc_under_the_default_configuration():
-    """The default staged configuration 4 needs a weight buffer the fixed
-    scratch does not have, so the call runs configuration 2; its outputs agree
-    with qlora_linear_fwd under configuration 4 and with the oracle."""
-    assert ops.qlora_set_tile_config(4) == 4
+@pytest.mark.parametrize("tiles", [0, 4])
+def test_noalloc_under_the_default_and_the_staged_configuration(tiles):
+    """Under the automatic setting (the library's default) and under the staged
+    configuration 4 the workspace forward stages the weight, which the fixed
+    scratch has no room for, so this call runs configuration 2; its outputs
+    agree with qlora_linear_fwd under the same setting and with the oracle."""
+    ops.qlora_set_tile_config(tiles)
     p = make_linear_problem(777, 512, 1032, r=16, alpha=16.0, seed=8)
     lin = _lin(p)
     X = bits_to_torch(p["X"], "cuda")
