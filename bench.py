@@ -214,50 +214,71 @@ class ClockSampler:
 
 # ------------------------------------------------------------ oracle arm ---
 
-def oracle_sample(wl, rows=None, seed_rows=0, target_s=12.0):
-    """Time the fp64 oracle's MLP fwd+bwd on `rows` tokens of the workload.
-
-    With rows None, a 64-row probe sizes the sample to about `target_s` seconds
-    of CPU work; when the whole batch takes less, whole-batch steps repeat
-    until `target_s` has passed.  Returns (seconds, flop, threads, rows,
-    steps).  Weights are quantised/dequantised by the oracle itself before
-    timing (one-time, like the GPU side's quantisation).
-    """
+def _oracle_step(wl, op):
+    """(run, flops): run(n, off) times the fp64 oracle's fwd+bwd on token rows [off, off + n) of the workload
+    (a gated MLP, or one projection for op "linear"); flops(n) is its algorithmic FLOP count.  Weights are
+    quantised and dequantised by the oracle itself first (one-time, like the GPU side's quantisation)."""
     import oracle
     from oracle.nf4 import nf4_dequantize_f64
-    from qlora_fine_tuning_nf4_b200.synth import make_mlp_problem
+    from qlora_fine_tuning_nf4_b200.synth import make_linear_problem, make_mlp_problem
+    from qlora_fine_tuning_nf4_b200.workloads import linear_flops
 
+    f64 = oracle.bf16_bits_to_f64
+    if op == "linear":
+        p = make_linear_problem(wl["M"], wl["K"], wl["N"], wl["r"], wl["alpha"], wl["seed"])
+        n_out, k_in = p["W"].shape
+        c, a = oracle.nf4_quantize(p["W"], n_out, k_in)
+        W, A, B = nf4_dequantize_f64(c, a, n_out, k_in), f64(p["A"]), f64(p["B"])
+
+        def run(n, off):
+            X, dY = f64(p["X"][off:off + n]), f64(p["dY"][off:off + n])
+            t0 = time.perf_counter()
+            oracle.linear_fwd(X, W, A, B, p["s"])
+            oracle.linear_bwd(X, W, A, B, p["s"], dY)
+            return time.perf_counter() - t0
+
+        return run, lambda n: linear_flops(n, wl["K"], wl["N"], wl["r"])
     p = make_mlp_problem(wl["M"], wl["d"], wl["h"], wl["r"], wl["alpha"], wl["seed"])
     lin = {}
     for k in ("g", "u", "d"):
-        n, kk = p["W_" + k].shape
-        c, a = oracle.nf4_quantize(p["W_" + k], n, kk)
-        lin[k] = (nf4_dequantize_f64(c, a, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
-                  oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
+        n_out, k_in = p["W_" + k].shape
+        c, a = oracle.nf4_quantize(p["W_" + k], n_out, k_in)
+        lin[k] = (nf4_dequantize_f64(c, a, n_out, k_in), f64(p["A_" + k]), f64(p["B_" + k]), p["s"])
 
-    def run(n):
-        X = oracle.bf16_bits_to_f64(p["X"][seed_rows:seed_rows + n])
-        dY = oracle.bf16_bits_to_f64(p["dY"][seed_rows:seed_rows + n])
+    def run(n, off):
+        X, dY = f64(p["X"][off:off + n]), f64(p["dY"][off:off + n])
         t0 = time.perf_counter()
         fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
         oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
         return time.perf_counter() - t0
 
+    return run, lambda n: mlp_flops(n, wl["d"], wl["h"], wl["r"])
+
+
+def oracle_sample(wl, rows=None, seed_rows=0, target_s=12.0, op="mlp"):
+    """Time the fp64 oracle's fwd+bwd (gated MLP, or one projection for op "linear") on `rows` tokens.
+
+    With rows None, a 64-row probe sizes the sample to about `target_s` seconds
+    of CPU work; when the whole batch takes less, whole-batch steps repeat
+    until `target_s` has passed.  Returns (seconds, flop, threads, rows,
+    steps).
+    """
+    run, flops = _oracle_step(wl, op)
     steps = 1
     if rows is None:
-        per_row = run(64) / 64
+        probe = min(64, wl["M"] - seed_rows)
+        per_row = run(probe, seed_rows) / probe
         rows = int(min(wl["M"] - seed_rows, max(64, target_s / max(per_row, 1e-9))))
         rows -= rows % 64
         if 2 * rows >= wl["M"] - seed_rows:  # the probe overestimates: take whole batches
             rows = wl["M"] - seed_rows
-            dt = run(rows)
+            dt = run(rows, seed_rows)
             while dt < target_s:
-                dt += run(rows)
+                dt += run(rows, seed_rows)
                 steps += 1
-            return (dt, steps * mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0)), rows,
-                    steps)
-    dt = run(rows)
-    return dt, mlp_flops(rows, wl["d"], wl["h"], wl["r"]), len(os.sched_getaffinity(0)), rows, steps
+            return dt, steps * flops(rows), len(os.sched_getaffinity(0)), rows, steps
+    dt = run(rows, seed_rows)
+    return dt, flops(rows), len(os.sched_getaffinity(0)), rows, steps
 
 
 def c_loop_oracle_sample():
@@ -287,23 +308,10 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
-    from oracle.nf4 import nf4_dequantize_f64
-    from qlora_fine_tuning_nf4_b200.synth import make_mlp_problem
-
-    p = make_mlp_problem(wl["M"], wl["d"], wl["h"], wl["r"], wl["alpha"], wl["seed"])
-    lin = {}
-    for k in ("g", "u", "d"):
-        n, kk = p["W_" + k].shape
-        c, a = oracle.nf4_quantize(p["W_" + k], n, kk)
-        lin[k] = (nf4_dequantize_f64(c, a, n, kk), oracle.bf16_bits_to_f64(p["A_" + k]),
-                  oracle.bf16_bits_to_f64(p["B_" + k]), p["s"])
+    run, flops = _oracle_step(wl, args.op)
 
     def step(rows, off):
-        X = oracle.bf16_bits_to_f64(p["X"][off:off + rows])
-        dY = oracle.bf16_bits_to_f64(p["dY"][off:off + rows])
-        fwd = oracle.mlp_fwd(wl["act"], X, lin["g"], lin["u"], lin["d"])
-        oracle.mlp_bwd(wl["act"], X, lin["g"], lin["u"], lin["d"], dY, saved=fwd)
+        run(rows, off)
 
     # size the per-step row sample so the whole run takes about two minutes
     t0 = time.perf_counter()
@@ -319,7 +327,7 @@ def run_reference(args, wl):
     for i in range(args.steps):
         step(rows, (i * rows) % (wl["M"] - rows + 1))
     dt = time.perf_counter() - t0
-    flop = mlp_flops(rows, wl["d"], wl["h"], wl["r"]) * args.steps
+    flop = flops(rows) * args.steps
     value = flop / dt / 1e12
     cores = len(os.sched_getaffinity(0))
     sample = f"{rows} of {wl['M']} token rows per step (fp64 numpy, BLAS threads = cores)"
@@ -327,8 +335,10 @@ def run_reference(args, wl):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "M": wl["M"], "d": wl["d"], "h": wl["h"], "r": wl["r"],
-                   "act": wl["act"], "sample_rows": rows},
+        "config": {"workload": args.workload, "op": args.op, "M": wl["M"],
+                   **({"K": wl["K"], "N": wl["N"]} if args.op == "linear" else {"d": wl["d"], "h": wl["h"],
+                                                                               "act": wl["act"]}),
+                   "r": wl["r"], "sample_rows": rows},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -686,8 +696,8 @@ def run_ours(args, wl):
                "ms_per_step": tot / args.steps}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op == "mlp":
-        dt, fl, cores, rows, n = oracle_sample(wl)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.op in ("mlp", "linear"):
+        dt, fl, cores, rows, n = oracle_sample(wl, op=args.op)
         what = f"{n} fwd+bwd steps of all {M} token rows" if rows == M else f"{rows} of {M} token rows, one fwd+bwd"
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{what} (fp64 numpy, {dt:.1f} s)",
@@ -762,8 +772,8 @@ def main():
         sys.exit(subprocess.call(torchrun_command(sys.argv[1:], args.gpus, free_port())))
     if (args.op == "linear") != (args.workload in LINEAR_WORKLOADS):
         sys.exit(f"--op {args.op} needs {'a single-projection' if args.op == 'linear' else 'an MLP'} workload")
-    if args.op == "linear" and args.impl == "reference":
-        sys.exit("--impl reference times the MLP workloads only")
+    if args.impl == "reference" and args.op not in ("mlp", "linear"):
+        sys.exit("--impl reference times the MLP (--op mlp) and single-projection (--op linear) workloads")
     wl = dict(LINEAR_WORKLOADS[args.workload] if args.op == "linear" else MLP_WORKLOADS[args.workload])
     if args.tokens:
         wl["M"] = args.tokens

@@ -68,3 +68,12 @@ def test_clock_summary_uses_the_timed_window_or_its_nearest_samples():
     short = bench.ClockSampler.summarize(out, t + 0.65, t + 0.655)  # a 5 ms window holds no sample
     assert short["samples"] == 1 and short["sm_mhz"] == 1965 and short["reasons"] == []
     assert "no sample inside" in short["window"]
+
+
+def test_cpu_baseline_for_a_single_projection():
+    """The projection workloads are timed against the oracle's projection fwd+bwd too."""
+    from qlora_fine_tuning_nf4_b200.workloads import LINEAR_WORKLOADS, linear_flops
+    wl = dict(LINEAR_WORKLOADS["tiny_linear"])
+    dt, flop, cores, rows, steps = bench.oracle_sample(wl, op="linear", target_s=0.3)
+    assert rows == wl["M"] and steps >= 1 and dt >= 0.3
+    assert flop == steps * linear_flops(wl["M"], wl["K"], wl["N"], wl["r"])
