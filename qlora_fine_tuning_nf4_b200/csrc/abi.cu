@@ -1060,10 +1060,13 @@ static qlora_status mlp_bwd(qlora_act act, const Lin* gate, const Lin* up, const
 // ------------------------------------------------------------ fused QKV --
 namespace {
 // QKV workspace: [status | 256 B][s XA, M x 3r][s G, M x 3r][partials][staged [nq+nk+nv, K] weight]
+// The backward's three dY passes (q, k, v) are reduced in one launch, so their
+// partial sums sit side by side: [q pass | k pass | v pass].
+size_t qkv_dy_part(int64_t M, int64_t n, int r) { return align256(dypass_part_bytes(M, n, r)); }
 size_t qkv_ws(int64_t M, int64_t K, int64_t nq, int64_t nk, int64_t nv, int r) {
   const size_t vec = align256(static_cast<size_t>(M) * 3 * r * 2);
   size_t part = rowproj_part_bytes(M, K, 3 * r);
-  for (int64_t n : {nq, nk, nv}) part = std::max(part, dypass_part_bytes(M, n, r));
+  part = std::max(part, qkv_dy_part(M, nq, r) + qkv_dy_part(M, nk, r) + qkv_dy_part(M, nv, r));
   part = std::max(part, 3 * r <= 128 ? colproj_part_bytes(M, K, 3 * r) : colproj_part_bytes(M, K, r));
   return 256 + 2 * vec + align256(part) + stage_bytes(nq + nk + nv, K);
 }
@@ -1196,13 +1199,20 @@ qlora_status qlora_qkv_bwd(const qlora_lora_linear* q_, const qlora_lora_linear*
   bf16* stage = reinterpret_cast<bf16*>(w + qkv_ws(M, K, nq, nk, nv, r) - stage_bytes(Nt, K));
   const bf16* dy = reinterpret_cast<const bf16*>(dY);
   const bf16* xa = reinterpret_cast<const bf16*>(XA_saved);
-  // per projection: G_p = dY_p B_p^T (stored s_p-scaled into [sG_q | sG_k | sG_v]), dB_p = s_p XA_p^T dY_p
-  for (int p = 0; p < 3; ++p) {
-    s = pass_dypass(dy + off[p], M, L[p]->w.n_out, xa + p * r, reinterpret_cast<const bf16*>(L[p]->B), r, part,
-                    routs(rout(sg + p * r, 0, r, 3 * r, 0, L[p]->scale)),
-                    routs(rout(reinterpret_cast<bf16*>(dB[p]), 0, r, (int)L[p]->w.n_out, 1, L[p]->scale)), status,
-                    st, Nt, 3 * r);
-    if (s != QLORA_OK) return s;
+  // per projection: G_p = dY_p B_p^T (stored s_p-scaled into [sG_q | sG_k | sG_v]), dB_p = s_p XA_p^T dY_p;
+  // the three passes' reductions share one launch (each pass has its own partial region)
+  {
+    ReduceBatch rb;
+    char* pp = reinterpret_cast<char*>(part);
+    for (int p = 0; p < 3; ++p) {
+      s = pass_dypass(dy + off[p], M, L[p]->w.n_out, xa + p * r, reinterpret_cast<const bf16*>(L[p]->B), r,
+                      reinterpret_cast<float*>(pp), routs(rout(sg + p * r, 0, r, 3 * r, 0, L[p]->scale)),
+                      routs(rout(reinterpret_cast<bf16*>(dB[p]), 0, r, (int)L[p]->w.n_out, 1, L[p]->scale)), status,
+                      st, Nt, 3 * r, &rb);
+      if (s != QLORA_OK) return s;
+      pp += qkv_dy_part(M, L[p]->w.n_out, r);
+    }
+    if ((s = flush_reduce(rb, st)) != QLORA_OK) return s;
   }
   if ((s = stage_qkv(&lq, &lk, &lv, stage, st)) != QLORA_OK) return s;
   // dX = dY [W_q ; W_k ; W_v] + sum_p (s_p G_p) A_p^T: one concatenated reduction and three LoRA blocks
