@@ -27,8 +27,9 @@ int gemm_nf4_b_cols_per_cta(int tiles);
 cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
                            const CUtensorMap& v1, const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
                            cudaStream_t st);
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc, int nch,
                            int* status, cudaStream_t st);
+int colproj_chunks(int R);  // column chunks of 64 per colproj unit (group) for a tile width R
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
 cudaError_t arm_inject_timeout();
@@ -231,8 +232,9 @@ constexpr int kDyCC = 4;  // column chunks of 64 per dypass unit (matches the ke
 SkPlan plan_rowproj(int64_t M, int64_t K, int fcols, int target = 0) {
   return plan_skinny(cdiv(M, 64), cdiv(K, 64), target > 0 ? target : skinny_target_ctas(fcols));
 }
+// colproj: groups of colproj_chunks(R) column chunks of 64 (R the factor-tile width)
 SkPlan plan_colproj(int64_t M, int64_t ncols, int R) {
-  return plan_skinny(cdiv(ncols, 64), cdiv(M, 64), skinny_target_ctas(R));
+  return plan_skinny(cdiv(cdiv(ncols, 64), colproj_chunks(R)), cdiv(M, 64), skinny_target_ctas(R));
 }
 SkPlan plan_dypass(int64_t M, int64_t N) {
   return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64), skinny_target_ctas(32));
@@ -242,7 +244,8 @@ size_t rowproj_part_bytes(int64_t M, int64_t K, int R, int target = 0) {
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
   R = R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 128));  // the kernel's tile width
-  return static_cast<size_t>(cdiv(ncols, 64)) * plan_colproj(M, ncols, R).slot_cap * 64 * R * 4;
+  const int cc = colproj_chunks(R);
+  return static_cast<size_t>(cdiv(cdiv(ncols, 64), cc)) * plan_colproj(M, ncols, R).slot_cap * cc * 64 * R * 4;
 }
 size_t dypass_gpart_bytes(int64_t M, int64_t N) {
   return align256(static_cast<size_t>(cdiv(M, 64)) * cdiv(cdiv(N, 64), kDyCC) * 64 * 16 * 4);
@@ -373,12 +376,13 @@ qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U
   if (!map_factor(&mu, U, M, R, ldu ? ldu : R, colproj_width(R))) return QLORA_ERR_CUDA;
   R = colproj_width(R);
   const SkPlan p = plan_colproj(M, ncols, R);
-  const int64_t ncc = cdiv(ncols, 64);
-  ReduceJob j = reduce_job(part, ncc, 64, ncols, R, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
+  const int cc = colproj_chunks(R);
+  const int64_t nch = cdiv(ncols, 64);
+  ReduceJob j = reduce_job(part, cdiv(nch, cc), cc * 64, ncols, R, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
   j.status = status;
   {
     KScope k(K_COLPROJ, st);
-    const qlora_status s = cuda_status(launch_colproj(R, mt, mu, j, (int)cdiv(M, 64), status, st));
+    const qlora_status s = cuda_status(launch_colproj(R, mt, mu, j, (int)cdiv(M, 64), (int)nch, status, st));
     if (s != QLORA_OK) return s;
   }
   return reduce_now_or_later(&j, 1, batch, st);

@@ -229,13 +229,21 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------- colproj ---
-// Units: 64x64 tiles (cc, mc), mc fastest; group = column block cc (nmc units).
-// job.part[cc][slot][64][R]: T^T U over the CTA's tiles of column block cc.
-template <int R>
+// Units: (cb, mc) = 64 rows x CC column chunks of 64, mc fastest; group =
+// column block cb (CC * 64 columns, nmc units).  A unit's chunks are 64x64
+// tiles of T, one ring stage each, side by side in the same 64 rows, so a CTA
+// walking down its column block reads CC * 128 contiguous bytes of every row;
+// each stage also carries the unit's U rows (from L2).
+// job.part[cb][slot][CC * 64][R]: T^T U over the CTA's rows of column block cb.
+// CC for a factor-tile width R (16 to 128): the accumulators hold CC * R / 2
+// floats per thread, at most 64.
+constexpr int colproj_cc(int R) { return R <= 32 ? 4 : (R == 64 ? 2 : 1); }
+int colproj_chunks(int R) { return colproj_cc(R); }
+template <int R, int CC>
 __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_constant__ CUtensorMap tmap_t,
                                                              const __grid_constant__ CUtensorMap tmap_u,
                                                              const __grid_constant__ ReduceJob job, int nmc,
-                                                             int* status) {
+                                                             int nch, int* status) {
   using F = FTile<R>;
   constexpr int STAGE = T_TILE + F::BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -243,48 +251,65 @@ __global__ void __launch_bounds__(SK_THREADS) colproj_kernel(const __grid_consta
   const uint32_t bars = sbase + SK_STAGES * STAGE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
-  int t0, t1;
-  sk_range(job.sp, job.groups * nmc, c, t0, t1);
-  const int nt = t1 - t0;
+  int u0, u1;
+  sk_range(job.sp, job.groups * nmc, c, u0, u1);
+  auto chunks = [&](int cb) { return min(CC, nch - cb * CC); };
+  int nt = 0;
+  for (int u = u0; u < u1; ++u) nt += chunks(u / nmc);
   sk_init(bars);
 
   if (warp == SK_CWARPS) {
-    if (lane == 0)
-      sk_produce(nt, bars, status, [&](int i, int s, uint32_t fb) {
-        const int t = t0 + i, cc = t / nmc, mc = t % nmc;
+    if (lane == 0) {
+      int u = u0, cc = 0;
+      sk_produce(nt, bars, status, [&](int, int s, uint32_t fb) {
+        const int cb = u / nmc, mc = u % nmc;
         const uint32_t st = sbase + s * STAGE;
         mbar_arrive_expect_tx(fb, STAGE);
-        tma_load_2d(st, &tmap_t, fb, cc * 64, mc * 64);
+        tma_load_2d(st, &tmap_t, fb, (cb * CC + cc) * 64, mc * 64);
 #pragma unroll
         for (int sub = 0; sub < R / F::SUBW; ++sub)
           tma_load_2d(st + T_TILE + sub * F::SUB_BYTES, &tmap_u, fb, sub * F::SUBW, mc * 64);
+        if (++cc == chunks(cb)) {
+          cc = 0;
+          ++u;
+        }
       });
+    }
     return;
   }
-  float acc[R / 8][4] = {};
+  float acc[CC][R / 8][4] = {};
+  int i = 0;
   bool ok = true;
-  for (int i = 0; i < nt; ++i) {
-    const int t = t0 + i, cc = t / nmc, mc = t % nmc;
-    ok = sk_acquire(bars, i, ok, status);
-    if (ok) {
-      const uint32_t tb = sbase + (i % SK_STAGES) * STAGE;
+  for (int u = u0; u < u1; ++u) {
+    const int cb = u / nmc, ncc = chunks(cb);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t a[4];
-        frag_a_cols(tb, kk * 16, warp * 16, lane, a);
+    for (int cc = 0; cc < CC; ++cc) {
+      if (cc >= ncc) break;
+      ok = sk_acquire(bars, i, ok, status);
+      if (ok) {
+        const uint32_t tb = sbase + (i % SK_STAGES) * STAGE;
 #pragma unroll
-        for (int nb = 0; nb < R / 8; ++nb) {
-          uint32_t b[2];
-          frag_b_kn_f<R>(tb + T_TILE, kk * 16, nb * 8, lane, b);
-          mma_bf16_16816(acc[nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t a[4];
+          frag_a_cols(tb, kk * 16, warp * 16, lane, a);
+#pragma unroll
+          for (int nb = 0; nb < R / 8; ++nb) {
+            uint32_t b[2];
+            frag_b_kn_f<R>(tb + T_TILE, kk * 16, nb * 8, lane, b);
+            mma_bf16_16816(acc[cc][nb], a[0], a[1], a[2], a[3], b[0], b[1]);
+          }
         }
+        sk_release(bars, i, lane);
       }
-      sk_release(bars, i, lane);
+      ++i;
     }
-    if (mc == nmc - 1 || i == nt - 1) {
-      const int slot = c - sk_first(job.sp, cc);
-      if (dev_check(cc < job.groups && slot >= 0 && slot < job.slot_cap, status))
-        store_acc(job.part + static_cast<size_t>(cc * job.slot_cap + slot) * 64 * R, R, warp * 16, lane, acc);
+    if (u == u1 - 1 || (u + 1) / nmc != cb) {
+      const int slot = c - sk_first(job.sp, cb);
+      float* qb = job.part + static_cast<size_t>(cb * job.slot_cap + slot) * (CC * 64) * R;
+      if (dev_check(cb < job.groups && slot >= 0 && slot < job.slot_cap, status)) {
+#pragma unroll
+        for (int q = 0; q < CC; ++q) store_acc(qb + q * 64 * R, R, warp * 16, lane, acc[q]);
+      }
     }
   }
 }
@@ -495,20 +520,22 @@ cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const 
 
 template <int R>
 static cudaError_t launch_colproj_t(const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
-                                    int* status, cudaStream_t st) {
+                                    int nch, int* status, cudaStream_t st) {
+  constexpr int CC = colproj_cc(R);
   const int smem = sk_smem(T_TILE + FTile<R>::BYTES);
-  cudaError_t e = set_smem((const void*)colproj_kernel<R>, smem);
+  auto k = colproj_kernel<R, CC>;
+  cudaError_t e = set_smem((const void*)k, smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(colproj_kernel<R>, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, u, job, nmc, status);
+  return launch_pdl(k, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, u, job, nmc, nch, status);
 }
 
-// R in {16, 32, 64, 128}
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+// R in {16, 32, 64, 128}; nch = column chunks of 64 in T
+cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc, int nch,
                            int* status, cudaStream_t st) {
-  if (R == 16) return launch_colproj_t<16>(t, u, job, nmc, status, st);
-  if (R == 32) return launch_colproj_t<32>(t, u, job, nmc, status, st);
-  if (R == 64) return launch_colproj_t<64>(t, u, job, nmc, status, st);
-  if (R == 128) return launch_colproj_t<128>(t, u, job, nmc, status, st);
+  if (R == 16) return launch_colproj_t<16>(t, u, job, nmc, nch, status, st);
+  if (R == 32) return launch_colproj_t<32>(t, u, job, nmc, nch, status, st);
+  if (R == 64) return launch_colproj_t<64>(t, u, job, nmc, nch, status, st);
+  if (R == 128) return launch_colproj_t<128>(t, u, job, nmc, nch, status, st);
   return cudaErrorInvalidValue;
 }
 
