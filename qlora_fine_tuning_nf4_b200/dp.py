@@ -64,9 +64,10 @@ def shard_rows(M_total, rank, world):
 
 
 def allreduce_lora_grads(flat, group=None):
-    """Sum the flat gradient buffer over all ranks (in place, one collective)."""
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    """Sum the flat gradient buffer over all ranks, in place (GradAllReduce in one part)."""
+    sync = GradAllReduce(flat, 0, group)
+    sync.launch()
+    sync.wait()
     return flat
 
 
@@ -81,12 +82,20 @@ class GradAllReduce:
     rewrites them).  On CPU (gloo) both collectives run synchronously.  With one
     rank nothing is enqueued.  Every rank must make the same calls in the same
     order.
+
+    The sums run in binary32 at least: a bf16 buffer is widened into a binary32
+    copy, summed there and rounded back once, so each summed gradient carries
+    one rounding after the ranks' own, whatever the number of ranks (a bf16 sum
+    would round again at every step of the reduction).  Wider buffers are
+    summed as they are.
     """
 
     def __init__(self, flat, early=0, group=None):
         self.flat, self.early, self.group = flat, int(early), group
         self.world = dist.get_world_size(group) if (dist.is_available() and dist.is_initialized()) else 1
-        self.stream = self.ready = None
+        self.stream = self.ready = self.acc = None
+        if self.world > 1 and torch.promote_types(flat.dtype, torch.float32) != flat.dtype:
+            self.acc = torch.empty(flat.numel(), dtype=torch.float32, device=flat.device)
         if flat.is_cuda and self.world > 1:
             self.stream = torch.cuda.Stream(device=flat.device)
             if self.early > 0:
@@ -97,25 +106,35 @@ class GradAllReduce:
         """Raw cudaEvent_t of ``ready`` for the library to record (0 = none)."""
         return self.ready.cuda_event if self.ready is not None else 0
 
-    def _parts(self):
-        return [p for p in (self.flat[:self.early], self.flat[self.early:]) if p.numel()]
+    def _sum(self, lo, hi):
+        """All-reduce flat[lo:hi] (through the binary32 copy for a bf16 buffer)."""
+        part = self.flat[lo:hi]
+        if self.acc is None:
+            dist.all_reduce(part, op=dist.ReduceOp.SUM, group=self.group)
+            return
+        acc = self.acc[lo:hi]
+        acc.copy_(part)
+        dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=self.group)
+        part.copy_(acc)
 
     def launch(self):
         """Enqueue the sums; call right after enqueueing the backward."""
         if self.world == 1:
             return
+        n = self.flat.numel()
         if self.stream is None:
-            for p in self._parts():
-                dist.all_reduce(p, op=dist.ReduceOp.SUM, group=self.group)
+            for lo, hi in ((0, self.early), (self.early, n)):
+                if hi > lo:
+                    self._sum(lo, hi)
             return
         main = torch.cuda.current_stream(self.flat.device)
         with torch.cuda.stream(self.stream):
             if self.early > 0:
                 self.stream.wait_event(self.ready)
-                dist.all_reduce(self.flat[:self.early], op=dist.ReduceOp.SUM, group=self.group)
+                self._sum(0, self.early)
             self.stream.wait_stream(main)
-            if self.early < self.flat.numel():
-                dist.all_reduce(self.flat[self.early:], op=dist.ReduceOp.SUM, group=self.group)
+            if self.early < n:
+                self._sum(self.early, n)
 
     def wait(self):
         if self.stream is not None:

@@ -112,6 +112,43 @@ def test_benchmark_step_plumbing_sums_shards_to_full_batch(M, world):
         np.testing.assert_allclose(got[k], full[k], rtol=1e-12, atol=1e-12)
 
 
+def _bf16_contrib(rank, n=4096):
+    """Rank `rank`'s bf16 contribution: magnitudes within a factor 2^6 of each other, so the sum of
+    four of them is exact in binary32 and its bf16 rounding is the correctly rounded sum."""
+    g = torch.Generator().manual_seed(100 + rank)
+    mag = torch.exp2(torch.randint(-3, 3, (n,), generator=g).float())
+    return (torch.randn(n, generator=g) * mag).to(torch.bfloat16)
+
+
+def _bf16_sum_worker(rank, world, port, q, early):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        flat = _bf16_contrib(rank).clone()
+        sync = dp.GradAllReduce(flat, early)
+        sync.launch()
+        sync.wait()
+        if rank == 0:
+            q.put(flat.clone())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("early", [0, 1000])
+def test_bf16_gradients_are_summed_in_binary32_and_rounded_once(early):
+    world = 4
+    got = _spawn(_bf16_sum_worker, early, world)
+    parts = [_bf16_contrib(rk) for rk in range(world)]
+    exact = sum(p.float() for p in parts)  # exact in binary32 (see _bf16_contrib)
+    assert torch.equal(got, exact.to(torch.bfloat16))
+    # the check has teeth: adding in bf16, rank after rank, rounds differently for many elements
+    seq = parts[0]
+    for p in parts[1:]:
+        seq = (seq.float() + p.float()).to(torch.bfloat16)
+    assert (seq != exact.to(torch.bfloat16)).sum() > 100
+
+
 def test_early_part_of_the_flat_buffer_is_the_four_gradients_final_before_the_gate_up_dx_gemm():
     d, h, r = 4096, 11008, 16
     flat, views, early = dp.flat_lora_grads(d, h, r, "cpu")
