@@ -27,9 +27,9 @@ int gemm_nf4_b_cols_per_cta(int tiles);
 cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const CUtensorMap& v0,
                            const CUtensorMap& v1, const CUtensorMap& v2, const ReduceJob& job, int nkc, int* status,
                            cudaStream_t st);
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc, int nch,
-                           int* status, cudaStream_t st);
-int colproj_chunks(int R);  // column chunks of 64 per colproj unit (group) for a tile width R
+cudaError_t launch_colproj(int R, int cc, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+                           int nch, int* status, cudaStream_t st);
+int colproj_chunks(int R);  // the widest colproj unit (column chunks of 64) for a tile width R
 cudaError_t launch_dypass(const CUtensorMap& t, const CUtensorMap& u, const CUtensorMap& b, const ReduceJob& gjob,
                           const ReduceJob& qjob, int nch, int* status, cudaStream_t st);
 cudaError_t arm_inject_timeout();
@@ -232,9 +232,17 @@ constexpr int kDyCC = 4;  // column chunks of 64 per dypass unit (matches the ke
 SkPlan plan_rowproj(int64_t M, int64_t K, int fcols, int target = 0) {
   return plan_skinny(cdiv(M, 64), cdiv(K, 64), target > 0 ? target : skinny_target_ctas(fcols));
 }
-// colproj: groups of colproj_chunks(R) column chunks of 64 (R the factor-tile width)
+// colproj units of `cc` column chunks of 64 (R the factor-tile width).  Several chunks side by
+// side read colproj_chunks(R) x 128 contiguous bytes of each row, which pays on wide operands, but
+// every CTA then writes a partial that many times taller; one chunk is kept unless those partials
+// stay within 1/16 of the bytes the pass streams.
+int colproj_cc_for(int64_t M, int64_t ncols, int R) {
+  const int cmax = colproj_chunks(R);
+  const double partials = static_cast<double>(skinny_target_ctas(R)) * cmax * 64 * R * 4;
+  return partials * 16 <= static_cast<double>(M) * ncols * 2 ? cmax : 1;
+}
 SkPlan plan_colproj(int64_t M, int64_t ncols, int R) {
-  return plan_skinny(cdiv(cdiv(ncols, 64), colproj_chunks(R)), cdiv(M, 64), skinny_target_ctas(R));
+  return plan_skinny(cdiv(cdiv(ncols, 64), colproj_cc_for(M, ncols, R)), cdiv(M, 64), skinny_target_ctas(R));
 }
 SkPlan plan_dypass(int64_t M, int64_t N) {
   return plan_skinny(cdiv(cdiv(N, 64), kDyCC), cdiv(M, 64), skinny_target_ctas(32));
@@ -244,7 +252,7 @@ size_t rowproj_part_bytes(int64_t M, int64_t K, int R, int target = 0) {
 }
 size_t colproj_part_bytes(int64_t M, int64_t ncols, int R) {
   R = R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 128));  // the kernel's tile width
-  const int cc = colproj_chunks(R);
+  const int cc = colproj_cc_for(M, ncols, R);
   return static_cast<size_t>(cdiv(cdiv(ncols, 64), cc)) * plan_colproj(M, ncols, R).slot_cap * cc * 64 * R * 4;
 }
 size_t dypass_gpart_bytes(int64_t M, int64_t N) {
@@ -376,13 +384,13 @@ qlora_status pass_colproj(const bf16* T, int64_t M, int64_t ncols, const bf16* U
   if (!map_factor(&mu, U, M, R, ldu ? ldu : R, colproj_width(R))) return QLORA_ERR_CUDA;
   R = colproj_width(R);
   const SkPlan p = plan_colproj(M, ncols, R);
-  const int cc = colproj_chunks(R);
+  const int cc = colproj_cc_for(M, ncols, R);
   const int64_t nch = cdiv(ncols, 64);
   ReduceJob j = reduce_job(part, cdiv(nch, cc), cc * 64, ncols, R, planned_slot_cap(p.slot_cap), 0, p.sp, outs);
   j.status = status;
   {
     KScope k(K_COLPROJ, st);
-    const qlora_status s = cuda_status(launch_colproj(R, mt, mu, j, (int)cdiv(M, 64), (int)nch, status, st));
+    const qlora_status s = cuda_status(launch_colproj(R, cc, mt, mu, j, (int)cdiv(M, 64), (int)nch, status, st));
     if (s != QLORA_OK) return s;
   }
   return reduce_now_or_later(&j, 1, batch, st);

@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(SK_THREADS) rowproj_kernel(const __grid_consta
 // walking down its column block reads CC * 128 contiguous bytes of every row;
 // each stage also carries the unit's U rows (from L2).
 // job.part[cb][slot][CC * 64][R]: T^T U over the CTA's rows of column block cb.
-// CC for a factor-tile width R (16 to 128): the accumulators hold CC * R / 2
-// floats per thread, at most 64.
+// CC is 1 or, for wide operands (chosen on the host), colproj_cc(R): the
+// accumulators then hold CC * R / 2 floats per thread, at most 64.
 constexpr int colproj_cc(int R) { return R <= 32 ? 4 : (R == 64 ? 2 : 1); }
 int colproj_chunks(int R) { return colproj_cc(R); }
 template <int R, int CC>
@@ -518,10 +518,9 @@ cudaError_t launch_rowproj(int rw, int nf, bool bt, const CUtensorMap& t, const 
   return cudaErrorInvalidValue;
 }
 
-template <int R>
+template <int R, int CC>
 static cudaError_t launch_colproj_t(const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
                                     int nch, int* status, cudaStream_t st) {
-  constexpr int CC = colproj_cc(R);
   const int smem = sk_smem(T_TILE + FTile<R>::BYTES);
   auto k = colproj_kernel<R, CC>;
   cudaError_t e = set_smem((const void*)k, smem);
@@ -529,13 +528,20 @@ static cudaError_t launch_colproj_t(const CUtensorMap& t, const CUtensorMap& u, 
   return launch_pdl(k, dim3(job.sp.P), dim3(SK_THREADS), smem, st, t, u, job, nmc, nch, status);
 }
 
-// R in {16, 32, 64, 128}; nch = column chunks of 64 in T
-cudaError_t launch_colproj(int R, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc, int nch,
-                           int* status, cudaStream_t st) {
-  if (R == 16) return launch_colproj_t<16>(t, u, job, nmc, nch, status, st);
-  if (R == 32) return launch_colproj_t<32>(t, u, job, nmc, nch, status, st);
-  if (R == 64) return launch_colproj_t<64>(t, u, job, nmc, nch, status, st);
-  if (R == 128) return launch_colproj_t<128>(t, u, job, nmc, nch, status, st);
+// R in {16, 32, 64, 128}; cc = 1 or colproj_cc(R) column chunks per unit; nch = column chunks of 64 in T
+cudaError_t launch_colproj(int R, int cc, const CUtensorMap& t, const CUtensorMap& u, const ReduceJob& job, int nmc,
+                           int nch, int* status, cudaStream_t st) {
+#define QL_COL(R_)                                                                              \
+  if (R == R_) {                                                                                \
+    if (cc == 1) return launch_colproj_t<R_, 1>(t, u, job, nmc, nch, status, st);               \
+    if (cc == colproj_cc(R_)) return launch_colproj_t<R_, colproj_cc(R_)>(t, u, job, nmc, nch, status, st); \
+    return cudaErrorInvalidValue;                                                               \
+  }
+  QL_COL(16)
+  QL_COL(32)
+  QL_COL(64)
+  QL_COL(128)
+#undef QL_COL
   return cudaErrorInvalidValue;
 }
 
