@@ -58,7 +58,8 @@ def run_qkv_oracle(p, rows=None):
 
 @pytest.mark.parametrize("r", [16, 32, 64])
 @pytest.mark.parametrize("M,K,nq,nk,nv", [(300, 512, 512, 256, 256), (256, 1024, 1024, 256, 256),
-                                           (200, 512, 768, 256, 136), (130, 320, 512, 256, 256)])
+                                           (200, 512, 768, 256, 136), (130, 320, 512, 256, 256),
+                                           (1, 256, 256, 256, 8)])  # one token, an 8-wide v
 def test_qkv_parity(r, M, K, nq, nk, nv):
     p = make_qkv_problem(M, K, nq, nk, nv, r=r, alpha=2.0 * r, seed=M + K + nq + nv + r)
     g = run_qkv_gpu(p)
