@@ -11,7 +11,7 @@ import oracle
 from qlora_fine_tuning_nf4_b200 import ops
 from qlora_fine_tuning_nf4_b200.synth import bits_to_torch, make_qkv_problem
 
-from parity import TOL, assert_close, f64, gpu_f64, oracle_weight
+from parity import TOL, assert_close, assert_saved, f64, gpu_f64, oracle_weight
 
 pytestmark = pytest.mark.gpu
 
@@ -69,7 +69,12 @@ def test_qkv_parity(r, M, K, nq, nk, nv):
         assert_close(k, g[k], o[k])
     for n in "qkv":
         for k in ("dA_" + n, "dB_" + n):
-            assert_close(k, g[k], o[k])
+            if M == 1:
+                # one token row: dA and dB are outer products, each element two bf16 roundings
+                # (of s G or X A, and of the result) away from the exact value, 2^-8 relative each
+                assert_saved(k, g[k], o[k], 2.0 ** -7 * np.abs(o[k]) + 2.0 ** -12 * np.sqrt(np.mean(o[k] ** 2)))
+            else:
+                assert_close(k, g[k], o[k])
 
 
 def test_qkv_mistral_widths_sampled_rows():
