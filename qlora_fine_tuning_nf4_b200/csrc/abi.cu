@@ -18,9 +18,8 @@
 namespace ql {
 // kernels implemented in the other translation units
 cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, float* absmax, cudaStream_t st);
-cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
-                                  const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
-                                  cudaStream_t st, int num_sms);
+cudaError_t launch_nf4_dequantize(const uint8_t* const* codes, const float* const* absmax, const int64_t* numel,
+                                  bf16* const* out, int n, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm_nf4(int mode, int epi, int tiles, const GemmMaps& maps, const GemmArgs& args,
                             cudaStream_t stream);
 int gemm_nf4_b_cols_per_cta(int tiles);
@@ -472,12 +471,25 @@ bool map_staged(CUtensorMap* m, const void* wq, const Wt& w, bool bwd, int bnc) 
   if (!bwd) return map_bf16(m, wq, K, N, K, 64, bnc < 128 ? bnc : 128, CU_TENSOR_MAP_SWIZZLE_128B);
   return map_bf16(m, wq, K, N, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
 }
-// Dequantises one weight (w1 == nullptr) or two in one launch into their staging buffers.
-qlora_status stage_weights(const Wt& w0, bf16* dst0, const Wt* w1, bf16* dst1, cudaStream_t st) {
+// Dequantises one weight (w1 == nullptr), two, or three (w2 too) in one launch into their staging buffers.
+qlora_status stage_weights(const Wt& w0, bf16* dst0, const Wt* w1, bf16* dst1, cudaStream_t st,
+                           const Wt* w2 = nullptr, bf16* dst2 = nullptr) {
+  const Wt* w[3] = {&w0, w1, w2};
+  bf16* const dst[3] = {dst0, dst1, dst2};
+  const uint8_t* codes[3];
+  const float* absmax[3];
+  int64_t numel[3];
+  bf16* out[3];
+  int n = 0;
+  for (int i = 0; i < 3; ++i) {
+    if (!w[i]) continue;
+    codes[n] = w[i]->codes;
+    absmax[n] = w[i]->absmax;
+    numel[n] = w[i]->n_out * w[i]->k_in;
+    out[n++] = dst[i];
+  }
   KScope k(K_DEQUANT, st);
-  return cuda_status(launch_nf4_dequantize(w0.codes, w0.absmax, w0.n_out * w0.k_in, dst0, w1 ? w1->codes : nullptr,
-                                           w1 ? w1->absmax : nullptr, w1 ? w1->n_out * w1->k_in : 0, dst1, st,
-                                           num_sms()));
+  return cuda_status(launch_nf4_dequantize(codes, absmax, numel, out, n, st, num_sms()));
 }
 // Output maps of the staged configuration's TMA-store epilogue: bf16 [rows, cols]
 // with row stride ld, written in 32 x 32 boxes (64B swizzle).  No-ops otherwise.
@@ -663,8 +675,9 @@ qlora_status nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t n
   if (misaligned(codes) || misaligned(absmax) || misaligned(out)) return QLORA_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   KScope k(K_DEQUANT, st);
-  return cuda_status(launch_nf4_dequantize(codes, absmax, n_out * k_in, reinterpret_cast<bf16*>(out), nullptr, nullptr,
-                                           0, nullptr, st, num_sms()));
+  const int64_t numel = n_out * k_in;
+  bf16* dst = reinterpret_cast<bf16*>(out);
+  return cuda_status(launch_nf4_dequantize(&codes, &absmax, &numel, &dst, 1, st, num_sms()));
 }
 
 namespace {
@@ -1093,12 +1106,11 @@ qlora_status check_qkv(const Lin* q, const Lin* k, const Lin* v) {
   if (q->w.n_out + k->w.n_out + v->w.n_out > kMaxDim) return QLORA_ERR_UNSUPPORTED_SHAPE;
   return QLORA_OK;
 }
-// the three weights dequantised into consecutive rows of one [nq + nk + nv, K] buffer
+// the three weights dequantised (one launch) into consecutive rows of one [nq + nk + nv, K] buffer
 qlora_status stage_qkv(const Lin* q, const Lin* k, const Lin* v, bf16* stage, cudaStream_t st) {
   const int64_t K = q->w.k_in;
-  qlora_status s = stage_weights(q->w, stage, &k->w, stage + q->w.n_out * K, st);
-  if (s != QLORA_OK) return s;
-  return stage_weights(v->w, stage + (q->w.n_out + k->w.n_out) * K, nullptr, nullptr, st);
+  return stage_weights(q->w, stage, &k->w, stage + q->w.n_out * K, st, &v->w,
+                       stage + (q->w.n_out + k->w.n_out) * K);
 }
 }  // namespace
 

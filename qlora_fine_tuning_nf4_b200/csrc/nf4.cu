@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const bf16* __restric
   if (part == 0) absmax[blk] = m;
 }
 
-// Dequantisation of up to two tensors in one launch.  A warp takes runs of
+// Dequantisation of up to three tensors in one launch.  A warp takes runs of
 // 1024 elements: lane l expands the 8 elements at 8l + 256i (i = 0..3), so
 // each warp-wide load of codes is 128 contiguous bytes and each bf16 store
 // 512 contiguous bytes.  The 16 levels sit in shared memory (lanes reading
@@ -99,7 +99,7 @@ struct DqJob {
   int64_t runs;  // numel / 1024, rounded up
   int64_t numel;
 };
-__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, const DqJob j1) {
+__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, const DqJob j1, const DqJob j2) {
   __shared__ float lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = __uint_as_float(c_nf4_bits[threadIdx.x]);
   __syncthreads();
@@ -107,14 +107,14 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const DqJob j0, con
   grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t total = j0.runs + j1.runs;
+  const int64_t r01 = j0.runs + j1.runs, total = r01 + j2.runs;
   for (int64_t run = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; run < total; run += warps) {
-    const bool second = run >= j0.runs;
-    const int64_t base = (second ? run - j0.runs : run) * 1024;
-    const uint8_t* codes = second ? j1.codes : j0.codes;
-    const float* absmax = second ? j1.absmax : j0.absmax;
-    bf16* out = second ? j1.out : j0.out;
-    const int64_t numel = second ? j1.numel : j0.numel;
+    const int which = run < j0.runs ? 0 : (run < r01 ? 1 : 2);
+    const int64_t base = (run - (which == 0 ? 0 : (which == 1 ? j0.runs : r01))) * 1024;
+    const uint8_t* codes = which == 0 ? j0.codes : (which == 1 ? j1.codes : j2.codes);
+    const float* absmax = which == 0 ? j0.absmax : (which == 1 ? j1.absmax : j2.absmax);
+    bf16* out = which == 0 ? j0.out : (which == 1 ? j1.out : j2.out);
+    const int64_t numel = which == 0 ? j0.numel : (which == 1 ? j1.numel : j2.numel);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t e = base + i * 256 + lane * 8;
@@ -140,18 +140,19 @@ cudaError_t launch_nf4_quantize(const bf16* w, int64_t numel, uint8_t* codes, fl
                     absmax);
 }
 
-// Dequantises one tensor, or two (codes1 != nullptr) in the same launch.
-cudaError_t launch_nf4_dequantize(const uint8_t* codes0, const float* absmax0, int64_t numel0, bf16* out0,
-                                  const uint8_t* codes1, const float* absmax1, int64_t numel1, bf16* out1,
-                                  cudaStream_t st, int num_sms) {
-  DqJob j0 = {codes0, absmax0, out0, (numel0 + 1023) / 1024, numel0};
-  DqJob j1 = {codes1, absmax1, out1, codes1 ? (numel1 + 1023) / 1024 : 0, codes1 ? numel1 : 0};
-  int64_t grid = (j0.runs + j1.runs + 7) / 8;             // one run per warp, 8 warps per CTA
+// Dequantises n = 1 to 3 tensors in one launch: tensor i has numel[i] elements,
+// its codes and absmax, and goes to out[i].
+cudaError_t launch_nf4_dequantize(const uint8_t* const* codes, const float* const* absmax, const int64_t* numel,
+                                  bf16* const* out, int n, cudaStream_t st, int num_sms) {
+  if (n < 1 || n > 3) return cudaErrorInvalidValue;
+  DqJob j[3] = {};
+  for (int i = 0; i < n; ++i) j[i] = {codes[i], absmax[i], out[i], (numel[i] + 1023) / 1024, numel[i]};
+  int64_t grid = (j[0].runs + j[1].runs + j[2].runs + 7) / 8;  // one run per warp, 8 warps per CTA
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 CTAs of 256 threads per SM
   if (grid > cap) grid = cap;
   grid = apply_grid_cap(static_cast<int>(grid), 1);
   if (grid < 1) grid = 1;
-  return launch_pdl(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, j0, j1);
+  return launch_pdl(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, j[0], j[1], j[2]);
 }
 
 }  // namespace ql
