@@ -178,6 +178,17 @@ def checked_lib():
     return _check_lib
 
 
+_normal_lib = None
+
+
+def normal_lib():
+    """Load the normal build, libqlora.so, whatever QLORA_LIBRARY selects."""
+    global _normal_lib
+    if _normal_lib is None:
+        _normal_lib = _load(LIB_PATH)
+    return _normal_lib
+
+
 class use_library:
     """Context manager that routes every wrapper of this module to another
     build of the library (e.g. checked_lib()) and restores the previous one."""

@@ -29,7 +29,7 @@ def _lin(p):
 
 def test_checked_build_computes_what_the_oracle_computes():
     L = ops.checked_lib()
-    assert L.qlora_checked_build() == 1 and ops.lib().qlora_checked_build() == 0
+    assert L.qlora_checked_build() == 1 and ops.normal_lib().qlora_checked_build() == 0
     p = make_linear_problem(300, 768, 520, r=16, alpha=32.0, seed=21)
     with ops.use_library(L):
         g = run_linear_gpu(p, 4)
@@ -69,5 +69,10 @@ def test_checked_build_reports_a_plan_mismatch_without_trapping():
 
 def test_normal_build_does_not_check():
     p = make_linear_problem(256, 4096, 256, r=16, alpha=16.0, seed=22)
-    st, st_next, _, _ = _forward_with_shrunk_plan(p)
+    with ops.use_library(ops.normal_lib()):  # also when QLORA_LIBRARY=checked runs the suite on the checked build
+        prev = ops.qlora_set_tile_config(4)
+        try:
+            st, st_next, _, _ = _forward_with_shrunk_plan(p)
+        finally:
+            ops.qlora_set_tile_config(prev)
     assert st == 0 and st_next == 0
