@@ -158,11 +158,13 @@ class ClockSampler:
 
     def start(self):
         # samples go to a file, not a pipe: nothing reads them until stop(), and a full
-        # pipe would stall nvidia-smi (and drop the later samples) in a long run
+        # pipe would stall nvidia-smi (and drop the later samples) in a long run.  Every 20 ms,
+        # so that a 20-step window (about 75 ms) holds a few samples (the driver refreshes the
+        # clock and power readings about every 100 ms, so neighbouring samples may repeat).
         try:
             self.out = tempfile.TemporaryFile(mode="w+")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                          "-lms", "50", "-i", str(self.dev)], stdout=self.out,
+                                          "-lms", "20", "-i", str(self.dev)], stdout=self.out,
                                          stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
